@@ -1,0 +1,393 @@
+#!/usr/bin/env python3
+"""Benchmark of the fused Q4_K dequant + GEMV hot path on B200.
+
+One step = one q4k_gemv call (+ argmax epilogue) over the Q4_K LM-head
+workload (N = 248320 vocab rows x K = 4096, batch 1, ~572 MB of blocks; seed
+4; x ~ N(0,1)/64): block streaming, header decode, scale/min and quant unpack,
+dequant-MAC, reduction, logits + argmax.  The matrix is larger than the 126 MB
+L2, so no flush is needed between steps.
+
+Metric: effective HBM GB/s = (weight bytes + activation bytes) / time.
+  value  - device time of K steps (CUDA events, inputs resident in HBM), max over ranks
+  e2e    - the same metric through the same C-ABI call, with each step's x copied
+           host->device from pinned memory and its logits + argmax copied back
+           (weights stay resident, as a decode loop keeps them)
+  roofline - dominant kernel (q4k_gemv_kernel) timed alone with CUDA events on its
+           stream, against the measured HBM copy bandwidth in MEASURED_PEAKS.json
+  cpu_baseline - the CPU oracle timed on this host (rank 0, N = 1)
+
+--impl reference times the CPU oracle itself (there is no other implementation
+of this path to install): each step is a bounded row sample of the workload.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own independent
+problem (rows do not interact; no collective on the data path); value is the
+total bytes of all ranks over the max-over-ranks time ("scaling": "weak").
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "dequant-GEMV effective HBM GB/s and % of B200 peak (Q4_K, batch 1)"
+UNIT = "GB/s"
+WORKLOAD = "q4k_lmhead_248320x4096"
+FALLBACK_HBM_GBS = 6650.0
+
+# DRAM bytes (read + write) per launch of q4k_gemv_kernel on this workload, from
+# one ncu capture, valid only for the kernel sources whose hash is recorded.
+NCU_TRAFFIC = {"sources_sha1": None, "bytes_per_launch": None}
+
+
+def kernel_sources_sha1() -> str:
+    h = hashlib.sha1()
+    for f in ("q4k_gemv.cu", "q4k_decode.cuh", "dq_common.cuh"):
+        with open(os.path.join(ROOT, "dequant_gemv_q4_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="approximate CPU budget of the oracle baseline")
+    return ap.parse_args()
+
+
+def algorithmic_bytes(wl, B=1):
+    from dequant_gemv_q4_b200 import synth
+    per_block = synth.Q4K_BLOCK_BYTES if wl.fmt == "q4k" else synth.Q8_0_BLOCK_BYTES
+    elems = synth.Q4K_BLOCK_ELEMS if wl.fmt == "q4k" else synth.Q8_0_BLOCK_ELEMS
+    nmat = 2 if wl.op == "swiglu" else 1
+    return nmat * wl.N * (wl.K // elems) * per_block + 4 * B * wl.K
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML in a thread."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            self._ok = False
+
+    def _poll(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(0.002)
+
+    def _sample(self):
+        try:
+            self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+            self.reasons |= int(self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+        except Exception:
+            pass
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._poll, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._ok:
+            self._stop.set()
+            self._t.join()
+            self._sample()
+
+    def summary(self):
+        if not self._ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+def cpu_baseline(wl, inp, budget_s):
+    """Time the CPU oracle (single thread, as it stands) on a bounded row sample."""
+    import oracle
+    from dequant_gemv_q4_b200 import synth
+    # ~90 M weights/s per thread: size the sample to the budget
+    weights_per_row = wl.K * (2 if wl.op == "swiglu" else 1)
+    rows = int(max(64, min(wl.N, budget_s * 9.0e7 / weights_per_row)))
+    sel = np.arange(rows, dtype=np.int64)
+    t = time.perf_counter()
+    if wl.op == "swiglu":
+        g, _ = oracle.q4k_gemv(inp["w_gate"], wl.N, wl.K, inp["x"], rows=sel)
+        u, _ = oracle.q4k_gemv(inp["w_up"], wl.N, wl.K, inp["x"], rows=sel)
+        oracle.swiglu(g, u)
+    elif wl.fmt == "q4k":
+        y, _ = oracle.q4k_gemv(inp["w"], wl.N, wl.K, inp["x"], rows=sel)
+        if wl.op == "gemv_argmax":
+            oracle.argmax(y[0])
+    else:
+        oracle.q8_0_gemv(inp["w"], wl.N, wl.K, inp["x"], rows=sel)
+    dt = time.perf_counter() - t
+    per_block = synth.Q4K_BLOCK_BYTES if wl.fmt == "q4k" else synth.Q8_0_BLOCK_BYTES
+    elems = synth.Q4K_BLOCK_ELEMS if wl.fmt == "q4k" else synth.Q8_0_BLOCK_ELEMS
+    nbytes = (2 if wl.op == "swiglu" else 1) * rows * (wl.K // elems) * per_block + 4 * wl.K
+    return {"value": nbytes / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": "%d of %d rows (%.3g weights), single thread, %.1f s" % (rows, wl.N, rows * weights_per_row, dt)}
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the CPU oracle on host cores, rank 0 only."""
+    if rank != 0:
+        return
+    from dequant_gemv_q4_b200 import synth
+    import oracle
+    wl = synth.WORKLOADS[args.workload]
+    inp = synth.make_inputs(wl)
+    # each step: a bounded sample of rows so that warmup + steps stay within minutes
+    weights_per_row = wl.K * (2 if wl.op == "swiglu" else 1)
+    per_step_s = min(2.0, 150.0 / max(1, args.steps + args.warmup))
+    rows = int(max(16, min(wl.N, per_step_s * 9.0e7 / weights_per_row)))
+    elems = synth.Q4K_BLOCK_ELEMS if wl.fmt == "q4k" else synth.Q8_0_BLOCK_ELEMS
+    per_block = synth.Q4K_BLOCK_BYTES if wl.fmt == "q4k" else synth.Q8_0_BLOCK_BYTES
+    nbytes = (2 if wl.op == "swiglu" else 1) * rows * (wl.K // elems) * per_block + 4 * wl.K
+
+    def step(i):
+        start = (i * rows) % max(1, wl.N - rows + 1)
+        sel = np.arange(start, start + rows, dtype=np.int64)
+        if wl.op == "swiglu":
+            g, _ = oracle.q4k_gemv(inp["w_gate"], wl.N, wl.K, inp["x"], rows=sel)
+            u, _ = oracle.q4k_gemv(inp["w_up"], wl.N, wl.K, inp["x"], rows=sel)
+            oracle.swiglu(g, u)
+        elif wl.fmt == "q4k":
+            y, _ = oracle.q4k_gemv(inp["w"], wl.N, wl.K, inp["x"], rows=sel)
+            if wl.op == "gemv_argmax":
+                oracle.argmax(y[0])
+        else:
+            oracle.q8_0_gemv(inp["w"], wl.N, wl.K, inp["x"], rows=sel)
+
+    for i in range(args.warmup):
+        step(i)
+    t = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    dt = (time.perf_counter() - t) / max(1, args.steps)
+    value = nbytes / dt / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "N": wl.N, "K": wl.K, "B": 1, "format": "Q4_K" if wl.fmt == "q4k" else "Q8_0",
+                   "sample_rows_per_step": rows},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": "%d consecutive rows per step of %d, single thread" % (rows, wl.N)},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import dequant_gemv_q4_b200 as dq
+    from dequant_gemv_q4_b200 import synth
+
+    torch.cuda.set_device(local_rank)
+    dist_on = world > 1
+    if dist_on:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+
+    wl = synth.WORKLOADS[args.workload]
+    B = 1
+    if wl.seed is not None and dist_on:
+        wl = synth.Workload(wl.name, wl.fmt, wl.op, wl.N, wl.K, wl.batches, wl.seed + 1000 * rank,
+                            wl.x_scale)
+    inp = synth.make_inputs(wl, B=B)
+    dev = torch.device("cuda", local_rank)
+    argmax = wl.op == "gemv_argmax"
+    if wl.op == "swiglu":
+        wg = torch.from_numpy(inp["w_gate"]).to(dev)
+        wu = torch.from_numpy(inp["w_up"]).to(dev)
+        op = dq.DQ_OP_Q4K_SWIGLU
+    else:
+        w = torch.from_numpy(inp["w"]).to(dev)
+        op = dq.DQ_OP_Q4K_GEMV if wl.fmt == "q4k" else dq.DQ_OP_Q8_0_GEMV
+    x = torch.from_numpy(inp["x"]).to(dev)
+    y = torch.empty((B, wl.N), dtype=torch.float32, device=dev)
+    ws_bytes = dq.dq_workspace_bytes(op, wl.N, wl.K, B, argmax)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    split = dq.dq_workspace_bytes(op, wl.N, wl.K, B, False) > 0
+    launches_per_step = 1 + (1 if split else 0) + (1 if argmax else 0)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(xin, yout, with_argmax=argmax):
+        if wl.op == "swiglu":
+            dq.q4k_swiglu_gemv(wg, wu, xin, wl.N, wl.K, out=yout, workspace=ws)
+            return None
+        if wl.fmt == "q4k":
+            r = dq.q4k_gemv(w, xin, wl.N, wl.K, y=yout, argmax=with_argmax, workspace=ws)
+            return r[1] if with_argmax else None
+        dq.q8_0_gemv(w, xin, wl.N, wl.K, y=yout, workspace=ws)
+        return None
+
+    def barrier():
+        if dist_on:
+            dist.barrier(device_ids=[local_rank])
+        torch.cuda.synchronize(dev)
+
+    def max_over_ranks(v):
+        if not dist_on:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    nbytes = algorithmic_bytes(wl, B)
+
+    # ---- device-resident steps (the headline value) ----
+    for _ in range(max(3, args.warmup)):
+        step(x, y)
+    barrier()
+    sampler = ClockSampler(local_rank)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with sampler:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step(x, y)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    value = nbytes * world / (ms * 1e-3) / 1e9
+
+    # ---- dominant kernel alone (one launch per call, no epilogue kernels) ----
+    if not split:
+        for _ in range(3):
+            step(x, y, with_argmax=False)
+        torch.cuda.synchronize(dev)
+        k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        k0.record(stream)
+        for _ in range(args.steps):
+            step(x, y, with_argmax=False)
+        k1.record(stream)
+        torch.cuda.synchronize(dev)
+        kms = k0.elapsed_time(k1) / args.steps
+    else:
+        kms = ms
+    barrier()
+
+    # ---- end to end: host x in, host logits + argmax out ----
+    x_host = torch.from_numpy(inp["x"]).pin_memory()
+    y_host = torch.empty((B, wl.N), dtype=torch.float32).pin_memory()
+    i_host = torch.empty(1, dtype=torch.int64).pin_memory()
+    x_dev = torch.empty_like(x)
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        idx = step(x_dev, y)
+        y_host.copy_(y, non_blocking=True)
+        if idx is not None:
+            i_host.copy_(idx, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    barrier()
+    h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    h1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = max_over_ranks(h0.elapsed_time(h1) / args.steps)
+    e2e_value = nbytes * world / (e2e_ms * 1e-3) / 1e9
+    h2d = x_host.numel() * 4
+    d2h = y_host.numel() * 4 + (8 if argmax else 0)
+
+    peak, peak_kind = measured_peak()
+    achieved = nbytes / (kms * 1e-3) / 1e9
+    traffic = None
+    if NCU_TRAFFIC["sources_sha1"] == kernel_sources_sha1() and wl.name == WORKLOAD:
+        traffic = NCU_TRAFFIC["bytes_per_launch"]
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": wl.name, "N": wl.N, "K": wl.K, "B": B,
+                   "format": "Q4_K" if wl.fmt == "q4k" else "Q8_0", "layout": "aos",
+                   "epilogue": "argmax" if argmax else ("swiglu" if wl.op == "swiglu" else "none"),
+                   "bytes_per_step": nbytes,
+                   "l2": "weights %.0f MB > 126 MB L2; no flush" % (nbytes / 1e6) if nbytes > 126e6
+                   else "weights fit in L2: NOT flushed (value is L2-assisted)",
+                   "parallelism": "replicas x%d (independent problems, no collective)" % world},
+        "pct_of_peak_hbm": 100.0 * value / world / peak,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
+                     "traffic": traffic, "kernel": "q4k_gemv_kernel", "kernel_ms": kms,
+                     "peak_kind": peak_kind + " (MEASURED_PEAKS.json hbm_gbs, burst)" if peak_kind == "measured"
+                     else "fallback"},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms, "note": "weights resident; x in, logits+argmax out per step"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": sampler.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, inp, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist_on:
+        dist.barrier(device_ids=[local_rank])
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

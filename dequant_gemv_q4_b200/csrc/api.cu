@@ -1,0 +1,320 @@
+// api.cu -- the C ABI of libdqgemv (declared and documented in dqgemv.h):
+// argument validation, launch planning, workspace carving and kernel launch.
+// Nothing here allocates device memory; every pointer comes from the caller.
+#include <cstdint>
+#include <cstring>
+#include <cuda_runtime.h>
+
+#include "dq_common.cuh"
+#include "dq_internal.h"
+#include "dqgemv.h"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+dq_status cuda_fail(cudaError_t e)
+{
+    g_last_cuda_error = static_cast<int>(e);
+    return DQ_ERR_CUDA;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+struct DevInfo {
+    int device;
+    int sm_count;
+    int smem_optin;
+};
+
+dq_status dev_info(DevInfo &di)
+{
+    static int cached_sm[64] = {};
+    static int cached_smem[64] = {};
+    cudaError_t e = cudaGetDevice(&di.device);
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    if (di.device >= 0 && di.device < 64 && cached_sm[di.device] > 0) {
+        di.sm_count = cached_sm[di.device];
+        di.smem_optin = cached_smem[di.device];
+        return DQ_OK;
+    }
+    e = cudaDeviceGetAttribute(&di.sm_count, cudaDevAttrMultiProcessorCount, di.device);
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    e = cudaDeviceGetAttribute(&di.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, di.device);
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    if (di.device >= 0 && di.device < 64) {
+        cached_sm[di.device] = di.sm_count;
+        cached_smem[di.device] = di.smem_optin;
+    }
+    return DQ_OK;
+}
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Workspace layout of the Q4_K GEMV for a plan: [split partials][argmax candidates].
+struct Q4KWorkspace {
+    size_t part_bytes;
+    size_t cand_bytes;
+    int ncand;
+    size_t total() const { return part_bytes + cand_bytes; }
+};
+
+Q4KWorkspace q4k_ws(const dq::Q4KPlan &pl, long long N, int B, int NS, bool argmax)
+{
+    Q4KWorkspace ws{};
+    if (pl.splits > 1)
+        ws.part_bytes = round_up(static_cast<size_t>(pl.splits) * NS * B * N * sizeof(float), 256);
+    if (argmax) {
+        ws.ncand = (pl.splits > 1) ? dq::reduce_grid(N, B) : pl.grid;
+        ws.cand_bytes = round_up(static_cast<size_t>(ws.ncand) * sizeof(dq::ArgmaxCand), 256);
+    }
+    return ws;
+}
+
+dq_status check_q4k_shape(int64_t N, int64_t K, int B)
+{
+    if (N < 1 || K < 256 || K % 256 != 0 || K > DQ_MAX_K || B < 1 || B > 8)
+        return DQ_ERR_SHAPE;
+    return DQ_OK;
+}
+
+dq_status q4k_common(const void *w0, const void *w1, int layout, const float *x, float *y, int64_t N, int64_t K,
+                     int B, int NS, int64_t *argmax_out, void *workspace, size_t ws_bytes, void *stream)
+{
+    if (!w0 || (NS == 2 && !w1) || !x || !y)
+        return DQ_ERR_NULL;
+    if (layout != DQ_LAYOUT_AOS && layout != DQ_LAYOUT_SOA)
+        return DQ_ERR_LAYOUT;
+    dq_status st = check_q4k_shape(N, K, B);
+    if (st != DQ_OK)
+        return st;
+    if (argmax_out && (B != 1 || NS != 1))
+        return DQ_ERR_ARG;
+    if (!aligned(w0, 16) || (w1 && !aligned(w1, 16)) || !aligned(x, 16) || !aligned(y, 4) ||
+        (argmax_out && !aligned(argmax_out, 8)))
+        return DQ_ERR_ALIGN;
+    DevInfo di;
+    st = dev_info(di);
+    if (st != DQ_OK)
+        return st;
+    const dq::Q4KPlan pl = dq::q4k_plan(N, static_cast<int>(K), B, NS, layout == DQ_LAYOUT_SOA, di.sm_count,
+                                        di.smem_optin);
+    if (!pl.ok)
+        return DQ_ERR_SHAPE;
+    const Q4KWorkspace ws = q4k_ws(pl, N, B, NS, argmax_out != nullptr);
+    if (ws.total() > 0 && (!workspace || ws_bytes < ws.total()))
+        return DQ_ERR_WORKSPACE;
+    if (ws.total() > 0 && !aligned(workspace, 16))
+        return DQ_ERR_ALIGN;
+
+    uint8_t *wsb = static_cast<uint8_t *>(workspace);
+    dq::Q4KParams p{};
+    p.w[0] = static_cast<const uint8_t *>(w0);
+    p.w[1] = static_cast<const uint8_t *>(NS == 2 ? w1 : w0);
+    p.x = x;
+    p.y = y;
+    p.part = pl.splits > 1 ? reinterpret_cast<float *>(wsb) : nullptr;
+    p.cand = argmax_out ? reinterpret_cast<dq::ArgmaxCand *>(wsb + ws.part_bytes) : nullptr;
+    p.err = dq::device_error_flag(di.device);
+    p.N = N;
+    p.K = static_cast<int>(K);
+    p.nb = static_cast<int>(K / 256);
+    p.splits = pl.splits;
+    p.chunks_per_split = pl.chunks_per_split;
+    p.ctas_per_split = pl.ctas_per_split;
+    p.depth = pl.depth;
+    p.soa = layout == DQ_LAYOUT_SOA;
+    p.argmax = argmax_out != nullptr;
+    p.tiles = pl.tiles;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = dq::q4k_gemv_launch(p, pl, B, NS, s);
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    if (pl.splits > 1) {
+        e = dq::splitk_reduce_launch(p.part, pl.splits, NS, B, N, y, p.cand, dq::reduce_grid(N, B), s);
+        if (e != cudaSuccess)
+            return cuda_fail(e);
+    }
+    if (argmax_out) {
+        e = dq::argmax_finalize_launch(p.cand, ws.ncand, reinterpret_cast<long long *>(argmax_out), s);
+        if (e != cudaSuccess)
+            return cuda_fail(e);
+    }
+    return DQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+dq_status q4k_gemv(const void *w, int layout, const float *x, float *y, int64_t N, int64_t K, int B,
+                   int64_t *argmax_out, void *workspace, size_t ws_bytes, void *stream)
+{
+    return q4k_common(w, nullptr, layout, x, y, N, K, B, 1, argmax_out, workspace, ws_bytes, stream);
+}
+
+dq_status q4k_swiglu_gemv(const void *w_gate, const void *w_up, int layout, const float *x, float *out, int64_t N,
+                          int64_t K, int B, void *workspace, size_t ws_bytes, void *stream)
+{
+    if (!w_up)
+        return DQ_ERR_NULL;
+    return q4k_common(w_gate, w_up, layout, x, out, N, K, B, 2, nullptr, workspace, ws_bytes, stream);
+}
+
+dq_status q8_0_gemv(const void *w, const float *x, float *y, int64_t N, int64_t K, int B, void *workspace,
+                    size_t ws_bytes, void *stream)
+{
+    (void)workspace;
+    (void)ws_bytes;
+    if (!w || !x || !y)
+        return DQ_ERR_NULL;
+    if (N < 1 || K < 32 || K % 32 != 0 || K > DQ_MAX_K || B < 1 || B > 8)
+        return DQ_ERR_SHAPE;
+    if (!aligned(w, 16) || !aligned(x, 16) || !aligned(y, 4))
+        return DQ_ERR_ALIGN;
+    DevInfo di;
+    dq_status st = dev_info(di);
+    if (st != DQ_OK)
+        return st;
+    const dq::Q8Plan pl = dq::q8_plan(N, static_cast<int>(K), B, di.sm_count, di.smem_optin);
+    if (!pl.ok)
+        return DQ_ERR_SHAPE;
+    dq::Q8Params p{};
+    p.w = static_cast<const uint8_t *>(w);
+    p.x = x;
+    p.y = y;
+    p.err = dq::device_error_flag(di.device);
+    p.N = N;
+    p.K = static_cast<int>(K);
+    p.nb = static_cast<int>(K / 32);
+    cudaError_t e = dq::q8_0_gemv_launch(p, pl, B, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DQ_OK : cuda_fail(e);
+}
+
+dq_status q4k_repack_soa(const void *w_aos, void *w_soa, int64_t N, int64_t K, void *stream)
+{
+    if (!w_aos || !w_soa)
+        return DQ_ERR_NULL;
+    if (N < 1 || K < 256 || K % 256 != 0 || K > DQ_MAX_K)
+        return DQ_ERR_SHAPE;
+    if (!aligned(w_aos, 16) || !aligned(w_soa, 16))
+        return DQ_ERR_ALIGN;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(w_aos), b0 = reinterpret_cast<uintptr_t>(w_soa);
+    const uintptr_t bytes = static_cast<uintptr_t>(N) * static_cast<uintptr_t>(K / 256) * 144u;
+    if (a0 < b0 + bytes && b0 < a0 + bytes)
+        return DQ_ERR_ARG;
+    cudaError_t e = dq::q4k_repack_soa_launch(static_cast<const uint8_t *>(w_aos), static_cast<uint8_t *>(w_soa), N,
+                                              static_cast<int>(K), static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DQ_OK : cuda_fail(e);
+}
+
+size_t dq_workspace_bytes(int op, int64_t N, int64_t K, int B, int with_argmax)
+{
+    const size_t bad = static_cast<size_t>(-1);
+    if (op == DQ_OP_Q8_0_GEMV) {
+        if (N < 1 || K < 32 || K % 32 != 0 || K > DQ_MAX_K || B < 1 || B > 8 || with_argmax)
+            return bad;
+        return 0;
+    }
+    if (op != DQ_OP_Q4K_GEMV && op != DQ_OP_Q4K_SWIGLU)
+        return bad;
+    if (check_q4k_shape(N, K, B) != DQ_OK)
+        return bad;
+    const int NS = (op == DQ_OP_Q4K_SWIGLU) ? 2 : 1;
+    if (with_argmax && (B != 1 || NS != 1))
+        return bad;
+    DevInfo di;
+    if (dev_info(di) != DQ_OK)
+        return bad;
+    // the plan does not depend on the layout except through the chunk width,
+    // so take the larger of the two requirements
+    size_t need = 0;
+    for (int soa = 0; soa < 2; ++soa) {
+        const dq::Q4KPlan pl = dq::q4k_plan(N, static_cast<int>(K), B, NS, soa, di.sm_count, di.smem_optin);
+        if (!pl.ok)
+            return bad;
+        const size_t t = q4k_ws(pl, N, B, NS, with_argmax != 0).total();
+        if (t > need)
+            need = t;
+    }
+    return need;
+}
+
+dq_status q8_0_dequant(const void *w, float *out, int64_t N, int64_t K, void *stream)
+{
+    if (!w || !out)
+        return DQ_ERR_NULL;
+    if (N < 1 || K < 32 || K % 32 != 0 || K > DQ_MAX_K)
+        return DQ_ERR_SHAPE;
+    if (!aligned(w, 2) || !aligned(out, 4))
+        return DQ_ERR_ALIGN;
+    cudaError_t e = dq::q8_0_dequant_launch(static_cast<const uint8_t *>(w), out, N, static_cast<int>(K),
+                                            static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DQ_OK : cuda_fail(e);
+}
+
+dq_status q4k_dequant(const void *w, int layout, float *out, int64_t N, int64_t K, void *stream)
+{
+    if (!w || !out)
+        return DQ_ERR_NULL;
+    if (layout != DQ_LAYOUT_AOS && layout != DQ_LAYOUT_SOA)
+        return DQ_ERR_LAYOUT;
+    if (N < 1 || K < 256 || K % 256 != 0 || K > DQ_MAX_K)
+        return DQ_ERR_SHAPE;
+    if (!aligned(w, 16) || !aligned(out, 4))
+        return DQ_ERR_ALIGN;
+    cudaError_t e = dq::q4k_dequant_launch(static_cast<const uint8_t *>(w), layout == DQ_LAYOUT_SOA, out, N,
+                                           static_cast<int>(K), static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DQ_OK : cuda_fail(e);
+}
+
+const char *dq_status_string(int status)
+{
+    switch (status) {
+    case DQ_OK: return "DQ_OK";
+    case DQ_ERR_NULL: return "DQ_ERR_NULL: a required pointer is NULL";
+    case DQ_ERR_SHAPE: return "DQ_ERR_SHAPE: N, K or B outside the supported range";
+    case DQ_ERR_ALIGN: return "DQ_ERR_ALIGN: a pointer is not suitably aligned";
+    case DQ_ERR_WORKSPACE: return "DQ_ERR_WORKSPACE: workspace missing or too small";
+    case DQ_ERR_LAYOUT: return "DQ_ERR_LAYOUT: unknown weight layout";
+    case DQ_ERR_CUDA: return "DQ_ERR_CUDA: a CUDA runtime call failed";
+    case DQ_ERR_ARG: return "DQ_ERR_ARG: invalid argument combination";
+    default: return "unknown dq_status";
+    }
+}
+
+int dq_last_cuda_error(void) { return g_last_cuda_error; }
+
+dq_status dq_device_error(int *flag, int clear, void *stream)
+{
+    if (!flag)
+        return DQ_ERR_NULL;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    int *d = dq::device_error_flag(dev);
+    if (!d)
+        return cuda_fail(cudaErrorInvalidSymbol);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    e = cudaMemcpy(flag, d, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    if (clear) {
+        e = cudaMemset(d, 0, sizeof(int));
+        if (e != cudaSuccess)
+            return cuda_fail(e);
+        e = cudaDeviceSynchronize();
+        if (e != cudaSuccess)
+            return cuda_fail(e);
+    }
+    return DQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,324 @@
+// aux_kernels.cu -- debug dequantization, the SoA repack, the split-K
+// reduction (with the SwiGLU epilogue and argmax candidates) and the argmax
+// finalisation, plus the per-device error flag.
+#include <cuda_fp16.h>
+#include <cstdint>
+
+#include "dq_common.cuh"
+#include "dq_internal.h"
+#include "q4k_decode.cuh"
+#include "q8_decode.cuh"
+
+namespace dq {
+
+// Set by kernels whose bounded waits gave up (see dq_device_error in dqgemv.h).
+__device__ int g_dq_error_flag;
+
+int *device_error_flag(int device)
+{
+    static int *addr[64] = {};
+    if (device < 0 || device >= 64)
+        return nullptr;
+    if (!addr[device]) {
+        void *a = nullptr;
+        if (cudaGetSymbolAddress(&a, g_dq_error_flag) != cudaSuccess)
+            return nullptr;
+        addr[device] = static_cast<int *>(a);
+    }
+    return addr[device];
+}
+
+// ---------------------------------------------------------------------------
+// Q4_K debug dequant: one thread per (row, super-block, 16-byte quant slice)
+// writes that slice's 32 weights with the GEMV's own weight formation.
+// ---------------------------------------------------------------------------
+
+// Byte offset within a row of the header (byte < 16) or of quant slice s of
+// super-block kb in the SoA layout (groups of 16 super-blocks; see dqgemv.h).
+__device__ __forceinline__ long long soa_hdr_off(int nb, int kb)
+{
+    const int first = (kb / 16) * 16;
+    return static_cast<long long>(first) * kQ4KBlockBytes + 16 * (kb - first);
+}
+__device__ __forceinline__ long long soa_slice_off(int nb, int kb, int s)
+{
+    const int first = (kb / 16) * 16;
+    const int g = min(16, nb - first);
+    return static_cast<long long>(first) * kQ4KBlockBytes + 16 * g + 16 * g * s + 16 * (kb - first);
+}
+
+__global__ void q4k_dequant_kernel(const uint8_t *__restrict__ w, int soa, float *__restrict__ out,
+                                   long long N, int K)
+{
+    const int nb = K / kQ4KBlockElems;
+    const long long total = N * nb * 8;
+    const long long row_bytes = static_cast<long long>(nb) * kQ4KBlockBytes;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const int s = static_cast<int>(i % 8);
+        const long long blk = i / 8;
+        const int kb = static_cast<int>(blk % nb);
+        const long long n = blk / nb;
+        const uint8_t *row = w + n * row_bytes;
+        const uint8_t *hp = soa ? row + soa_hdr_off(nb, kb) : row + static_cast<long long>(kb) * kQ4KBlockBytes;
+        const uint8_t *qp = soa ? row + soa_slice_off(nb, kb, s)
+                                : row + static_cast<long long>(kb) * kQ4KBlockBytes + 16 + 16 * s;
+        const Hdr h = decode_hdr(*reinterpret_cast<const uint4 *>(hp));
+        const uint4 q = *reinterpret_cast<const uint4 *>(qp);
+        const int c = s / 2;
+        float2 sL, mL, sH, mH;
+        chunk_scales(h, c, sL, mL, sH, mH);
+        const long long L = n * K + static_cast<long long>(kb) * kQ4KBlockElems + 64 * c + 16 * (s % 2);
+        const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            float2 wv[4];
+            q4_word_weights(words[t], sL, mL, sH, mH, wv);
+            float4 lo = make_float4(wv[0].x * 0x1p64f, wv[0].y * 0x1p64f, wv[1].x * 0x1p64f, wv[1].y * 0x1p64f);
+            float4 hi = make_float4(wv[2].x * 0x1p64f, wv[2].y * 0x1p64f, wv[3].x * 0x1p64f, wv[3].y * 0x1p64f);
+            *reinterpret_cast<float4 *>(out + L + 4 * t) = lo;
+            *reinterpret_cast<float4 *>(out + L + 32 + 4 * t) = hi;
+        }
+    }
+}
+
+// out may be any 4-byte aligned pointer; the float4 stores above need 16-byte
+// alignment, so an unaligned `out` goes through this scalar variant.
+__global__ void q4k_dequant_kernel_scalar(const uint8_t *__restrict__ w, int soa, float *__restrict__ out,
+                                          long long N, int K)
+{
+    const int nb = K / kQ4KBlockElems;
+    const long long total = N * nb * 8;
+    const long long row_bytes = static_cast<long long>(nb) * kQ4KBlockBytes;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const int s = static_cast<int>(i % 8);
+        const long long blk = i / 8;
+        const int kb = static_cast<int>(blk % nb);
+        const long long n = blk / nb;
+        const uint8_t *row = w + n * row_bytes;
+        const uint8_t *hp = soa ? row + soa_hdr_off(nb, kb) : row + static_cast<long long>(kb) * kQ4KBlockBytes;
+        const uint8_t *qp = soa ? row + soa_slice_off(nb, kb, s)
+                                : row + static_cast<long long>(kb) * kQ4KBlockBytes + 16 + 16 * s;
+        const Hdr h = decode_hdr(*reinterpret_cast<const uint4 *>(hp));
+        const uint4 q = *reinterpret_cast<const uint4 *>(qp);
+        const int c = s / 2;
+        float2 sL, mL, sH, mH;
+        chunk_scales(h, c, sL, mL, sH, mH);
+        const long long L = n * K + static_cast<long long>(kb) * kQ4KBlockElems + 64 * c + 16 * (s % 2);
+        const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            float2 wv[4];
+            q4_word_weights(words[t], sL, mL, sH, mH, wv);
+            out[L + 4 * t + 0] = wv[0].x * 0x1p64f;
+            out[L + 4 * t + 1] = wv[0].y * 0x1p64f;
+            out[L + 4 * t + 2] = wv[1].x * 0x1p64f;
+            out[L + 4 * t + 3] = wv[1].y * 0x1p64f;
+            out[L + 32 + 4 * t + 0] = wv[2].x * 0x1p64f;
+            out[L + 32 + 4 * t + 1] = wv[2].y * 0x1p64f;
+            out[L + 32 + 4 * t + 2] = wv[3].x * 0x1p64f;
+            out[L + 32 + 4 * t + 3] = wv[3].y * 0x1p64f;
+        }
+    }
+}
+
+static int grid_for(long long work, int block)
+{
+    long long g = (work + block - 1) / block;
+    if (g > 65535LL * 16)
+        g = 65535LL * 16;
+    if (g < 1)
+        g = 1;
+    return static_cast<int>(g);
+}
+
+cudaError_t q4k_dequant_launch(const uint8_t *w, int soa, float *out, long long N, int K, cudaStream_t s)
+{
+    const long long total = N * (K / kQ4KBlockElems) * 8;
+    if ((reinterpret_cast<uintptr_t>(out) & 15) == 0)
+        q4k_dequant_kernel<<<grid_for(total, 256), 256, 0, s>>>(w, soa, out, N, K);
+    else
+        q4k_dequant_kernel_scalar<<<grid_for(total, 256), 256, 0, s>>>(w, soa, out, N, K);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Q8_0 debug dequant: one thread per block, the GEMV's weight formation.
+// ---------------------------------------------------------------------------
+__global__ void q8_0_dequant_kernel(const uint8_t *__restrict__ w, float *__restrict__ out, long long N, int K)
+{
+    const int nb = K / kQ8BlockElems;
+    const long long total = N * nb;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const uint8_t *blk = w + i * kQ8BlockBytes;  // blocks are contiguous over rows
+        const uint16_t *h = reinterpret_cast<const uint16_t *>(blk);
+        const float d = __half2float(__ushort_as_half(h[0]));
+        float2 s01, s23, off;
+        q8_scales(d, s01, s23, off);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const uint32_t wq = static_cast<uint32_t>(h[1 + 2 * j]) | (static_cast<uint32_t>(h[2 + 2 * j]) << 16);
+            float2 wv[2];
+            q8_word_weights(wq, s01, s23, off, wv);
+            float *o = out + i * kQ8BlockElems + 4 * j;
+            o[0] = wv[0].x * 0x1p64f;
+            o[1] = wv[0].y * 0x1p64f;
+            o[2] = wv[1].x * 0x1p64f;
+            o[3] = wv[1].y * 0x1p64f;
+        }
+    }
+}
+
+cudaError_t q8_0_dequant_launch(const uint8_t *w, float *out, long long N, int K, cudaStream_t s)
+{
+    const long long total = N * (K / kQ8BlockElems);
+    q8_0_dequant_kernel<<<grid_for(total, 256), 256, 0, s>>>(w, out, N, K);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// AoS -> SoA repack: one thread per (row, super-block, 16-byte piece).
+// Piece 0 is the header, pieces 1..8 the quant slices 0..7.
+// ---------------------------------------------------------------------------
+__global__ void q4k_repack_soa_kernel(const uint8_t *__restrict__ aos, uint8_t *__restrict__ soa, long long N,
+                                      int K)
+{
+    const int nb = K / kQ4KBlockElems;
+    const long long total = N * nb * 9;
+    const long long row_bytes = static_cast<long long>(nb) * kQ4KBlockBytes;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const int piece = static_cast<int>(i % 9);
+        const long long blk = i / 9;
+        const int kb = static_cast<int>(blk % nb);
+        const long long n = blk / nb;
+        const uint4 v = *reinterpret_cast<const uint4 *>(aos + n * row_bytes + static_cast<long long>(kb) * kQ4KBlockBytes +
+                                                         16 * piece);
+        const long long dst = n * row_bytes + (piece == 0 ? soa_hdr_off(nb, kb) : soa_slice_off(nb, kb, piece - 1));
+        *reinterpret_cast<uint4 *>(soa + dst) = v;
+    }
+}
+
+cudaError_t q4k_repack_soa_launch(const uint8_t *aos, uint8_t *soa, long long N, int K, cudaStream_t s)
+{
+    const long long total = N * (K / kQ4KBlockElems) * 9;
+    q4k_repack_soa_kernel<<<grid_for(total, 256), 256, 0, s>>>(aos, soa, N, K);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Split-K reduction: out = sum over splits in split order; SwiGLU epilogue when
+// NS == 2; per-CTA argmax candidates when cand != nullptr (B == 1).
+// ---------------------------------------------------------------------------
+constexpr int kReduceThreads = 256;
+
+int reduce_grid(long long N, int B)
+{
+    long long g = (N * B + kReduceThreads - 1) / kReduceThreads;
+    if (g > 1024)
+        g = 1024;
+    return static_cast<int>(g < 1 ? 1 : g);
+}
+
+__global__ void __launch_bounds__(kReduceThreads) splitk_reduce_kernel(const float *__restrict__ part, int splits,
+                                                                       int NS, int B, long long N,
+                                                                       float *__restrict__ y, ArgmaxCand *cand)
+{
+    float best_v = -INFINITY;
+    long long best_i = 0x7fffffffffffffffLL;
+    const long long total = N * B;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long n = i % N;
+        const int b = static_cast<int>(i / N);
+        float g = 0.f, u = 0.f;
+        for (int s = 0; s < splits; ++s) {
+            g += part[((static_cast<long long>(s) * NS + 0) * B + b) * N + n];
+            if (NS == 2)
+                u += part[((static_cast<long long>(s) * NS + 1) * B + b) * N + n];
+        }
+        const float out = (NS == 2) ? g / (1.0f + expf(-g)) * u : g;
+        y[i] = out;
+        if (cand && cand_better(out, n, best_v, best_i)) {
+            best_v = out;
+            best_i = n;
+        }
+    }
+    if (cand) {
+        __shared__ ArgmaxCand red[kReduceThreads / 32];
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, best_v, o);
+            const long long oi = __shfl_xor_sync(0xffffffffu, best_i, o);
+            if (cand_better(ov, oi, best_v, best_i)) {
+                best_v = ov;
+                best_i = oi;
+            }
+        }
+        if ((threadIdx.x & 31) == 0) {
+            red[threadIdx.x >> 5].v = best_v;
+            red[threadIdx.x >> 5].idx = best_i;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            ArgmaxCand c = red[0];
+            for (int w = 1; w < kReduceThreads / 32; ++w)
+                if (cand_better(red[w].v, red[w].idx, c.v, c.idx))
+                    c = red[w];
+            cand[blockIdx.x] = c;
+        }
+    }
+}
+
+cudaError_t splitk_reduce_launch(const float *part, int splits, int NS, int B, long long N, float *y,
+                                 ArgmaxCand *cand, int grid, cudaStream_t s)
+{
+    splitk_reduce_kernel<<<grid, kReduceThreads, 0, s>>>(part, splits, NS, B, N, y, cand);
+    return cudaGetLastError();
+}
+
+// One CTA folds all candidates into the final index.
+__global__ void __launch_bounds__(1024) argmax_finalize_kernel(const ArgmaxCand *__restrict__ cand, int ncand,
+                                                               long long *out)
+{
+    float best_v = -INFINITY;
+    long long best_i = 0x7fffffffffffffffLL;
+    for (int i = threadIdx.x; i < ncand; i += blockDim.x)
+        if (cand_better(cand[i].v, cand[i].idx, best_v, best_i)) {
+            best_v = cand[i].v;
+            best_i = cand[i].idx;
+        }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, best_v, o);
+        const long long oi = __shfl_xor_sync(0xffffffffu, best_i, o);
+        if (cand_better(ov, oi, best_v, best_i)) {
+            best_v = ov;
+            best_i = oi;
+        }
+    }
+    __shared__ ArgmaxCand red[32];
+    if ((threadIdx.x & 31) == 0) {
+        red[threadIdx.x >> 5].v = best_v;
+        red[threadIdx.x >> 5].idx = best_i;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        ArgmaxCand c = red[0];
+        for (int w = 1; w < static_cast<int>(blockDim.x >> 5); ++w)
+            if (cand_better(red[w].v, red[w].idx, c.v, c.idx))
+                c = red[w];
+        // every value NaN leaves no candidate: report -1
+        *out = (c.idx == 0x7fffffffffffffffLL) ? -1 : c.idx;
+    }
+}
+
+cudaError_t argmax_finalize_launch(const ArgmaxCand *cand, int ncand, long long *out, cudaStream_t s)
+{
+    argmax_finalize_kernel<<<1, 1024, 0, s>>>(cand, ncand, out);
+    return cudaGetLastError();
+}
+
+}  // namespace dq

@@ -1,0 +1,152 @@
+// dq_common.cuh -- device helpers shared by the sm_100a kernels of libdqgemv.
+//
+// mbarrier + bulk-copy (cp.async.bulk, the TMA engine's 1-D form) wrappers,
+// the bounded wait that replaces an unbounded spin, and the device error flag.
+// Bulk copies here always read this GPU's own global memory into the issuing
+// CTA's shared memory; no multicast form is used anywhere.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace dq {
+
+constexpr int kQ4KBlockElems = 256;
+constexpr int kQ4KBlockBytes = 144;
+constexpr int kQ8BlockElems = 32;
+constexpr int kQ8BlockBytes = 34;
+
+// Error codes written to the device error flag.
+constexpr int kDevErrWaitTimeout = 1;
+
+// A wait for one of the kernel's own bulk copies is declared lost after this
+// many nanoseconds of the global timer (a legitimate wait is microseconds), or
+// after kWaitLimit polls, whichever comes first.
+constexpr unsigned long long kWaitNanos = 2000000000ull;
+constexpr uint32_t kWaitLimit = 1u << 26;
+
+__device__ __forceinline__ unsigned long long global_ns()
+{
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+// Makes barrier initialisation visible to the async proxy (the bulk-copy unit).
+__device__ __forceinline__ void mbar_fence_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for phase `parity` of barrier `bar`.  Returns false (after
+// setting the device error flag) if the phase did not complete in time.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, int *err)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const unsigned long long t0 = global_ns();
+    for (uint32_t i = 0; i < kWaitLimit; ++i) {
+        if (mbar_try_wait(bar, parity))
+            return true;
+        if ((i & 63) == 63 && global_ns() - t0 > kWaitNanos)
+            break;
+    }
+    if (err)
+        atomicExch(err, kDevErrWaitTimeout);
+    return false;
+}
+
+// Orders this thread's earlier generic-proxy shared-memory accesses before its
+// later async-proxy ones (a bulk copy about to overwrite a consumed slot).
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 1-D bulk copy global -> shared, completing `bytes` of transaction count on
+// barrier `bar`.  dst, src and bytes must be multiples of 16.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ float4 lds128f(uint32_t addr)
+{
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ float4 ldg_nc_f4(const float4 *p)
+{
+    float4 v;
+    asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// fp16 bit pattern -> fp32 (exact; subnormals included).
+__device__ __forceinline__ float half_bits_to_float(uint32_t h)
+{
+    float f;
+    asm("{ .reg .b16 t; cvt.u16.u32 t, %1; cvt.f32.f16 %0, t; }" : "=f"(f) : "r"(h));
+    return f;
+}
+
+// Argmax candidate: the largest value seen and its (lowest) index.
+struct ArgmaxCand {
+    float v;
+    int pad;
+    long long idx;
+};
+
+__device__ __forceinline__ bool cand_better(float v, long long i, float bv, long long bi)
+{
+    return v > bv || (v == bv && i < bi);
+}
+
+}  // namespace dq

@@ -1,0 +1,83 @@
+// dq_internal.h -- declarations shared between the C-ABI layer (api.cu) and the
+// kernel translation units of libdqgemv.  Not installed, not part of the ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace dq {
+
+struct ArgmaxCand;
+
+// Q4_K GEMV kernel arguments (one weight stream, or gate + up for SwiGLU).
+struct Q4KParams {
+    const uint8_t *w[2];
+    const float *x;        // B x K
+    float *y;              // B x N final output (splits == 1)
+    float *part;           // [splits][NS][B][N] partial sums (splits > 1)
+    ArgmaxCand *cand;      // per-CTA argmax candidates (argmax, splits == 1)
+    int *err;              // device error flag
+    long long N;
+    int K;
+    int nb;                // K / 256
+    int splits;
+    int chunks_per_split;  // K-chunks (of LPR super-blocks) per split
+    int ctas_per_split;
+    int depth;             // ring slots per warp
+    int soa;
+    int argmax;
+    long long tiles;       // row tiles
+};
+
+struct Q4KPlan {
+    bool ok;
+    int lpr;               // lanes per row group (4 or 16)
+    int R;                 // rows per lane
+    int warps;             // warps per CTA
+    long long tiles;
+    int splits;
+    int chunks_per_split;
+    int ctas_per_split;
+    int grid;
+    int depth;
+    int smem;
+};
+
+Q4KPlan q4k_plan(long long N, int K, int B, int NS, int soa, int sm_count, int smem_optin);
+cudaError_t q4k_gemv_launch(const Q4KParams &p, const Q4KPlan &pl, int B, int NS, cudaStream_t s);
+
+// Q8_0 GEMV
+struct Q8Params {
+    const uint8_t *w;
+    const float *x;
+    float *y;
+    int *err;
+    long long N;
+    int K;
+    int nb;                // K / 32
+};
+struct Q8Plan {
+    bool ok;
+    int grid;
+    int block;
+    int smem;
+};
+Q8Plan q8_plan(long long N, int K, int B, int sm_count, int smem_optin);
+cudaError_t q8_0_gemv_launch(const Q8Params &p, const Q8Plan &pl, int B, cudaStream_t s);
+
+// split-K reduction (+ SwiGLU epilogue, + argmax candidates), argmax finalisation
+int reduce_grid(long long N, int B);
+cudaError_t splitk_reduce_launch(const float *part, int splits, int NS, int B, long long N, float *y,
+                                 ArgmaxCand *cand, int grid, cudaStream_t s);
+cudaError_t argmax_finalize_launch(const ArgmaxCand *cand, int ncand, long long *out, cudaStream_t s);
+
+// debug dequant, repack
+cudaError_t q4k_dequant_launch(const uint8_t *w, int soa, float *out, long long N, int K, cudaStream_t s);
+cudaError_t q8_0_dequant_launch(const uint8_t *w, float *out, long long N, int K, cudaStream_t s);
+cudaError_t q4k_repack_soa_launch(const uint8_t *aos, uint8_t *soa, long long N, int K, cudaStream_t s);
+
+// device error flag
+int *device_error_flag(int device);
+
+}  // namespace dq

@@ -1,0 +1,520 @@
+// q4k_gemv.cu -- fused Q4_K dequantize + GEMV (plain, fused SwiGLU, B <= 8,
+// optional argmax) for sm_100a.
+//
+// The operation is the pages' fused dequant+GEMV over raw Q4_K bytes (trueno
+// WgslForwardPass: upload_q4k_weight; qualiaDB cuda_lane: try_q4k_soa_gemv,
+// try_q4k_soa_fused_swiglu).  The kernel design below is this library's own.
+//
+// Work decomposition
+//   A warp owns a set of row tiles.  A row tile is TR = (32/LPR)*R rows; lane
+//   (rg, l) = (lane / LPR, lane % LPR) handles rows rg*R .. rg*R+R-1 of the
+//   tile and, in every K-chunk of LPR super-blocks, super-block l of each of
+//   those rows.  One "slot" is one K-chunk of one tile of one weight stream
+//   (TR rows x LPR super-blocks, 9 KB for R = 2).  Each warp streams its own
+//   ring of `depth` slots: lane 0 issues 1-D bulk copies (cp.async.bulk from
+//   this GPU's global memory into the warp's shared-memory slot, completing on
+//   an mbarrier), the whole warp computes on the oldest slot and lane 0 reuses
+//   it for the slot `depth` steps ahead.  CTAs are persistent: a grid of about
+//   one CTA per SM walks all tiles.  K may be split across CTAs (split-K) when
+//   the activations of all of K do not fit in shared memory or when there are
+//   too few row tiles to occupy the GPU; split partial sums go to the caller's
+//   workspace and a second kernel reduces them in a fixed order.
+//
+// Arithmetic (per weight, no factoring of scales or mins)
+//   A quant q at bit position p of a 32-bit word, isolated with one AND, is
+//   the fp32 bit pattern q*2^p, i.e. the subnormal (or smallest-normal) value
+//   q*2^(p-149).  One fma with d*scale*2^(85-p) and -dmin*min*2^-64 then gives
+//   (d*scale*q - dmin*min) * 2^-64 rounded once: exactly the fp32 weight that
+//   q4k_dequant returns, times 2^-64 (all operands are exact: d has 11
+//   significant bits, scale and min 6, q 4).  A second fma accumulates
+//   weight*x.  Sums are taken in units of 2^-64 and scaled back at the end, so
+//   any finite fp32 x is accepted.  Both fmas run as fma.rn.f32x2 on pairs.
+//   Subnormal operands are kept (the library is built without flush-to-zero).
+
+#include <cuda_fp16.h>
+#include <cstdint>
+
+#include "dq_common.cuh"
+#include "dq_internal.h"
+#include "q4k_decode.cuh"
+
+namespace dq {
+
+// One quant word: form its eight weights and accumulate weight*x (low nibbles
+// into accL, high nibbles into accH).  xl = x[L+4t .. L+4t+3], xh = x[H+4t ..].
+__device__ __forceinline__ void q4_word(uint32_t w, float2 sL, float2 mL, float2 sH, float2 mH,
+                                        float4 xl, float4 xh, float2 &accL, float2 &accH)
+{
+    float2 wv[4];
+    q4_word_weights(w, sL, mL, sH, mH, wv);
+    accL = __ffma2_rn(wv[0], f2(xl.x, xl.y), accL);
+    accH = __ffma2_rn(wv[2], f2(xh.x, xh.y), accH);
+    accL = __ffma2_rn(wv[1], f2(xl.z, xl.w), accL);
+    accH = __ffma2_rn(wv[3], f2(xh.z, xh.w), accH);
+}
+
+constexpr int kMaxWarps = 8;
+constexpr int kMaxThreads = kMaxWarps * 32;
+constexpr int kXBlockPitch = 1040;  // bytes per staged 256-float block of x (16 B pad)
+
+template <int LPR, int R>
+struct Geo {
+    static constexpr int RG = 32 / LPR;                       // row groups per warp
+    static constexpr int TR = RG * R;                         // rows per tile
+    static constexpr int ROW_BYTES = LPR * kQ4KBlockBytes;    // one row of a slot
+    static constexpr int PAD = (LPR < 8) ? 64 : 0;            // bank-shift between row groups
+    static constexpr int RG_PITCH = R * ROW_BYTES + PAD;
+    static constexpr int SLOT_BYTES = RG * RG_PITCH;
+    static_assert(SLOT_BYTES % 128 == 0, "slot must keep 128-byte alignment");
+};
+
+// Transposing butterfly over the LPR lanes of a row group: on entry each lane
+// holds M partial values; on exit lane l holds the sums of a contiguous run of
+// value indices (the kernel recomputes which).  M is a power of two.
+template <int O, int M>
+struct GroupReduce {
+    static __device__ __forceinline__ void run(float *v, int lane)
+    {
+        if constexpr (M > 1) {
+            const bool up = (lane & O) != 0;
+#pragma unroll
+            for (int i = 0; i < M / 2; ++i) {
+                const float send = up ? v[i] : v[i + M / 2];
+                const float keep = up ? v[i + M / 2] : v[i];
+                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, O);
+            }
+            if constexpr (O > 1)
+                GroupReduce<O / 2, M / 2>::run(v, lane);
+        } else {
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], O);
+            if constexpr (O > 1)
+                GroupReduce<O / 2, 1>::run(v, lane);
+        }
+    }
+};
+
+template <int N>
+struct Pow2Ceil {
+    static constexpr int value = (N <= 1) ? 1 : 2 * Pow2Ceil<(N + 1) / 2>::value;
+};
+template <>
+struct Pow2Ceil<1> {
+    static constexpr int value = 1;
+};
+
+// Issues the bulk copies of slot-sequence element i of one warp into ring slot
+// `slot`: K-chunk kc of stream st of tile t (rows row0 .. row0+rows-1).
+template <int LPR, int R>
+__device__ __forceinline__ void issue_slot(const Q4KParams &p, long long i, int slot, long long per_tile, int nch,
+                                           int c_begin, long long t0, long long tstride, uint32_t ring_s,
+                                           uint32_t bars_s)
+{
+    using G = Geo<LPR, R>;
+    const long long row_bytes_g = static_cast<long long>(p.nb) * kQ4KBlockBytes;
+    const long long tk = i / per_tile;
+    const int rem = static_cast<int>(i - tk * per_tile);
+    const int st = rem / nch;
+    const int kc = c_begin + rem % nch;
+    const long long tile = t0 + tk * tstride;
+    const long long row0 = tile * G::TR;
+    const int rows = static_cast<int>(min(static_cast<long long>(G::TR), p.N - row0));
+    const int kb0 = kc * LPR;
+    const int nblk = min(LPR, p.nb - kb0);
+    const uint8_t *src = (st == 0 ? p.w[0] : p.w[1]) + row0 * row_bytes_g + static_cast<long long>(kb0) * kQ4KBlockBytes;
+    const uint32_t dst = ring_s + slot * G::SLOT_BYTES;
+    const uint32_t bar = bars_s + slot * 8;
+    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(rows * nblk * kQ4KBlockBytes));
+    if (nblk == p.nb && p.nb == LPR) {
+        // whole rows, contiguous in global memory: one copy per row group
+        for (int g = 0; g * R < rows; ++g) {
+            const int gr = min(R, rows - g * R);
+            bulk_g2s(dst + g * G::RG_PITCH, src + static_cast<long long>(g) * R * row_bytes_g,
+                     static_cast<uint32_t>(gr * G::ROW_BYTES), bar);
+        }
+    } else {
+        for (int r = 0; r < rows; ++r)
+            bulk_g2s(dst + (r / R) * G::RG_PITCH + (r % R) * G::ROW_BYTES, src + r * row_bytes_g,
+                     static_cast<uint32_t>(nblk * kQ4KBlockBytes), bar);
+    }
+}
+
+template <int LPR, int B, int NS, int R>
+__global__ void __launch_bounds__(kMaxThreads, 1) q4k_gemv_kernel(const Q4KParams p)
+{
+    using G = Geo<LPR, R>;
+    constexpr int MV = R * B;                         // values per lane per stream
+    constexpr int MP = Pow2Ceil<MV>::value;           // padded to a power of two
+    constexpr int VPL = (MP > LPR) ? MP / LPR : 1;    // values per lane after reduce
+
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int nwarps = blockDim.x >> 5;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int rg = lane / LPR;
+    const int l = lane % LPR;
+
+    const int split = blockIdx.x / p.ctas_per_split;
+    const int cj = blockIdx.x % p.ctas_per_split;
+    const int nchunk_total = (p.nb + LPR - 1) / LPR;
+    const int c_begin = split * p.chunks_per_split;
+    const int c_end = min(c_begin + p.chunks_per_split, nchunk_total);
+    const int nch = c_end - c_begin;
+    const int kb_begin = c_begin * LPR;
+    const int nbs = min(nch * LPR, p.nb - kb_begin);  // super-blocks of this split
+
+    // shared memory: [x staging][barriers][ring][argmax scratch]
+    const int x_bytes = (B * nbs * kXBlockPitch + 127) & ~127;
+    uint8_t *xs = smem;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + x_bytes);
+    const int bar_bytes = (nwarps * p.depth * 8 + 127) & ~127;
+    uint8_t *ring = smem + x_bytes + bar_bytes;
+    uint8_t *my_ring = ring + static_cast<size_t>(warp) * p.depth * G::SLOT_BYTES;
+    const uint32_t my_ring_s = smem_u32(my_ring);
+    const uint32_t my_bars_s = smem_u32(bars + warp * p.depth);
+    ArgmaxCand *red = reinterpret_cast<ArgmaxCand *>(ring + static_cast<size_t>(nwarps) * p.depth * G::SLOT_BYTES);
+
+    // this warp's tiles
+    const long long tstride = static_cast<long long>(p.ctas_per_split) * nwarps;
+    const long long t0 = static_cast<long long>(cj) * nwarps + warp;
+    const long long ntiles_w = (t0 < p.tiles) ? (p.tiles - t0 + tstride - 1) / tstride : 0;
+    const long long per_tile = static_cast<long long>(NS) * nch;
+    const long long total = ntiles_w * per_tile;
+
+    if (lane == 0) {
+        for (int s = 0; s < p.depth; ++s)
+            mbar_init(my_bars_s + s * 8, 1);
+        mbar_fence_init();
+        const long long pre = min(static_cast<long long>(p.depth), total);
+        for (long long i = 0; i < pre; ++i)
+            issue_slot<LPR, R>(p, i, static_cast<int>(i), per_tile, nch, c_begin, t0, tstride, my_ring_s, my_bars_s);
+    }
+
+    // stage this split's activations (fp32, 16-byte padded per super-block)
+    {
+        const int per_b = nbs * 64;  // float4 per batch row
+        for (int idx = threadIdx.x; idx < B * per_b; idx += blockDim.x) {
+            const int b = idx / per_b;
+            const int rem = idx - b * per_b;
+            const int kbl = rem >> 6;
+            const int q = rem & 63;
+            const float4 *src = reinterpret_cast<const float4 *>(
+                p.x + static_cast<long long>(b) * p.K + static_cast<long long>(kb_begin + kbl) * 256) + q;
+            float4 v = ldg_nc_f4(src);
+            *reinterpret_cast<float4 *>(xs + (b * nbs + kbl) * kXBlockPitch + q * 16) = v;
+        }
+    }
+    __syncthreads();
+    __syncwarp();
+
+    const uint32_t xs_s = smem_u32(xs);
+    float best_v = -INFINITY;
+    long long best_i = 0x7fffffffffffffffLL;
+    bool failed = false;
+    long long consumed = 0;
+
+    float2 accL[R][B], accH[R][B];
+    float gsum[NS == 2 ? MP : 1];  // stream-0 sums kept for the SwiGLU epilogue
+
+    for (long long i = 0; i < total; ++i) {
+        const int slot = static_cast<int>(i % p.depth);
+        const uint32_t parity = static_cast<uint32_t>((i / p.depth) & 1);
+        const bool ok = mbar_wait_bounded(my_bars_s + slot * 8, parity, p.err);
+        if (!__all_sync(0xffffffffu, ok)) {
+            failed = true;
+            break;
+        }
+        consumed = i + 1;
+        const long long tk = i / per_tile;
+        const int rem = static_cast<int>(i - tk * per_tile);
+        const int st = rem / nch;
+        const int kcl = rem % nch;
+        const int kc = c_begin + kcl;
+        const long long tile = t0 + tk * tstride;
+        const long long row0 = tile * G::TR;
+
+        if (kcl == 0) {
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int b = 0; b < B; ++b) {
+                    accL[r][b] = f2(0.f, 0.f);
+                    accH[r][b] = f2(0.f, 0.f);
+                }
+        }
+
+        const int kb0 = kc * LPR;
+        const int nblk = min(LPR, p.nb - kb0);
+        if (l < nblk) {
+            const uint32_t slot_s = my_ring_s + slot * G::SLOT_BYTES + rg * G::RG_PITCH;
+            // byte offsets of this lane's header and quant slices within a row of the slot
+            uint32_t hdr_off, qs_off0, qs_step;
+            if (p.soa) {
+                hdr_off = 16u * l;
+                qs_off0 = 16u * nblk + 16u * l;
+                qs_step = 16u * nblk;
+            } else {
+                hdr_off = kQ4KBlockBytes * l;
+                qs_off0 = hdr_off + 16u;
+                qs_step = 16u;
+            }
+            Hdr hd[R];
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+                hd[r] = decode_hdr(lds128(slot_s + r * G::ROW_BYTES + hdr_off));
+            const uint32_t xblk = xs_s + (kb0 - kb_begin + l) * kXBlockPitch;
+
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float2 sL[R], mL[R], sH[R], mH[R];
+#pragma unroll
+                for (int r = 0; r < R; ++r)
+                    chunk_scales(hd[r], c, sL[r], mL[r], sH[r], mH[r]);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int s = 2 * c + h;  // 16-byte quant slice
+                    uint4 q[R];
+#pragma unroll
+                    for (int r = 0; r < R; ++r)
+                        q[r] = lds128(slot_s + r * G::ROW_BYTES + qs_off0 + s * qs_step);
+                    const uint32_t xoffL = (64 * c + 16 * h) * 4;
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+#pragma unroll
+                        for (int b = 0; b < B; ++b) {
+                            const uint32_t xb = xblk + b * nbs * kXBlockPitch + xoffL + 16 * t;
+                            const float4 xl = lds128f(xb);
+                            const float4 xh = lds128f(xb + 128);
+#pragma unroll
+                            for (int r = 0; r < R; ++r) {
+                                const uint32_t wv = (t == 0) ? q[r].x : (t == 1) ? q[r].y : (t == 2) ? q[r].z : q[r].w;
+                                q4_word(wv, sL[r], mL[r], sH[r], mH[r], xl, xh, accL[r][b], accH[r][b]);
+                            }
+                        }
+                    }
+                }
+            }
+        }
+
+        __syncwarp();
+        if (lane == 0 && i + p.depth < total) {
+            fence_proxy_async_smem();
+            issue_slot<LPR, R>(p, i + p.depth, slot, per_tile, nch, c_begin, t0, tstride, my_ring_s, my_bars_s);
+        }
+
+        if (kcl == nch - 1) {
+            // end of this stream's K range for the tile: reduce across the row group
+            float v[MP];
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int b = 0; b < B; ++b) {
+                    const float2 a = __fadd2_rn(accL[r][b], accH[r][b]);
+                    v[r * B + b] = a.x + a.y;
+                }
+#pragma unroll
+            for (int j = MV; j < MP; ++j)
+                v[j] = 0.f;
+            if constexpr (LPR > 1)
+                GroupReduce<LPR / 2, MP>::run(v, l);
+
+            // which value indices this lane now holds
+            int off = 0;
+            bool writer = true;
+            {
+                int m = MP;
+#pragma unroll
+                for (int o = LPR / 2; o >= 1; o >>= 1) {
+                    if (m > 1) {
+                        if (l & o)
+                            off += m / 2;
+                        m /= 2;
+                    } else if (l & o) {
+                        writer = false;
+                    }
+                }
+            }
+
+            if constexpr (NS == 2) {
+                if (st == 0) {
+#pragma unroll
+                    for (int j = 0; j < VPL; ++j)
+                        gsum[j] = v[j];
+                    continue;
+                }
+            }
+            if (writer) {
+#pragma unroll
+                for (int j = 0; j < VPL; ++j) {
+                    const int idx = off + j;
+                    if (idx >= MV)
+                        continue;
+                    const int r = idx / B;
+                    const int b = idx % B;
+                    const long long n = row0 + rg * R + r;
+                    if (n >= p.N)
+                        continue;
+                    if (p.splits > 1) {
+                        if constexpr (NS == 2) {
+                            p.part[((static_cast<long long>(split) * 2 + 0) * B + b) * p.N + n] = gsum[j] * 0x1p64f;
+                            p.part[((static_cast<long long>(split) * 2 + 1) * B + b) * p.N + n] = v[j] * 0x1p64f;
+                        } else {
+                            p.part[(static_cast<long long>(split) * B + b) * p.N + n] = v[j] * 0x1p64f;
+                        }
+                    } else {
+                        float out;
+                        if constexpr (NS == 2) {
+                            const float g = gsum[j] * 0x1p64f;
+                            const float u = v[j] * 0x1p64f;
+                            out = g / (1.0f + expf(-g)) * u;
+                        } else {
+                            out = v[j] * 0x1p64f;
+                        }
+                        p.y[static_cast<long long>(b) * p.N + n] = out;
+                        if (p.argmax && cand_better(out, n, best_v, best_i)) {
+                            best_v = out;
+                            best_i = n;
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    if (failed) {
+        // the copies already issued into this warp's ring must land before the CTA exits
+        const long long issued = min(total, consumed + p.depth);
+        for (long long i = consumed; i < issued; ++i) {
+            const int slot = static_cast<int>(i % p.depth);
+            const uint32_t parity = static_cast<uint32_t>((i / p.depth) & 1);
+            mbar_wait_bounded(my_bars_s + slot * 8, parity, nullptr);
+        }
+    }
+
+    if (p.argmax && p.splits == 1) {
+        // CTA-wide (max, lowest index) candidate
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, best_v, o);
+            const long long oi = __shfl_xor_sync(0xffffffffu, best_i, o);
+            if (cand_better(ov, oi, best_v, best_i)) {
+                best_v = ov;
+                best_i = oi;
+            }
+        }
+        if (lane == 0) {
+            red[warp].v = best_v;
+            red[warp].idx = best_i;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            ArgmaxCand c = red[0];
+            for (int w = 1; w < nwarps; ++w)
+                if (cand_better(red[w].v, red[w].idx, c.v, c.idx))
+                    c = red[w];
+            p.cand[blockIdx.x] = c;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+int q4k_slot_bytes(int lpr) { return lpr == 16 ? Geo<16, 2>::SLOT_BYTES : Geo<4, 2>::SLOT_BYTES; }
+
+// Launch plan for a shape; the same function sizes the workspace, so the two
+// always agree.
+Q4KPlan q4k_plan(long long N, int K, int B, int NS, int soa, int sm_count, int smem_optin)
+{
+    Q4KPlan pl{};
+    const int nb = K / kQ4KBlockElems;
+    const int misc = 128 /*argmax scratch*/ + 256 /*barriers*/;
+    // SoA groups are 16 super-blocks, so SoA always walks K in 16-block chunks.
+    const int lpr_opts[2] = {(soa || nb % 16 == 0) ? 16 : 4, 4};
+    const int n_opts = (soa || nb % 16 != 0) ? 1 : 2;
+    for (int oi = 0; oi < n_opts && !pl.ok; ++oi) {
+        const int lpr = lpr_opts[oi];
+        const int sb = q4k_slot_bytes(lpr);
+        const int TR = (32 / lpr) * 2;
+        const long long tiles = (N + TR - 1) / TR;
+        const int nchunk = (nb + lpr - 1) / lpr;
+        for (int warps = kMaxWarps; warps >= 4 && !pl.ok; warps /= 2) {
+            const int min_ring = warps * 2 * sb;
+            // smallest split count whose activations fit beside a two-deep ring
+            int splits = 1;
+            int cps = nchunk;
+            for (;;) {
+                cps = (nchunk + splits - 1) / splits;
+                const int xb = B * cps * lpr * kXBlockPitch;
+                if (xb + min_ring + misc <= smem_optin || cps == 1)
+                    break;
+                ++splits;
+            }
+            // split K further while fewer than half of the warps would have a tile
+            const long long warps_total = static_cast<long long>(sm_count) * warps;
+            while (tiles * NS * splits * 2 < warps_total && splits < nchunk) {
+                ++splits;
+                cps = (nchunk + splits - 1) / splits;
+            }
+            splits = (nchunk + cps - 1) / cps;
+            const int x_bytes = (B * cps * lpr * kXBlockPitch + 127) & ~127;
+            int depth = (smem_optin - x_bytes - misc) / (warps * sb);
+            if (depth > 4)
+                depth = 4;
+            if (depth < 2)
+                continue;
+            long long ctas = (tiles + warps - 1) / warps;
+            const long long max_ctas = sm_count / splits > 0 ? sm_count / splits : 1;
+            if (ctas > max_ctas)
+                ctas = max_ctas;
+            pl.lpr = lpr;
+            pl.R = 2;
+            pl.warps = warps;
+            pl.tiles = tiles;
+            pl.splits = splits;
+            pl.chunks_per_split = cps;
+            pl.depth = depth;
+            pl.ctas_per_split = static_cast<int>(ctas);
+            pl.grid = pl.ctas_per_split * splits;
+            pl.smem = x_bytes + ((warps * depth * 8 + 127) & ~127) + warps * depth * sb + 128;
+            pl.ok = pl.smem <= smem_optin;
+        }
+    }
+    return pl;
+}
+
+template <int LPR, int B, int NS>
+static cudaError_t launch_one(const Q4KParams &p, const Q4KPlan &pl, cudaStream_t s)
+{
+    auto k = q4k_gemv_kernel<LPR, B, NS, 2>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
+    if (e != cudaSuccess)
+        return e;
+    k<<<pl.grid, pl.warps * 32, pl.smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+template <int LPR, int NS>
+static cudaError_t launch_b(const Q4KParams &p, const Q4KPlan &pl, int B, cudaStream_t s)
+{
+    switch (B) {
+    case 1: return launch_one<LPR, 1, NS>(p, pl, s);
+    case 2: return launch_one<LPR, 2, NS>(p, pl, s);
+    case 3: return launch_one<LPR, 3, NS>(p, pl, s);
+    case 4: return launch_one<LPR, 4, NS>(p, pl, s);
+    case 5: return launch_one<LPR, 5, NS>(p, pl, s);
+    case 6: return launch_one<LPR, 6, NS>(p, pl, s);
+    case 7: return launch_one<LPR, 7, NS>(p, pl, s);
+    case 8: return launch_one<LPR, 8, NS>(p, pl, s);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t q4k_gemv_launch(const Q4KParams &p, const Q4KPlan &pl, int B, int NS, cudaStream_t s)
+{
+    if (pl.lpr == 16)
+        return NS == 1 ? launch_b<16, 1>(p, pl, B, s) : launch_b<16, 2>(p, pl, B, s);
+    return NS == 1 ? launch_b<4, 1>(p, pl, B, s) : launch_b<4, 2>(p, pl, B, s);
+}
+
+}  // namespace dq

@@ -1,0 +1,167 @@
+/*
+ * dqgemv.h -- C ABI of libdqgemv.so: fused block-quantized dequantize + GEMV
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The operation.  y = W x for one decode step, where W (N rows x K columns) is
+ * stored as GGML-style quantized blocks and x is fp32.  The pages this library
+ * follows call it the fused dequant+GEMV ("upload raw Q4K weight bytes for
+ * fused dequant+GEMV on GPU": trueno WgslForwardPass, upload_q4k_weight) and
+ * ship it as a CUDA lane with a Q4_K structure-of-arrays GEMV, a fused SwiGLU
+ * variant and a Q8_0 GEMV (qualiaDB cuda_lane module map: try_q4k_soa_gemv,
+ * try_q4k_soa_fused_swiglu, try_q8_0_cuda_gemv, preload_q4k_soa_weights).
+ *
+ * Block formats (little-endian):
+ *   Q8_0  34 bytes / 32 weights:  d (fp16) | q[32] (int8)         w = d*q
+ *   Q4_K 144 bytes / 256 weights: d (fp16) | dmin (fp16) | 12 scale bytes
+ *         (8 six-bit scale/min pairs, GGML get_scale_min_k4 packing)
+ *         | 128 quant bytes (4-bit; chunk c = bytes 32c..32c+31 holds weights
+ *         64c..64c+31 in its low nibbles and 64c+32..64c+63 in its high ones)
+ *         w = d*scale_j*q - dmin*min_j  for sub-block j = weight/32.
+ *   A row is K/32 (Q8_0) or K/256 (Q4_K) consecutive blocks; rows follow each
+ *   other without padding, so W occupies N*K*34/32 or N*K*144/256 bytes.
+ *
+ * Numerics.  Every weight is formed exactly as the fp32 value nearest to its
+ * exact dequantized value (the same bits the *_dequant entry points return)
+ * and the products are accumulated in fp32.  Results satisfy
+ *     |y - y_exact| <= 1e-4 * sum_k |W[n][k] * x[k]| + 1e-6
+ * for finite inputs.
+ *
+ * Conventions shared by every entry point:
+ *   - All data pointers are DEVICE pointers owned by the caller (for example
+ *     allocated by PyTorch).  The library never allocates or frees memory.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *     are asynchronous: they enqueue work and return without synchronizing.
+ *     Inputs must stay alive, and outputs untouched, until the stream reaches
+ *     the call.
+ *   - Every argument is validated on the host before anything is enqueued.
+ *     On any error status nothing is launched and no memory is touched.
+ *   - The device of the call is the current CUDA device of the calling thread.
+ *   - Batched activations are row-major: x is B x K (row b at x + b*K) and y is
+ *     B x N (row b at y + b*N).
+ */
+#ifndef DQGEMV_H
+#define DQGEMV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum dq_status {
+    DQ_OK = 0,
+    DQ_ERR_NULL = 1,      /* a required pointer is NULL                              */
+    DQ_ERR_SHAPE = 2,     /* N < 1, K not a positive multiple of the block size,
+                             K above the supported maximum, or B outside [1, 8]      */
+    DQ_ERR_ALIGN = 3,     /* w or x is not 16-byte aligned, y not 4-byte aligned     */
+    DQ_ERR_WORKSPACE = 4, /* workspace NULL or smaller than dq_workspace_bytes()     */
+    DQ_ERR_LAYOUT = 5,    /* layout is not DQ_LAYOUT_AOS / DQ_LAYOUT_SOA             */
+    DQ_ERR_CUDA = 6,      /* a CUDA runtime call failed; see dq_last_cuda_error()    */
+    DQ_ERR_ARG = 7        /* any other invalid argument (e.g. argmax with B != 1)    */
+} dq_status;
+
+typedef enum dq_layout {
+    DQ_LAYOUT_AOS = 0,    /* GGML block order: 144-byte super-blocks back to back    */
+    DQ_LAYOUT_SOA = 1     /* q4k_repack_soa() order (see there)                      */
+} dq_layout;
+
+typedef enum dq_op {
+    DQ_OP_Q8_0_GEMV = 0,
+    DQ_OP_Q4K_GEMV = 1,
+    DQ_OP_Q4K_SWIGLU = 2
+} dq_op;
+
+/* Largest K accepted by the GEMV entry points (fp32 activations of one split
+ * of K are staged in shared memory). */
+#define DQ_MAX_K 1048576
+
+/*
+ * Q8_0 GEMV:  y[b][n] = sum_k W[n][k] * x[b][k].
+ *   w   N*(K/32) Q8_0 blocks (34 bytes each), 16-byte aligned.
+ *   x   B x K fp32, 16-byte aligned.       y  B x N fp32, 4-byte aligned.
+ *   K   positive multiple of 32.           B  1..8.
+ *   workspace / ws_bytes: scratch of at least
+ *       dq_workspace_bytes(DQ_OP_Q8_0_GEMV, N, K, B, 0) bytes (may be NULL/0
+ *       when that is 0).  Contents on entry are ignored; the library keeps no
+ *       state in it between calls.
+ */
+dq_status q8_0_gemv(const void *w, const float *x, float *y, int64_t N, int64_t K, int B,
+                    void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Q4_K GEMV:  y[b][n] = sum_k W[n][k] * x[b][k],  optionally with argmax.
+ *   w          N*(K/256) Q4_K super-blocks, 16-byte aligned, in `layout`.
+ *   x, y, B    as for q8_0_gemv.           K  positive multiple of 256.
+ *   argmax_out NULL, or (B == 1 only) a device int64: receives the index n of
+ *              the largest y[0][n]; among equal largest values the lowest n.
+ *              (The LM-head epilogue; NaN outputs make it unspecified.)
+ *   workspace  at least dq_workspace_bytes(DQ_OP_Q4K_GEMV, N, K, B,
+ *              argmax_out != NULL) bytes.
+ */
+dq_status q4k_gemv(const void *w, int layout, const float *x, float *y, int64_t N, int64_t K,
+                   int B, int64_t *argmax_out, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Fused gate/up SwiGLU GEMV (qualiaDB cuda_lane: try_q4k_soa_fused_swiglu;
+ * trueno WgslForwardPass: silu_mul_shader, here fused into the GEMV):
+ *   out[b][n] = silu(g) * u,  g = (W_gate x_b)[n],  u = (W_up x_b)[n],
+ *   silu(g) = g / (1 + exp(-g)).
+ *   w_gate, w_up  two N x K Q4_K matrices in the same `layout`, 16-byte aligned.
+ *   out           B x N fp32.  Other arguments as for q4k_gemv.
+ *   workspace     at least dq_workspace_bytes(DQ_OP_Q4K_SWIGLU, N, K, B, 0).
+ */
+dq_status q4k_swiglu_gemv(const void *w_gate, const void *w_up, int layout, const float *x,
+                          float *out, int64_t N, int64_t K, int B, void *workspace,
+                          size_t ws_bytes, void *stream);
+
+/*
+ * Offline repack of a Q4_K matrix from GGML block order (AoS) into this
+ * library's structure-of-arrays order (qualiaDB cuda_lane:
+ * preload_q4k_soa_weights; the pages do not define the SoA layout, this is the
+ * library's own).  Every row keeps its byte range and size.  Within a row the
+ * super-blocks are taken in groups of 16 (the last group holds the remaining
+ * g <= 16); a group of g blocks is stored as g 16-byte headers (d, dmin, 12
+ * scale bytes of block t at 16*t) followed by 8 slices, slice s holding quant
+ * bytes 16s..16s+15 of each block t at 16*g + 16*g*s + 16*t.
+ *   w_aos, w_soa  N*(K/256)*144 bytes each, 16-byte aligned, not overlapping.
+ */
+dq_status q4k_repack_soa(const void *w_aos, void *w_soa, int64_t N, int64_t K, void *stream);
+
+/*
+ * Scratch bytes the GEMV entry points need for this shape on the current
+ * device (split-K partial sums, argmax candidates).  0 means none.
+ * `op` is a dq_op; `with_argmax` is nonzero when argmax_out will be passed.
+ * Returns (size_t)-1 for an invalid op or shape.
+ */
+size_t dq_workspace_bytes(int op, int64_t N, int64_t K, int B, int with_argmax);
+
+/*
+ * Debug dequantization (the bit-exact check of the weights the GEMVs use):
+ * out[n][k] = the fp32 value nearest to the exact dequantized W[n][k]
+ * (round to nearest even).  out is N x K fp32, 4-byte aligned.  Rows are
+ * independent, so a row slice is a pointer offset on w and out.
+ */
+dq_status q8_0_dequant(const void *w, float *out, int64_t N, int64_t K, void *stream);
+dq_status q4k_dequant(const void *w, int layout, float *out, int64_t N, int64_t K, void *stream);
+
+/* Static string naming a status code. */
+const char *dq_status_string(int status);
+
+/* cudaError_t of the most recent DQ_ERR_CUDA returned on this thread (0 if none). */
+int dq_last_cuda_error(void);
+
+/*
+ * Device-side error flag of the current device.  Kernels that wait for their
+ * own asynchronous copies give up after a bounded wait instead of hanging;
+ * when that happens they set this flag (and their output is invalid).
+ * Synchronizes `stream`, writes the flag value to *flag (0 = no error) and,
+ * when `clear` is nonzero, resets it.
+ */
+dq_status dq_device_error(int *flag, int clear, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DQGEMV_H */

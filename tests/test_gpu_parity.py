@@ -1,0 +1,332 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Bars (from the method's definition):
+  * dequantized weights and the SoA repack: bit-exact;
+  * GEMV outputs: |y_gpu - y_ref| <= 1e-4 * sum_k |w_nk x_k| + 1e-6, with y_ref
+    and the sum accumulated in double over the exact weights;
+  * SwiGLU: the GEMV bound propagated through silu (oracle.swiglu_tolerance);
+  * argmax: exactly the oracle's index (lowest index on ties), asserted only
+    when the oracle's top-2 margin exceeds the two logits' tolerances.
+Inputs are the seeded synthetic workloads (dequant_gemv_q4_b200.synth).
+"""
+
+import concurrent.futures
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from dequant_gemv_q4_b200 import synth
+
+torch = pytest.importorskip("torch")
+import dequant_gemv_q4_b200 as dq  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+THREADS = max(1, min(16, os.cpu_count() or 1))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.init()
+    dq.load_library()
+    yield
+    assert dq.dq_device_error(clear=True) == 0
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host(t):
+    torch.cuda.synchronize()
+    return t.cpu().numpy()
+
+
+def oracle_rows(fn, N, rows, **kw):
+    """Run an oracle GEMV over `rows` in THREADS threads (ctypes drops the GIL)."""
+    rows = np.asarray(rows, dtype=np.int64)
+    parts = np.array_split(rows, THREADS)
+    with concurrent.futures.ThreadPoolExecutor(THREADS) as ex:
+        res = list(ex.map(lambda r: fn(rows=r, **kw), [p for p in parts if p.size]))
+    return np.concatenate([r[0] for r in res], axis=1), np.concatenate([r[1] for r in res], axis=1)
+
+
+def assert_within(y_gpu, y_ref, a_ref, what=""):
+    y_gpu = np.asarray(y_gpu, dtype=np.float64).reshape(y_ref.shape)
+    err = np.abs(y_gpu - y_ref)
+    tol = oracle.gemv_tolerance(a_ref)
+    ratio = err / tol
+    assert np.all(np.isfinite(y_gpu)), what + ": non-finite output"
+    assert ratio.max() <= 1.0, "%s: %d of %d outputs out of tolerance, worst err/tol %.3g" % (
+        what, int((ratio > 1).sum()), ratio.size, ratio.max())
+
+
+# --- dequantization and repack: bit-exact -----------------------------------------------
+
+@pytest.mark.parametrize("N,K,seed", [(4096, 1024, 1), (37, 5120, 11), (5, 256, 12), (3, 12288, 13)])
+@pytest.mark.parametrize("layout", ["aos", "soa"])
+def test_q4k_dequant_bit_exact(N, K, seed, layout):
+    w = synth.q4k_matrix(np.random.default_rng(seed), N, K)
+    if layout == "soa":
+        w = oracle.q4k_repack_soa(w, N, K)
+    want = oracle.q4k_dequant_f32(w, N, K, layout=layout)
+    got = host(dq.q4k_dequant(dev(w), N, K, layout=layout))
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+
+
+def test_q4k_dequant_row_slice_of_lm_head_rows():
+    # rows are independent: a row slice is a pointer offset (here: rows 1000..1063)
+    N, K = 2048, 4096
+    w = synth.q4k_matrix(np.random.default_rng(4), N, K)
+    wd = dev(w)
+    row_bytes = K // 256 * 144
+    sl = wd.view(-1)[1000 * row_bytes:1064 * row_bytes]
+    got = host(dq.q4k_dequant(sl, 64, K))
+    want = oracle.q4k_dequant_f32(w[1000:1064], 64, K)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+
+
+def test_q4k_dequant_handworked_special_blocks():
+    # zero quants (w = -dmin*min), q=15/scale=63/min=0 (945*d), subnormal d and dmin
+    blocks = [
+        synth.q4k_pack([1.0], [0.25], [np.array([1, 2, 3, 4, 5, 6, 7, 8, 0, 0, 0, 0], np.uint8)],
+                       [np.zeros(128, np.uint8)]),
+        synth.q4k_pack([0.5], [1.0], [np.array([255] * 4 + [0] * 4 + [15] * 4, np.uint8)],
+                       [np.full(128, 255, np.uint8)]),
+        synth.q4k_pack(np.array([1], np.uint16).view(np.float16), np.array([512], np.uint16).view(np.float16),
+                       [np.full(12, 255, np.uint8)], [np.full(128, 15, np.uint8)]),
+    ]
+    w = np.concatenate(blocks).reshape(3, 144)
+    got = host(dq.q4k_dequant(dev(w), 3, 256))
+    want = oracle.q4k_dequant_f32(w, 3, 256)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+    assert np.all(got[1] == np.float32(945 * 0.5))
+
+
+@pytest.mark.parametrize("N,K,seed", [(1024, 1024, 0), (7, 96, 1), (3, 32, 2)])
+def test_q8_0_dequant_bit_exact(N, K, seed):
+    w = synth.q8_0_matrix(np.random.default_rng(seed), N, K)
+    got = host(dq.q8_0_dequant(dev(w), N, K))
+    want = oracle.q8_0_dequant_f32(w, N, K)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+
+
+@pytest.mark.parametrize("N,K", [(4096, 1024), (3, 5120), (5, 256), (2, 12288)])
+def test_repack_soa_bit_exact(N, K):
+    w = synth.q4k_matrix(np.random.default_rng(N + K), N, K)
+    got = host(dq.q4k_repack_soa(dev(w), N, K))
+    assert np.array_equal(got, oracle.q4k_repack_soa(w, N, K))
+
+
+# --- the five workloads -------------------------------------------------------------------
+
+def test_q8_0_gemv_1024x1024():
+    wl = synth.WORKLOADS["q8_0_gemv_1024x1024"]
+    inp = synth.make_inputs(wl)
+    y = host(dq.q8_0_gemv(dev(inp["w"]), dev(inp["x"]), wl.N, wl.K))
+    y_ref, a_ref = oracle_rows(lambda rows: oracle.q8_0_gemv(inp["w"], wl.N, wl.K, inp["x"], rows=rows),
+                               wl.N, np.arange(wl.N))
+    assert_within(y, y_ref, a_ref, "q8_0 1024x1024")
+
+
+@pytest.mark.parametrize("layout", ["aos", "soa"])
+def test_q4k_gemv_4096x1024(layout):
+    wl = synth.WORKLOADS["q4k_gemv_4096x1024"]
+    inp = synth.make_inputs(wl)
+    w = inp["w"] if layout == "aos" else oracle.q4k_repack_soa(inp["w"], wl.N, wl.K)
+    y = host(dq.q4k_gemv(dev(w), dev(inp["x"]), wl.N, wl.K, layout=layout))
+    y_ref, a_ref = oracle_rows(lambda rows: oracle.q4k_gemv(inp["w"], wl.N, wl.K, inp["x"], rows=rows),
+                               wl.N, np.arange(wl.N))
+    assert_within(y, y_ref, a_ref, "q4k 4096x1024 " + layout)
+
+
+def test_q4k_swiglu_12288x4096():
+    wl = synth.WORKLOADS["q4k_swiglu_12288x4096"]
+    inp = synth.make_inputs(wl)
+    out = host(dq.q4k_swiglu_gemv(dev(inp["w_gate"]), dev(inp["w_up"]), dev(inp["x"]), wl.N, wl.K))
+    rows = np.arange(wl.N)
+    g, ag = oracle_rows(lambda rows: oracle.q4k_gemv(inp["w_gate"], wl.N, wl.K, inp["x"], rows=rows), wl.N, rows)
+    u, au = oracle_rows(lambda rows: oracle.q4k_gemv(inp["w_up"], wl.N, wl.K, inp["x"], rows=rows), wl.N, rows)
+    ref = oracle.swiglu(g, u)
+    tol = oracle.swiglu_tolerance(g, u, ag, au)
+    err = np.abs(out.reshape(ref.shape).astype(np.float64) - ref)
+    assert np.all(err <= tol), "worst err/tol %.3g" % (err / tol).max()
+
+
+@pytest.mark.parametrize("B", [1, 2, 4, 8])
+def test_q4k_down_4096x12288(B):
+    wl = synth.WORKLOADS["q4k_down_4096x12288"]
+    inp = synth.make_inputs(wl, B=B)
+    y = host(dq.q4k_gemv(dev(inp["w"]), dev(inp["x"]), wl.N, wl.K))
+    y_ref, a_ref = oracle_rows(lambda rows: oracle.q4k_gemv(inp["w"], wl.N, wl.K, inp["x"], rows=rows),
+                               wl.N, np.arange(wl.N))
+    assert_within(y, y_ref, a_ref, "q4k down B=%d" % B)
+
+
+def test_q4k_lm_head_248320x4096_with_argmax():
+    wl = synth.WORKLOADS["q4k_lmhead_248320x4096"]
+    inp = synth.make_inputs(wl)
+    y, idx = dq.q4k_gemv(dev(inp["w"]), dev(inp["x"]), wl.N, wl.K, argmax=True)
+    y = host(y)[0]
+    idx = int(host(idx)[0])
+    y_ref, a_ref = oracle_rows(lambda rows: oracle.q4k_gemv(inp["w"], wl.N, wl.K, inp["x"], rows=rows),
+                               wl.N, np.arange(wl.N))
+    y_ref, a_ref = y_ref[0], a_ref[0]
+    assert_within(y, y_ref, a_ref, "lm head")
+    want = oracle.argmax(y_ref)
+    order = np.argsort(-y_ref, kind="stable")
+    first, second = order[0], order[1]
+    tol = oracle.gemv_tolerance(a_ref)
+    margin = y_ref[first] - y_ref[second]
+    assert margin > tol[first] + tol[second], "ambiguous argmax: top-2 margin within tolerance"
+    assert idx == want
+    assert idx == int(np.argmax(y))   # and consistent with the logits it returned
+
+
+# --- edge cases -----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("N,K,B", [(1, 256, 1), (5, 256, 3), (17, 1024, 1), (4097, 1024, 2), (33, 5120, 1),
+                                   (9, 12288, 5), (130, 4096, 7), (3, 768, 8), (64, 65536, 1), (16, 262144, 2)])
+@pytest.mark.parametrize("layout", ["aos", "soa"])
+def test_q4k_gemv_ragged_and_split_shapes(N, K, B, layout):
+    rng = np.random.default_rng(N * 7 + K + B)
+    w = synth.q4k_matrix(rng, N, K)
+    x = synth.activations(rng, B, K)
+    wl = w if layout == "aos" else oracle.q4k_repack_soa(w, N, K)
+    y = host(dq.q4k_gemv(dev(wl), dev(x), N, K, layout=layout))
+    y_ref, a_ref = oracle_rows(lambda rows: oracle.q4k_gemv(w, N, K, x, rows=rows), N, np.arange(N))
+    assert_within(y, y_ref, a_ref, "N=%d K=%d B=%d %s" % (N, K, B, layout))
+
+
+@pytest.mark.parametrize("N,K,B", [(7, 256, 1), (100, 4096, 3), (24, 65536, 1), (1, 1024, 8)])
+def test_q4k_swiglu_ragged_and_split_shapes(N, K, B):
+    rng = np.random.default_rng(N + K + B)
+    wg = synth.q4k_matrix(rng, N, K)
+    wu = synth.q4k_matrix(rng, N, K)
+    x = synth.activations(rng, B, K)
+    out = host(dq.q4k_swiglu_gemv(dev(wg), dev(wu), dev(x), N, K))
+    g, ag = oracle.q4k_gemv(wg, N, K, x)
+    u, au = oracle.q4k_gemv(wu, N, K, x)
+    ref = oracle.swiglu(g, u)
+    tol = oracle.swiglu_tolerance(g, u, ag, au)
+    assert np.all(np.abs(out.reshape(ref.shape) - ref) <= tol)
+
+
+@pytest.mark.parametrize("N,K,B", [(5, 32, 1), (33, 96, 2), (300, 4096, 4), (7, 8192, 8), (1, 64, 3)])
+def test_q8_0_gemv_ragged_shapes(N, K, B):
+    rng = np.random.default_rng(N + K + B)
+    w = synth.q8_0_matrix(rng, N, K)
+    x = synth.activations(rng, B, K)
+    y = host(dq.q8_0_gemv(dev(w), dev(x), N, K))
+    y_ref, a_ref = oracle.q8_0_gemv(w, N, K, x)
+    assert_within(y, y_ref, a_ref, "q8_0 N=%d K=%d B=%d" % (N, K, B))
+
+
+def _unit_matrix(N, nb, q_byte, m_val=0, dmin=0.0):
+    sc = np.array([1, 1, 1, 1, m_val, m_val, m_val, m_val] + [1 | (m_val << 4)] * 4, np.uint8)
+    n = N * nb
+    return synth.q4k_pack(np.ones(n, np.float16), np.full(n, dmin, np.float16), np.tile(sc, (n, 1)),
+                          np.full((n, 128), q_byte, np.uint8)).reshape(N, -1)
+
+
+@pytest.mark.parametrize("K", [256, 4096, 12288])
+def test_exact_integer_case_is_bit_exact(K):
+    # d=1, scale=1, min=0: integer weights q in [0,15]; small integer x keep
+    # every partial sum an integer below 2^24, so fp32 must equal the exact sum.
+    rng = np.random.default_rng(K)
+    N = 50
+    nblk = N * K // 256
+    sc = np.tile(np.array([1, 1, 1, 1, 0, 0, 0, 0, 1, 1, 1, 1], np.uint8), (nblk, 1))
+    w = synth.q4k_pack(np.ones(nblk, np.float16), np.zeros(nblk, np.float16), sc,
+                       rng.integers(0, 256, (nblk, 128), dtype=np.uint8)).reshape(N, -1)
+    x = rng.integers(-3, 4, (2, K)).astype(np.float32)
+    y = host(dq.q4k_gemv(dev(w), dev(x), N, K))
+    y_ref, _ = oracle.q4k_gemv(w, N, K, x)
+    assert np.array_equal(y.astype(np.float64), y_ref)
+
+
+def test_zero_quants_and_cancelling_weights():
+    K, N = 4096, 40
+    x = synth.activations(np.random.default_rng(9), 1, K)
+    # all quants 0, min 3, dmin 0.5: every weight is -1.5
+    w0 = _unit_matrix(N, K // 256, 0x00, m_val=3, dmin=0.5)
+    y0 = host(dq.q4k_gemv(dev(w0), dev(x), N, K))
+    y_ref, a_ref = oracle.q4k_gemv(w0, N, K, x)
+    assert_within(y0, y_ref, a_ref, "zero quants")
+    # q=1, scale=1, d=1, min=1, dmin=1: every weight is exactly 0, so y must be exactly 0
+    wz = _unit_matrix(N, K // 256, 0x11, m_val=1, dmin=1.0)
+    yz = host(dq.q4k_gemv(dev(wz), dev(x), N, K))
+    assert np.all(yz == 0.0)
+
+
+def test_argmax_ties_take_the_lowest_index():
+    N, K = 5000, 1024
+    rng = np.random.default_rng(21)
+    w = synth.q4k_matrix(rng, N, K)
+    x = synth.activations(rng, 1, K)
+    y_ref, _ = oracle.q4k_gemv(w, N, K, x)
+    top = int(np.argmax(y_ref[0]))
+    # copy the winning row to a lower and a higher index: three equal maxima
+    lo, hi = top // 2, min(N - 1, top + 1234)
+    w2 = w.copy()
+    w2[lo] = w[top]
+    w2[hi] = w[top]
+    y, idx = dq.q4k_gemv(dev(w2), dev(x), N, K, argmax=True)
+    y = host(y)[0]
+    assert y[lo] == y[top] == y[hi]
+    assert int(host(idx)[0]) == lo == oracle.argmax(oracle.q4k_gemv(w2, N, K, x)[0][0])
+    # all rows identical: index 0
+    w3 = np.tile(w[top], (N, 1))
+    _, idx3 = dq.q4k_gemv(dev(w3), dev(x), N, K, argmax=True)
+    assert int(host(idx3)[0]) == 0
+
+
+def test_argmax_through_split_k():
+    # few rows, long K: the plan splits K and the argmax runs in the reduction
+    N, K = 40, 131072
+    rng = np.random.default_rng(31)
+    w = synth.q4k_matrix(rng, N, K)
+    x = synth.activations(rng, 1, K)
+    y, idx = dq.q4k_gemv(dev(w), dev(x), N, K, argmax=True)
+    y_ref, a_ref = oracle.q4k_gemv(w, N, K, x)
+    assert_within(host(y), y_ref, a_ref, "split-K argmax")
+    assert int(host(idx)[0]) == oracle.argmax(y_ref[0])
+
+
+def test_soa_and_aos_outputs_are_bitwise_equal():
+    N, K = 1000, 12288
+    rng = np.random.default_rng(41)
+    w = synth.q4k_matrix(rng, N, K)
+    x = synth.activations(rng, 2, K)
+    wd = dev(w)
+    y_aos = host(dq.q4k_gemv(wd, dev(x), N, K))
+    y_soa = host(dq.q4k_gemv(dq.q4k_repack_soa(wd, N, K), dev(x), N, K, layout="soa"))
+    assert np.array_equal(y_aos.view(np.uint32), y_soa.view(np.uint32))
+
+
+def test_errors_launch_nothing_and_leave_the_stream_usable():
+    lib = dq.load_library()
+    N, K = 64, 1024
+    w = dev(synth.q4k_matrix(np.random.default_rng(1), N, K))
+    x = dev(synth.activations(np.random.default_rng(2), 1, K))
+    y = torch.full((N,), 12345.0, device="cuda")
+    s = torch.cuda.current_stream().cuda_stream
+    import ctypes
+    vp = ctypes.c_void_p
+    # K not a multiple of 256, B out of range, misaligned x, bad layout, missing workspace
+    assert lib.q4k_gemv(vp(w.data_ptr()), 0, vp(x.data_ptr()), vp(y.data_ptr()), N, K + 8, 1, None, None, 0, vp(s)) == 2
+    assert lib.q4k_gemv(vp(w.data_ptr()), 0, vp(x.data_ptr()), vp(y.data_ptr()), N, K, 9, None, None, 0, vp(s)) == 2
+    assert lib.q4k_gemv(vp(w.data_ptr()), 0, vp(x.data_ptr() + 4), vp(y.data_ptr()), N, K, 1, None, None, 0, vp(s)) == 3
+    assert lib.q4k_gemv(vp(w.data_ptr()), 3, vp(x.data_ptr()), vp(y.data_ptr()), N, K, 1, None, None, 0, vp(s)) == 5
+    idx = torch.zeros(1, dtype=torch.int64, device="cuda")
+    assert lib.q4k_gemv(vp(w.data_ptr()), 0, vp(x.data_ptr()), vp(y.data_ptr()), N, K, 1, vp(idx.data_ptr()),
+                        None, 0, vp(s)) == 4
+    torch.cuda.synchronize()
+    assert torch.all(y == 12345.0).item()          # nothing was written
+    y2 = dq.q4k_gemv(w, x, N, K)                     # a valid call still works
+    torch.cuda.synchronize()
+    assert torch.isfinite(y2).all().item()
