@@ -66,6 +66,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--rows", type=int, default=0,
+                    help="override N (a smaller case of the same kernel, e.g. for ncu captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="approximate CPU budget of the oracle baseline")
@@ -248,6 +250,9 @@ def main():
 
     wl = synth.WORKLOADS[args.workload]
     B = 1
+    if args.rows:
+        wl = synth.Workload("%s_rows%d" % (wl.name, args.rows), wl.fmt, wl.op, args.rows, wl.K, wl.batches,
+                            wl.seed, wl.x_scale)
     if wl.seed is not None and dist_on:
         wl = synth.Workload(wl.name, wl.fmt, wl.op, wl.N, wl.K, wl.batches, wl.seed + 1000 * rank,
                             wl.x_scale)

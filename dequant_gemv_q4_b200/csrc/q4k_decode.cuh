@@ -19,6 +19,10 @@
 #include <cuda_fp16.h>
 #include <cstdint>
 
+#ifndef DQ_PAIR64
+#define DQ_PAIR64 0
+#endif
+
 namespace dq {
 
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
@@ -80,11 +84,25 @@ __device__ __forceinline__ void chunk_scales(const Hdr &h, int c, float2 &sL, fl
 __device__ __forceinline__ void q4_word_weights(uint32_t w, float2 sL, float2 mL, float2 sH, float2 mH,
                                                 float2 wv[4])
 {
+#if DQ_PAIR64
+    // each pair isolated with one 64-bit AND of {w, w}, so that its two halves
+    // land in one register pair
+    const uint32_t u = w >> 16;
+    const uint64_t ww = (static_cast<uint64_t>(w) << 32) | w;
+    const uint64_t uu = (static_cast<uint64_t>(u) << 32) | u;
+    const uint64_t a = ww & 0x00000F000000000Full, b = uu & 0x00000F000000000Full;
+    const uint64_t c = ww & 0x0000F000000000F0ull, e = uu & 0x0000F000000000F0ull;
+    wv[0] = __ffma2_rn(*reinterpret_cast<const float2 *>(&a), sL, mL);
+    wv[1] = __ffma2_rn(*reinterpret_cast<const float2 *>(&b), sL, mL);
+    wv[2] = __ffma2_rn(*reinterpret_cast<const float2 *>(&c), sH, mH);
+    wv[3] = __ffma2_rn(*reinterpret_cast<const float2 *>(&e), sH, mH);
+#else
     const uint32_t u = w >> 16;
     wv[0] = __ffma2_rn(f2(__uint_as_float(w & 0xFu), __uint_as_float(w & 0xF00u)), sL, mL);
     wv[1] = __ffma2_rn(f2(__uint_as_float(u & 0xFu), __uint_as_float(u & 0xF00u)), sL, mL);
     wv[2] = __ffma2_rn(f2(__uint_as_float(w & 0xF0u), __uint_as_float(w & 0xF000u)), sH, mH);
     wv[3] = __ffma2_rn(f2(__uint_as_float(u & 0xF0u), __uint_as_float(u & 0xF000u)), sH, mH);
+#endif
 }
 
 }  // namespace dq

@@ -102,25 +102,37 @@ struct Pow2Ceil<1> {
     static constexpr int value = 1;
 };
 
-// Issues the bulk copies of slot-sequence element i of one warp into ring slot
-// `slot`: K-chunk kc of stream st of tile t (rows row0 .. row0+rows-1).
+// Position of a warp in its slot sequence: tile tk (of this warp's tiles),
+// weight stream st, K-chunk kcl (relative to the split's first chunk).
+struct Cursor {
+    long long tk;
+    int st;
+    int kcl;
+    __device__ __forceinline__ void advance(int nch, int ns)
+    {
+        if (++kcl == nch) {
+            kcl = 0;
+            if (++st == ns) {
+                st = 0;
+                ++tk;
+            }
+        }
+    }
+};
+
+// Issues the bulk copies of one slot: K-chunk (c_begin + cur.kcl) of stream
+// cur.st of tile t0 + cur.tk * tstride, into ring slot `slot`.
 template <int LPR, int R>
-__device__ __forceinline__ void issue_slot(const Q4KParams &p, long long i, int slot, long long per_tile, int nch,
-                                           int c_begin, long long t0, long long tstride, uint32_t ring_s,
-                                           uint32_t bars_s)
+__device__ __forceinline__ void issue_slot(const Q4KParams &p, const Cursor &cur, int slot, int c_begin, long long t0,
+                                           long long tstride, uint32_t ring_s, uint32_t bars_s)
 {
     using G = Geo<LPR, R>;
     const long long row_bytes_g = static_cast<long long>(p.nb) * kQ4KBlockBytes;
-    const long long tk = i / per_tile;
-    const int rem = static_cast<int>(i - tk * per_tile);
-    const int st = rem / nch;
-    const int kc = c_begin + rem % nch;
-    const long long tile = t0 + tk * tstride;
-    const long long row0 = tile * G::TR;
+    const long long row0 = (t0 + cur.tk * tstride) * G::TR;
     const int rows = static_cast<int>(min(static_cast<long long>(G::TR), p.N - row0));
-    const int kb0 = kc * LPR;
+    const int kb0 = (c_begin + cur.kcl) * LPR;
     const int nblk = min(LPR, p.nb - kb0);
-    const uint8_t *src = (st == 0 ? p.w[0] : p.w[1]) + row0 * row_bytes_g + static_cast<long long>(kb0) * kQ4KBlockBytes;
+    const uint8_t *src = (cur.st == 0 ? p.w[0] : p.w[1]) + row0 * row_bytes_g + static_cast<long long>(kb0) * kQ4KBlockBytes;
     const uint32_t dst = ring_s + slot * G::SLOT_BYTES;
     const uint32_t bar = bars_s + slot * 8;
     mbar_arrive_expect_tx(bar, static_cast<uint32_t>(rows * nblk * kQ4KBlockBytes));
@@ -138,7 +150,7 @@ __device__ __forceinline__ void issue_slot(const Q4KParams &p, long long i, int 
     }
 }
 
-template <int LPR, int B, int NS, int R>
+template <int LPR, int B, int NS, int R, bool SOA>
 __global__ void __launch_bounds__(kMaxThreads, 1) q4k_gemv_kernel(const Q4KParams p)
 {
     using G = Geo<LPR, R>;
@@ -173,20 +185,24 @@ __global__ void __launch_bounds__(kMaxThreads, 1) q4k_gemv_kernel(const Q4KParam
     const uint32_t my_bars_s = smem_u32(bars + warp * p.depth);
     ArgmaxCand *red = reinterpret_cast<ArgmaxCand *>(ring + static_cast<size_t>(nwarps) * p.depth * G::SLOT_BYTES);
 
-    // this warp's tiles
+    // this warp's tiles: t0, t0 + tstride, ...
     const long long tstride = static_cast<long long>(p.ctas_per_split) * nwarps;
     const long long t0 = static_cast<long long>(cj) * nwarps + warp;
     const long long ntiles_w = (t0 < p.tiles) ? (p.tiles - t0 + tstride - 1) / tstride : 0;
-    const long long per_tile = static_cast<long long>(NS) * nch;
-    const long long total = ntiles_w * per_tile;
+    const long long total = ntiles_w * NS * nch;
 
+    // producer cursor (meaningful in lane 0 only, advanced in every lane)
+    Cursor pc{0, 0, 0};
+    long long issued = 0;
     if (lane == 0) {
         for (int s = 0; s < p.depth; ++s)
             mbar_init(my_bars_s + s * 8, 1);
         mbar_fence_init();
-        const long long pre = min(static_cast<long long>(p.depth), total);
-        for (long long i = 0; i < pre; ++i)
-            issue_slot<LPR, R>(p, i, static_cast<int>(i), per_tile, nch, c_begin, t0, tstride, my_ring_s, my_bars_s);
+    }
+    for (int s = 0; s < p.depth && issued < total; ++s, ++issued) {
+        if (lane == 0)
+            issue_slot<LPR, R>(p, pc, s, c_begin, t0, tstride, my_ring_s, my_bars_s);
+        pc.advance(nch, NS);
     }
 
     // stage this split's activations (fp32, 16-byte padded per super-block)
@@ -199,14 +215,11 @@ __global__ void __launch_bounds__(kMaxThreads, 1) q4k_gemv_kernel(const Q4KParam
             const int q = rem & 63;
             const float4 *src = reinterpret_cast<const float4 *>(
                 p.x + static_cast<long long>(b) * p.K + static_cast<long long>(kb_begin + kbl) * 256) + q;
-            float4 v = ldg_nc_f4(src);
-            *reinterpret_cast<float4 *>(xs + (b * nbs + kbl) * kXBlockPitch + q * 16) = v;
+            *reinterpret_cast<float4 *>(xs + (b * nbs + kbl) * kXBlockPitch + q * 16) = ldg_nc_f4(src);
         }
     }
     __syncthreads();
-    __syncwarp();
 
-    const uint32_t xs_s = smem_u32(xs);
     float best_v = -INFINITY;
     long long best_i = 0x7fffffffffffffffLL;
     bool failed = false;
@@ -215,24 +228,19 @@ __global__ void __launch_bounds__(kMaxThreads, 1) q4k_gemv_kernel(const Q4KParam
     float2 accL[R][B], accH[R][B];
     float gsum[NS == 2 ? MP : 1];  // stream-0 sums kept for the SwiGLU epilogue
 
-    for (long long i = 0; i < total; ++i) {
-        const int slot = static_cast<int>(i % p.depth);
-        const uint32_t parity = static_cast<uint32_t>((i / p.depth) & 1);
+    Cursor cc{0, 0, 0};
+    int slot = 0;
+    uint32_t parity = 0;
+    for (; consumed < total; ++consumed) {
         const bool ok = mbar_wait_bounded(my_bars_s + slot * 8, parity, p.err);
         if (!__all_sync(0xffffffffu, ok)) {
             failed = true;
             break;
         }
-        consumed = i + 1;
-        const long long tk = i / per_tile;
-        const int rem = static_cast<int>(i - tk * per_tile);
-        const int st = rem / nch;
-        const int kcl = rem % nch;
-        const int kc = c_begin + kcl;
-        const long long tile = t0 + tk * tstride;
-        const long long row0 = tile * G::TR;
+        const int kc = c_begin + cc.kcl;
+        const long long row0 = (t0 + cc.tk * tstride) * G::TR;
 
-        if (kcl == 0) {
+        if (cc.kcl == 0) {
 #pragma unroll
             for (int r = 0; r < R; ++r)
 #pragma unroll
@@ -245,23 +253,23 @@ __global__ void __launch_bounds__(kMaxThreads, 1) q4k_gemv_kernel(const Q4KParam
         const int kb0 = kc * LPR;
         const int nblk = min(LPR, p.nb - kb0);
         if (l < nblk) {
-            const uint32_t slot_s = my_ring_s + slot * G::SLOT_BYTES + rg * G::RG_PITCH;
+            const uint8_t *slot_p = my_ring + slot * G::SLOT_BYTES + rg * G::RG_PITCH;
             // byte offsets of this lane's header and quant slices within a row of the slot
-            uint32_t hdr_off, qs_off0, qs_step;
-            if (p.soa) {
-                hdr_off = 16u * l;
-                qs_off0 = 16u * nblk + 16u * l;
-                qs_step = 16u * nblk;
+            int hdr_off, qs_off0, qs_step;
+            if constexpr (SOA) {
+                hdr_off = 16 * l;
+                qs_off0 = 16 * nblk + 16 * l;
+                qs_step = 16 * nblk;
             } else {
                 hdr_off = kQ4KBlockBytes * l;
-                qs_off0 = hdr_off + 16u;
-                qs_step = 16u;
+                qs_off0 = hdr_off + 16;
+                qs_step = 16;
             }
             Hdr hd[R];
 #pragma unroll
             for (int r = 0; r < R; ++r)
-                hd[r] = decode_hdr(lds128(slot_s + r * G::ROW_BYTES + hdr_off));
-            const uint32_t xblk = xs_s + (kb0 - kb_begin + l) * kXBlockPitch;
+                hd[r] = decode_hdr(*reinterpret_cast<const uint4 *>(slot_p + r * G::ROW_BYTES + hdr_off));
+            const uint8_t *xblk = xs + (kb0 - kb_begin + l) * kXBlockPitch;
 
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -275,15 +283,15 @@ __global__ void __launch_bounds__(kMaxThreads, 1) q4k_gemv_kernel(const Q4KParam
                     uint4 q[R];
 #pragma unroll
                     for (int r = 0; r < R; ++r)
-                        q[r] = lds128(slot_s + r * G::ROW_BYTES + qs_off0 + s * qs_step);
-                    const uint32_t xoffL = (64 * c + 16 * h) * 4;
+                        q[r] = *reinterpret_cast<const uint4 *>(slot_p + r * G::ROW_BYTES + qs_off0 + s * qs_step);
+                    const int xoffL = (64 * c + 16 * h) * 4;
 #pragma unroll
                     for (int t = 0; t < 4; ++t) {
 #pragma unroll
                         for (int b = 0; b < B; ++b) {
-                            const uint32_t xb = xblk + b * nbs * kXBlockPitch + xoffL + 16 * t;
-                            const float4 xl = lds128f(xb);
-                            const float4 xh = lds128f(xb + 128);
+                            const uint8_t *xb = xblk + b * nbs * kXBlockPitch + xoffL + 16 * t;
+                            const float4 xl = *reinterpret_cast<const float4 *>(xb);
+                            const float4 xh = *reinterpret_cast<const float4 *>(xb + 128);
 #pragma unroll
                             for (int r = 0; r < R; ++r) {
                                 const uint32_t wv = (t == 0) ? q[r].x : (t == 1) ? q[r].y : (t == 2) ? q[r].z : q[r].w;
@@ -296,12 +304,24 @@ __global__ void __launch_bounds__(kMaxThreads, 1) q4k_gemv_kernel(const Q4KParam
         }
 
         __syncwarp();
-        if (lane == 0 && i + p.depth < total) {
-            fence_proxy_async_smem();
-            issue_slot<LPR, R>(p, i + p.depth, slot, per_tile, nch, c_begin, t0, tstride, my_ring_s, my_bars_s);
+        if (issued < total) {
+            if (lane == 0) {
+                fence_proxy_async_smem();
+                issue_slot<LPR, R>(p, pc, slot, c_begin, t0, tstride, my_ring_s, my_bars_s);
+            }
+            pc.advance(nch, NS);
+            ++issued;
         }
 
-        if (kcl == nch - 1) {
+        const int cur_st = cc.st;
+        const bool last_chunk = (cc.kcl == nch - 1);
+        cc.advance(nch, NS);
+        if (++slot == p.depth) {
+            slot = 0;
+            parity ^= 1u;
+        }
+
+        if (last_chunk) {
             // end of this stream's K range for the tile: reduce across the row group
             float v[MP];
 #pragma unroll
@@ -335,7 +355,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) q4k_gemv_kernel(const Q4KParam
             }
 
             if constexpr (NS == 2) {
-                if (st == 0) {
+                if (cur_st == 0) {
 #pragma unroll
                     for (int j = 0; j < VPL; ++j)
                         gsum[j] = v[j];
@@ -382,11 +402,12 @@ __global__ void __launch_bounds__(kMaxThreads, 1) q4k_gemv_kernel(const Q4KParam
 
     if (failed) {
         // the copies already issued into this warp's ring must land before the CTA exits
-        const long long issued = min(total, consumed + p.depth);
         for (long long i = consumed; i < issued; ++i) {
-            const int slot = static_cast<int>(i % p.depth);
-            const uint32_t parity = static_cast<uint32_t>((i / p.depth) & 1);
             mbar_wait_bounded(my_bars_s + slot * 8, parity, nullptr);
+            if (++slot == p.depth) {
+                slot = 0;
+                parity ^= 1u;
+            }
         }
     }
 
@@ -486,7 +507,7 @@ Q4KPlan q4k_plan(long long N, int K, int B, int NS, int soa, int sm_count, int s
 template <int LPR, int B, int NS>
 static cudaError_t launch_one(const Q4KParams &p, const Q4KPlan &pl, cudaStream_t s)
 {
-    auto k = q4k_gemv_kernel<LPR, B, NS, 2>;
+    auto k = p.soa ? q4k_gemv_kernel<LPR, B, NS, 2, true> : q4k_gemv_kernel<LPR, B, NS, 2, false>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
     if (e != cudaSuccess)
         return e;
