@@ -31,7 +31,7 @@ Q8_0_BLOCK_ELEMS, Q8_0_BLOCK_BYTES = 32, 34
 
 EXPORTED = ("q8_0_gemv", "q4k_gemv", "q4k_swiglu_gemv", "q4k_repack_soa", "dq_workspace_bytes",
             "q8_0_dequant", "q4k_dequant", "dq_status_string", "dq_last_cuda_error",
-            "dq_device_error")
+            "dq_device_error", "q4k_gemv_noalloc", "dq_noalloc_scratch_bytes")
 
 
 class DQError(RuntimeError):
@@ -70,6 +70,7 @@ def load_library(path: str = LIB_PATH):
             "q8_0_dequant": [p, p, i64, i64, p],
             "q4k_dequant": [p, i32, p, i64, i64, p],
             "dq_device_error": [p, i32, p],
+            "q4k_gemv_noalloc": [p, i32, p, p, i64, i64, i32, p, p],
         }
         for name, args in sigs.items():
             f = getattr(lib, name)
@@ -79,6 +80,8 @@ def load_library(path: str = LIB_PATH):
         lib.dq_workspace_bytes.restype = sz
         lib.dq_status_string.argtypes = [i32]
         lib.dq_status_string.restype = ctypes.c_char_p
+        lib.dq_noalloc_scratch_bytes.argtypes = []
+        lib.dq_noalloc_scratch_bytes.restype = sz
         lib.dq_last_cuda_error.argtypes = []
         lib.dq_last_cuda_error.restype = i32
         _lib = lib
@@ -197,6 +200,38 @@ def q4k_gemv(w, x, N: int, K: int, layout="aos", y=None, argmax: bool = False, w
                                     ip, wsp, wsn, _stream(stream)))
     out = y.view(N) if one_d else y.view(B, N)
     return (out, idx) if argmax else out
+
+
+def q4k_gemv_noalloc(w, x, N: int, K: int, layout="aos", y=None, argmax: bool = False, stream=None):
+    """q4k_gemv through the entry point that allocates nothing.
+
+    For callers that cannot allocate device memory: the library's own fixed
+    scratch array (dq_noalloc_scratch_bytes()) replaces the workspace, so only
+    y (and the argmax slot, when asked for) are passed.  Calls sharing that
+    array must not overlap on the GPU.
+    """
+    torch = _torch()
+    lib = load_library()
+    one_d = x.dim() == 1
+    x2 = _x2d(x, K)
+    B = x2.shape[0]
+    wp = _weights(w, "w", N, K, Q4K_BLOCK_ELEMS, Q4K_BLOCK_BYTES)
+    if y is None:
+        y = torch.empty((B, N), dtype=torch.float32, device=x.device)
+    yp = _dev(y, "y", torch.float32)
+    idx = None
+    ip = ctypes.c_void_p(0)
+    if argmax:
+        idx = torch.empty(1, dtype=torch.int64, device=x.device)
+        ip = ctypes.c_void_p(idx.data_ptr())
+    _check("q4k_gemv_noalloc", lib.q4k_gemv_noalloc(wp, _layout(layout), ctypes.c_void_p(x2.data_ptr()), yp,
+                                                    N, K, B, ip, _stream(stream)))
+    out = y.view(N) if one_d else y.view(B, N)
+    return (out, idx) if argmax else out
+
+
+def dq_noalloc_scratch_bytes() -> int:
+    return int(load_library().dq_noalloc_scratch_bytes())
 
 
 def q4k_swiglu_gemv(w_gate, w_up, x, N: int, K: int, layout="aos", out=None, workspace=None,

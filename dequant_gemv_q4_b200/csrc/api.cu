@@ -3,6 +3,7 @@
 // Nothing here allocates device memory; every pointer comes from the caller.
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <cuda_runtime.h>
 
 #include "dq_common.cuh"
@@ -148,7 +149,58 @@ dq_status q4k_common(const void *w0, const void *w1, int layout, const float *x,
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Scratch for q4k_gemv_noalloc: a fixed device array in this library's own
+// image, for callers that cannot allocate device memory themselves.  Every GPU
+// that loads the library holds it until the process exits.
+// ---------------------------------------------------------------------------
+#define DQ_NOALLOC_SCRATCH_BYTES (4u << 20)
+static __device__ __align__(256) uint8_t g_noalloc_scratch[DQ_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+std::mutex g_noalloc_mutex;
+void *g_noalloc_ptr[64] = {};
+
+// Device address of g_noalloc_scratch on the current device.  The symbol's
+// host-side name is only a stand-in, so the address is looked up once per
+// device (with that device current) and cached.
+dq_status noalloc_scratch(int device, void **ptr)
+{
+    if (device < 0 || device >= 64)
+        return DQ_ERR_ARG;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[device]) {
+        void *p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess)
+            return cuda_fail(e);
+        g_noalloc_ptr[device] = p;
+    }
+    *ptr = g_noalloc_ptr[device];
+    return DQ_OK;
+}
+
+}  // namespace
+
 extern "C" {
+
+dq_status q4k_gemv_noalloc(const void *w, int layout, const float *x, float *y, int64_t N, int64_t K, int B,
+                           int64_t *argmax_out, void *stream)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    void *scratch = nullptr;
+    dq_status st = noalloc_scratch(dev, &scratch);
+    if (st != DQ_OK)
+        return st;
+    return q4k_common(w, nullptr, layout, x, y, N, K, B, 1, argmax_out, scratch, DQ_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+size_t dq_noalloc_scratch_bytes(void) { return DQ_NOALLOC_SCRATCH_BYTES; }
+
 
 dq_status q4k_gemv(const void *w, int layout, const float *x, float *y, int64_t N, int64_t K, int B,
                    int64_t *argmax_out, void *workspace, size_t ws_bytes, void *stream)

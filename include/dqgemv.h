@@ -145,6 +145,30 @@ size_t dq_workspace_bytes(int op, int64_t N, int64_t K, int B, int with_argmax);
 dq_status q8_0_dequant(const void *w, float *out, int64_t N, int64_t K, void *stream);
 dq_status q4k_dequant(const void *w, int layout, float *out, int64_t N, int64_t K, void *stream);
 
+/*
+ * q4k_gemv without a workspace argument, for callers that cannot allocate
+ * device memory (code that runs where no allocator is reachable, or that must
+ * not allocate once set up, such as a decode loop whose memory budget is fixed
+ * in advance).  No counterpart on the pages: this is a packaging of q4k_gemv.
+ *   Arguments and results are exactly those of q4k_gemv minus the workspace.
+ *   The scratch it needs (split-K partial sums, argmax candidates) lives in a
+ *   fixed array of dq_noalloc_scratch_bytes() bytes (4 MiB) inside the library,
+ *   held by every GPU that loads the library until the process exits.  A shape
+ *   whose q4k_gemv workspace (dq_workspace_bytes) is larger than that returns
+ *   DQ_ERR_WORKSPACE and launches nothing.
+ *   The first call on each device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   It never calls cudaMalloc, cudaFree or any allocating routine.
+ *   Every call shares the one array and nothing in it needs to start at zero;
+ *   calls that may overlap on the GPU (other streams, other host threads)
+ *   race on it, so serialize them.
+ */
+dq_status q4k_gemv_noalloc(const void *w, int layout, const float *x, float *y, int64_t N, int64_t K,
+                           int B, int64_t *argmax_out, void *stream);
+
+/* Size in bytes of the fixed scratch array q4k_gemv_noalloc uses. */
+size_t dq_noalloc_scratch_bytes(void);
+
 /* Static string naming a status code. */
 const char *dq_status_string(int status);
 
