@@ -30,7 +30,8 @@ int *device_error_flag(int device)
 
 // ---------------------------------------------------------------------------
 // Q4_K debug dequant: one thread per (row, super-block, 16-byte quant slice)
-// writes that slice's 32 weights with the GEMV's own weight formation.
+// writes that slice's 32 weights with the GEMV's own weight formation
+// (q4k_decode.cuh); vector stores when `out` is 16-byte aligned.
 // ---------------------------------------------------------------------------
 
 // Byte offset within a row of the header (byte < 16) or of quant slice s of
@@ -53,6 +54,7 @@ __global__ void q4k_dequant_kernel(const uint8_t *__restrict__ w, int soa, float
     const int nb = K / kQ4KBlockElems;
     const long long total = N * nb * 8;
     const long long row_bytes = static_cast<long long>(nb) * kQ4KBlockBytes;
+    const bool vec = (reinterpret_cast<uintptr_t>(out) & 15) == 0;
     for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
          i += static_cast<long long>(gridDim.x) * blockDim.x) {
         const int s = static_cast<int>(i % 8);
@@ -65,60 +67,26 @@ __global__ void q4k_dequant_kernel(const uint8_t *__restrict__ w, int soa, float
                                 : row + static_cast<long long>(kb) * kQ4KBlockBytes + 16 + 16 * s;
         const Hdr h = decode_hdr(*reinterpret_cast<const uint4 *>(hp));
         const uint4 q = *reinterpret_cast<const uint4 *>(qp);
-        const int c = s / 2;
-        float2 sL, mL, sH, mH;
-        chunk_scales(h, c, sL, mL, sH, mH);
-        const long long L = n * K + static_cast<long long>(kb) * kQ4KBlockElems + 64 * c + 16 * (s % 2);
+        const ChunkScales cs = chunk_scales(h, s / 2);
+        // lo weights of this slice start at L, hi weights at L + 32
+        const long long L = n * K + static_cast<long long>(kb) * kQ4KBlockElems + 64 * (s / 2) + 16 * (s % 2);
         const uint32_t words[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
             float2 wv[4];
-            q4_word_weights(words[t], sL, mL, sH, mH, wv);
-            float4 lo = make_float4(wv[0].x * 0x1p64f, wv[0].y * 0x1p64f, wv[1].x * 0x1p64f, wv[1].y * 0x1p64f);
-            float4 hi = make_float4(wv[2].x * 0x1p64f, wv[2].y * 0x1p64f, wv[3].x * 0x1p64f, wv[3].y * 0x1p64f);
-            *reinterpret_cast<float4 *>(out + L + 4 * t) = lo;
-            *reinterpret_cast<float4 *>(out + L + 32 + 4 * t) = hi;
-        }
-    }
-}
-
-// out may be any 4-byte aligned pointer; the float4 stores above need 16-byte
-// alignment, so an unaligned `out` goes through this scalar variant.
-__global__ void q4k_dequant_kernel_scalar(const uint8_t *__restrict__ w, int soa, float *__restrict__ out,
-                                          long long N, int K)
-{
-    const int nb = K / kQ4KBlockElems;
-    const long long total = N * nb * 8;
-    const long long row_bytes = static_cast<long long>(nb) * kQ4KBlockBytes;
-    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
-         i += static_cast<long long>(gridDim.x) * blockDim.x) {
-        const int s = static_cast<int>(i % 8);
-        const long long blk = i / 8;
-        const int kb = static_cast<int>(blk % nb);
-        const long long n = blk / nb;
-        const uint8_t *row = w + n * row_bytes;
-        const uint8_t *hp = soa ? row + soa_hdr_off(nb, kb) : row + static_cast<long long>(kb) * kQ4KBlockBytes;
-        const uint8_t *qp = soa ? row + soa_slice_off(nb, kb, s)
-                                : row + static_cast<long long>(kb) * kQ4KBlockBytes + 16 + 16 * s;
-        const Hdr h = decode_hdr(*reinterpret_cast<const uint4 *>(hp));
-        const uint4 q = *reinterpret_cast<const uint4 *>(qp);
-        const int c = s / 2;
-        float2 sL, mL, sH, mH;
-        chunk_scales(h, c, sL, mL, sH, mH);
-        const long long L = n * K + static_cast<long long>(kb) * kQ4KBlockElems + 64 * c + 16 * (s % 2);
-        const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+            q4_word_weights(words[t], cs, wv);
+            if (vec) {
+                *reinterpret_cast<float4 *>(out + L + 4 * t) =
+                    make_float4(wv[0].x * 0x1p64f, wv[1].x * 0x1p64f, wv[2].x * 0x1p64f, wv[3].x * 0x1p64f);
+                *reinterpret_cast<float4 *>(out + L + 32 + 4 * t) =
+                    make_float4(wv[0].y * 0x1p64f, wv[1].y * 0x1p64f, wv[2].y * 0x1p64f, wv[3].y * 0x1p64f);
+            } else {
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-            float2 wv[4];
-            q4_word_weights(words[t], sL, mL, sH, mH, wv);
-            out[L + 4 * t + 0] = wv[0].x * 0x1p64f;
-            out[L + 4 * t + 1] = wv[0].y * 0x1p64f;
-            out[L + 4 * t + 2] = wv[1].x * 0x1p64f;
-            out[L + 4 * t + 3] = wv[1].y * 0x1p64f;
-            out[L + 32 + 4 * t + 0] = wv[2].x * 0x1p64f;
-            out[L + 32 + 4 * t + 1] = wv[2].y * 0x1p64f;
-            out[L + 32 + 4 * t + 2] = wv[3].x * 0x1p64f;
-            out[L + 32 + 4 * t + 3] = wv[3].y * 0x1p64f;
+                for (int k = 0; k < 4; ++k) {
+                    out[L + 4 * t + k] = wv[k].x * 0x1p64f;
+                    out[L + 32 + 4 * t + k] = wv[k].y * 0x1p64f;
+                }
+            }
         }
     }
 }
@@ -136,10 +104,7 @@ static int grid_for(long long work, int block)
 cudaError_t q4k_dequant_launch(const uint8_t *w, int soa, float *out, long long N, int K, cudaStream_t s)
 {
     const long long total = N * (K / kQ4KBlockElems) * 8;
-    if ((reinterpret_cast<uintptr_t>(out) & 15) == 0)
-        q4k_dequant_kernel<<<grid_for(total, 256), 256, 0, s>>>(w, soa, out, N, K);
-    else
-        q4k_dequant_kernel_scalar<<<grid_for(total, 256), 256, 0, s>>>(w, soa, out, N, K);
+    q4k_dequant_kernel<<<grid_for(total, 256), 256, 0, s>>>(w, soa, out, N, K);
     return cudaGetLastError();
 }
 

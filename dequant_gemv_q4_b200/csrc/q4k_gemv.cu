@@ -40,22 +40,27 @@
 
 namespace dq {
 
-// One quant word: form its eight weights and accumulate weight*x (low nibbles
-// into accL, high nibbles into accH).  xl = x[L+4t .. L+4t+3], xh = x[H+4t ..].
-__device__ __forceinline__ void q4_word(uint32_t w, float2 sL, float2 mL, float2 sH, float2 mH,
-                                        float4 xl, float4 xh, float2 &accL, float2 &accH)
+// One quant word (bytes 4t..4t+3 of a 16-byte slice): form its eight weights
+// and accumulate weight*x.  xa = {x[L+4t], x[H+4t], x[L+4t+1], x[H+4t+1]},
+// xb = the same for bytes 4t+2, 4t+3 (x is staged in (lo, hi) pairs).
+__device__ __forceinline__ void q4_word(uint32_t w, const ChunkScales &cs, float4 xa, float4 xb, float2 &acc0,
+                                        float2 &acc1)
 {
     float2 wv[4];
-    q4_word_weights(w, sL, mL, sH, mH, wv);
-    accL = __ffma2_rn(wv[0], f2(xl.x, xl.y), accL);
-    accH = __ffma2_rn(wv[2], f2(xh.x, xh.y), accH);
-    accL = __ffma2_rn(wv[1], f2(xl.z, xl.w), accL);
-    accH = __ffma2_rn(wv[3], f2(xh.z, xh.w), accH);
+    q4_word_weights(w, cs, wv);
+    acc0 = __ffma2_rn(wv[0], f2(xa.x, xa.y), acc0);
+    acc1 = __ffma2_rn(wv[1], f2(xa.z, xa.w), acc1);
+    acc0 = __ffma2_rn(wv[2], f2(xb.x, xb.y), acc0);
+    acc1 = __ffma2_rn(wv[3], f2(xb.z, xb.w), acc1);
 }
 
 constexpr int kMaxWarps = 8;
-constexpr int kMaxThreads = kMaxWarps * 32;
-constexpr int kXBlockPitch = 1040;  // bytes per staged 256-float block of x (16 B pad)
+
+// x of one super-block is staged as 8 slices x 8 float4, float4 k of slice
+// s = 2c+h holding {x[L+2k], x[H+2k], x[L+2k+1], x[H+2k+1]} (L = 64c+16h,
+// H = L+32): the (lo, hi) weight pairs of quant bytes 2k and 2k+1.  16 bytes
+// of padding per super-block keep the lanes' reads free of bank conflicts.
+constexpr int kXBlockPitch = 1040;
 
 template <int LPR, int R>
 struct Geo {
@@ -102,46 +107,52 @@ struct Pow2Ceil<1> {
     static constexpr int value = 1;
 };
 
-// Position of a warp in its slot sequence: tile tk (of this warp's tiles),
-// weight stream st, K-chunk kcl (relative to the split's first chunk).
+// Position of a warp in its slot sequence: the tile's first row row0, weight
+// stream st, K-chunk kcl (relative to the split's first chunk).  row0 moves by
+// the warp's tile stride once every stream and chunk of a tile are done.
 struct Cursor {
-    long long tk;
+    long long row0;
     int st;
     int kcl;
-    __device__ __forceinline__ void advance(int nch, int ns)
+    __device__ __forceinline__ bool advance(int nch, int ns, long long row_step)
     {
         if (++kcl == nch) {
             kcl = 0;
             if (++st == ns) {
                 st = 0;
-                ++tk;
+                row0 += row_step;
+                return true;
             }
         }
+        return false;
     }
 };
 
-// Issues the bulk copies of one slot: K-chunk (c_begin + cur.kcl) of stream
-// cur.st of tile t0 + cur.tk * tstride, into ring slot `slot`.
+// Issues the bulk copies of one slot (K-chunk c_begin + cur.kcl of stream
+// cur.st of the tile at cur.row0) into ring slot `slot`.
 template <int LPR, int R>
-__device__ __forceinline__ void issue_slot(const Q4KParams &p, const Cursor &cur, int slot, int c_begin, long long t0,
-                                           long long tstride, uint32_t ring_s, uint32_t bars_s)
+__device__ __forceinline__ void issue_slot(const Q4KParams &p, const Cursor &cur, int slot, int c_begin,
+                                           uint32_t ring_s, uint32_t bars_s)
 {
     using G = Geo<LPR, R>;
     const long long row_bytes_g = static_cast<long long>(p.nb) * kQ4KBlockBytes;
-    const long long row0 = (t0 + cur.tk * tstride) * G::TR;
-    const int rows = static_cast<int>(min(static_cast<long long>(G::TR), p.N - row0));
+    const int rows = static_cast<int>(min(static_cast<long long>(G::TR), p.N - cur.row0));
     const int kb0 = (c_begin + cur.kcl) * LPR;
     const int nblk = min(LPR, p.nb - kb0);
-    const uint8_t *src = (cur.st == 0 ? p.w[0] : p.w[1]) + row0 * row_bytes_g + static_cast<long long>(kb0) * kQ4KBlockBytes;
+    const uint8_t *src = (cur.st == 0 ? p.w[0] : p.w[1]) + cur.row0 * row_bytes_g + kb0 * kQ4KBlockBytes;
     const uint32_t dst = ring_s + slot * G::SLOT_BYTES;
     const uint32_t bar = bars_s + slot * 8;
     mbar_arrive_expect_tx(bar, static_cast<uint32_t>(rows * nblk * kQ4KBlockBytes));
     if (nblk == p.nb && p.nb == LPR) {
-        // whole rows, contiguous in global memory: one copy per row group
-        for (int g = 0; g * R < rows; ++g) {
-            const int gr = min(R, rows - g * R);
-            bulk_g2s(dst + g * G::RG_PITCH, src + static_cast<long long>(g) * R * row_bytes_g,
-                     static_cast<uint32_t>(gr * G::ROW_BYTES), bar);
+        if (G::PAD == 0) {
+            // whole rows of a contiguous tile, laid out without padding: one copy
+            bulk_g2s(dst, src, static_cast<uint32_t>(rows * G::ROW_BYTES), bar);
+        } else {
+            for (int g = 0; g * R < rows; ++g) {
+                const int gr = min(R, rows - g * R);
+                bulk_g2s(dst + g * G::RG_PITCH, src + static_cast<long long>(g) * R * row_bytes_g,
+                         static_cast<uint32_t>(gr * G::ROW_BYTES), bar);
+            }
         }
     } else {
         for (int r = 0; r < rows; ++r)
@@ -150,9 +161,10 @@ __device__ __forceinline__ void issue_slot(const Q4KParams &p, const Cursor &cur
     }
 }
 
-template <int LPR, int B, int NS, int R, bool SOA>
-__global__ void __launch_bounds__(kMaxThreads, 1) q4k_gemv_kernel(const Q4KParams p)
+template <int LPR, int B, int NS, bool SOA>
+__global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_kernel(const Q4KParams p)
 {
+    constexpr int R = 2;
     using G = Geo<LPR, R>;
     constexpr int MV = R * B;                         // values per lane per stream
     constexpr int MP = Pow2Ceil<MV>::value;           // padded to a power of two
@@ -190,9 +202,28 @@ __global__ void __launch_bounds__(kMaxThreads, 1) q4k_gemv_kernel(const Q4KParam
     const long long t0 = static_cast<long long>(cj) * nwarps + warp;
     const long long ntiles_w = (t0 < p.tiles) ? (p.tiles - t0 + tstride - 1) / tstride : 0;
     const long long total = ntiles_w * NS * nch;
+    const long long row_step = tstride * G::TR;
 
-    // producer cursor (meaningful in lane 0 only, advanced in every lane)
-    Cursor pc{0, 0, 0};
+    // After the row-group reduction this lane holds value indices
+    // off .. off + VPL - 1 (value index = r * B + b); only `writer` lanes store.
+    int off = 0;
+    bool writer = true;
+    {
+        int m = MP;
+#pragma unroll
+        for (int o = LPR / 2; o >= 1; o >>= 1) {
+            if (m > 1) {
+                if (l & o)
+                    off += m / 2;
+                m /= 2;
+            } else if (l & o) {
+                writer = false;
+            }
+        }
+    }
+
+    // producer cursor (used by lane 0, advanced in every lane)
+    Cursor pc{t0 * G::TR, 0, 0};
     long long issued = 0;
     if (lane == 0) {
         for (int s = 0; s < p.depth; ++s)
@@ -201,21 +232,44 @@ __global__ void __launch_bounds__(kMaxThreads, 1) q4k_gemv_kernel(const Q4KParam
     }
     for (int s = 0; s < p.depth && issued < total; ++s, ++issued) {
         if (lane == 0)
-            issue_slot<LPR, R>(p, pc, s, c_begin, t0, tstride, my_ring_s, my_bars_s);
-        pc.advance(nch, NS);
+            issue_slot<LPR, R>(p, pc, s, c_begin, my_ring_s, my_bars_s);
+        pc.advance(nch, NS, row_step);
     }
 
-    // stage this split's activations (fp32, 16-byte padded per super-block)
+    // stage this split's activations in (lo, hi) pairs (fp32, padded per super-block);
+    // each thread keeps kStageBatch loads in flight before storing
     {
+        constexpr int kStageBatch = 8;
         const int per_b = nbs * 64;  // float4 per batch row
-        for (int idx = threadIdx.x; idx < B * per_b; idx += blockDim.x) {
-            const int b = idx / per_b;
-            const int rem = idx - b * per_b;
-            const int kbl = rem >> 6;
-            const int q = rem & 63;
-            const float4 *src = reinterpret_cast<const float4 *>(
-                p.x + static_cast<long long>(b) * p.K + static_cast<long long>(kb_begin + kbl) * 256) + q;
-            *reinterpret_cast<float4 *>(xs + (b * nbs + kbl) * kXBlockPitch + q * 16) = ldg_nc_f4(src);
+        const int n_out = B * per_b;
+        for (int base = threadIdx.x; base < n_out; base += kStageBatch * blockDim.x) {
+            float2 lo[kStageBatch], hi[kStageBatch];
+#pragma unroll
+            for (int u = 0; u < kStageBatch; ++u) {
+                const int idx = base + u * blockDim.x;
+                if (idx < n_out) {
+                    const int b = idx / per_b;
+                    const int rem = idx - b * per_b;
+                    const int kbl = rem >> 6;
+                    const int sl = (rem >> 3) & 7;    // slice
+                    const int k = rem & 7;            // float4 within the slice
+                    const float *xb = p.x + static_cast<long long>(b) * p.K +
+                                      static_cast<long long>(kb_begin + kbl) * 256 + 64 * (sl >> 1) + 16 * (sl & 1) +
+                                      2 * k;
+                    lo[u] = __ldg(reinterpret_cast<const float2 *>(xb));
+                    hi[u] = __ldg(reinterpret_cast<const float2 *>(xb + 32));
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kStageBatch; ++u) {
+                const int idx = base + u * blockDim.x;
+                if (idx < n_out) {
+                    const int b = idx / per_b;
+                    const int rem = idx - b * per_b;
+                    *reinterpret_cast<float4 *>(xs + (b * nbs + (rem >> 6)) * kXBlockPitch + ((rem >> 3) & 7) * 128 +
+                                                (rem & 7) * 16) = make_float4(lo[u].x, hi[u].x, lo[u].y, hi[u].y);
+                }
+            }
         }
     }
     __syncthreads();
@@ -225,10 +279,17 @@ __global__ void __launch_bounds__(kMaxThreads, 1) q4k_gemv_kernel(const Q4KParam
     bool failed = false;
     long long consumed = 0;
 
-    float2 accL[R][B], accH[R][B];
-    float gsum[NS == 2 ? MP : 1];  // stream-0 sums kept for the SwiGLU epilogue
+    float2 acc0[R][B], acc1[R][B];
+    float gsum[NS == 2 ? VPL : 1];  // stream-0 sums kept for the SwiGLU epilogue
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+            acc0[r][b] = f2(0.f, 0.f);
+            acc1[r][b] = f2(0.f, 0.f);
+        }
 
-    Cursor cc{0, 0, 0};
+    Cursor cc{t0 * G::TR, 0, 0};
     int slot = 0;
     uint32_t parity = 0;
     for (; consumed < total; ++consumed) {
@@ -237,20 +298,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) q4k_gemv_kernel(const Q4KParam
             failed = true;
             break;
         }
-        const int kc = c_begin + cc.kcl;
-        const long long row0 = (t0 + cc.tk * tstride) * G::TR;
-
-        if (cc.kcl == 0) {
-#pragma unroll
-            for (int r = 0; r < R; ++r)
-#pragma unroll
-                for (int b = 0; b < B; ++b) {
-                    accL[r][b] = f2(0.f, 0.f);
-                    accH[r][b] = f2(0.f, 0.f);
-                }
-        }
-
-        const int kb0 = kc * LPR;
+        const int kb0 = (c_begin + cc.kcl) * LPR;
         const int nblk = min(LPR, p.nb - kb0);
         if (l < nblk) {
             const uint8_t *slot_p = my_ring + slot * G::SLOT_BYTES + rg * G::RG_PITCH;
@@ -273,10 +321,10 @@ __global__ void __launch_bounds__(kMaxThreads, 1) q4k_gemv_kernel(const Q4KParam
 
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                float2 sL[R], mL[R], sH[R], mH[R];
+                ChunkScales cs[R];
 #pragma unroll
                 for (int r = 0; r < R; ++r)
-                    chunk_scales(hd[r], c, sL[r], mL[r], sH[r], mH[r]);
+                    cs[r] = chunk_scales(hd[r], c);
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int s = 2 * c + h;  // 16-byte quant slice
@@ -284,18 +332,17 @@ __global__ void __launch_bounds__(kMaxThreads, 1) q4k_gemv_kernel(const Q4KParam
 #pragma unroll
                     for (int r = 0; r < R; ++r)
                         q[r] = *reinterpret_cast<const uint4 *>(slot_p + r * G::ROW_BYTES + qs_off0 + s * qs_step);
-                    const int xoffL = (64 * c + 16 * h) * 4;
 #pragma unroll
                     for (int t = 0; t < 4; ++t) {
 #pragma unroll
                         for (int b = 0; b < B; ++b) {
-                            const uint8_t *xb = xblk + b * nbs * kXBlockPitch + xoffL + 16 * t;
-                            const float4 xl = *reinterpret_cast<const float4 *>(xb);
-                            const float4 xh = *reinterpret_cast<const float4 *>(xb + 128);
+                            const uint8_t *xq = xblk + b * nbs * kXBlockPitch + s * 128 + 32 * t;
+                            const float4 xa = *reinterpret_cast<const float4 *>(xq);
+                            const float4 xb = *reinterpret_cast<const float4 *>(xq + 16);
 #pragma unroll
                             for (int r = 0; r < R; ++r) {
                                 const uint32_t wv = (t == 0) ? q[r].x : (t == 1) ? q[r].y : (t == 2) ? q[r].z : q[r].w;
-                                q4_word(wv, sL[r], mL[r], sH[r], mH[r], xl, xh, accL[r][b], accH[r][b]);
+                                q4_word(wv, cs[r], xa, xb, acc0[r][b], acc1[r][b]);
                             }
                         }
                     }
@@ -307,94 +354,80 @@ __global__ void __launch_bounds__(kMaxThreads, 1) q4k_gemv_kernel(const Q4KParam
         if (issued < total) {
             if (lane == 0) {
                 fence_proxy_async_smem();
-                issue_slot<LPR, R>(p, pc, slot, c_begin, t0, tstride, my_ring_s, my_bars_s);
+                issue_slot<LPR, R>(p, pc, slot, c_begin, my_ring_s, my_bars_s);
             }
-            pc.advance(nch, NS);
+            pc.advance(nch, NS, row_step);
             ++issued;
         }
 
         const int cur_st = cc.st;
+        const long long row0 = cc.row0;
         const bool last_chunk = (cc.kcl == nch - 1);
-        cc.advance(nch, NS);
+        cc.advance(nch, NS, row_step);
         if (++slot == p.depth) {
             slot = 0;
             parity ^= 1u;
         }
+        if (!last_chunk)
+            continue;
 
-        if (last_chunk) {
-            // end of this stream's K range for the tile: reduce across the row group
-            float v[MP];
+        // end of this stream's K range for the tile: reduce across the row group
+        float v[MP];
 #pragma unroll
-            for (int r = 0; r < R; ++r)
+        for (int r = 0; r < R; ++r)
 #pragma unroll
-                for (int b = 0; b < B; ++b) {
-                    const float2 a = __fadd2_rn(accL[r][b], accH[r][b]);
-                    v[r * B + b] = a.x + a.y;
-                }
-#pragma unroll
-            for (int j = MV; j < MP; ++j)
-                v[j] = 0.f;
-            if constexpr (LPR > 1)
-                GroupReduce<LPR / 2, MP>::run(v, l);
-
-            // which value indices this lane now holds
-            int off = 0;
-            bool writer = true;
-            {
-                int m = MP;
-#pragma unroll
-                for (int o = LPR / 2; o >= 1; o >>= 1) {
-                    if (m > 1) {
-                        if (l & o)
-                            off += m / 2;
-                        m /= 2;
-                    } else if (l & o) {
-                        writer = false;
-                    }
-                }
+            for (int b = 0; b < B; ++b) {
+                const float2 a = __fadd2_rn(acc0[r][b], acc1[r][b]);
+                v[r * B + b] = a.x + a.y;
+                acc0[r][b] = f2(0.f, 0.f);
+                acc1[r][b] = f2(0.f, 0.f);
             }
+#pragma unroll
+        for (int j = MV; j < MP; ++j)
+            v[j] = 0.f;
+        if constexpr (LPR > 1)
+            GroupReduce<LPR / 2, MP>::run(v, l);
 
-            if constexpr (NS == 2) {
-                if (cur_st == 0) {
+        if constexpr (NS == 2) {
+            if (cur_st == 0) {
 #pragma unroll
-                    for (int j = 0; j < VPL; ++j)
-                        gsum[j] = v[j];
-                    continue;
-                }
+                for (int j = 0; j < VPL; ++j)
+                    gsum[j] = v[j];
+                continue;
             }
-            if (writer) {
+        }
+        if (!writer)
+            continue;
 #pragma unroll
-                for (int j = 0; j < VPL; ++j) {
-                    const int idx = off + j;
-                    if (idx >= MV)
-                        continue;
-                    const int r = idx / B;
-                    const int b = idx % B;
-                    const long long n = row0 + rg * R + r;
-                    if (n >= p.N)
-                        continue;
-                    if (p.splits > 1) {
-                        if constexpr (NS == 2) {
-                            p.part[((static_cast<long long>(split) * 2 + 0) * B + b) * p.N + n] = gsum[j] * 0x1p64f;
-                            p.part[((static_cast<long long>(split) * 2 + 1) * B + b) * p.N + n] = v[j] * 0x1p64f;
-                        } else {
-                            p.part[(static_cast<long long>(split) * B + b) * p.N + n] = v[j] * 0x1p64f;
-                        }
-                    } else {
-                        float out;
-                        if constexpr (NS == 2) {
-                            const float g = gsum[j] * 0x1p64f;
-                            const float u = v[j] * 0x1p64f;
-                            out = g / (1.0f + expf(-g)) * u;
-                        } else {
-                            out = v[j] * 0x1p64f;
-                        }
-                        p.y[static_cast<long long>(b) * p.N + n] = out;
-                        if (p.argmax && cand_better(out, n, best_v, best_i)) {
-                            best_v = out;
-                            best_i = n;
-                        }
-                    }
+        for (int j = 0; j < VPL; ++j) {
+            const int idx = off + j;
+            if (idx >= MV)
+                continue;
+            const int r = idx / B;
+            const int b = idx % B;
+            const long long n = row0 + rg * R + r;
+            if (n >= p.N)
+                continue;
+            if (p.splits > 1) {
+                if constexpr (NS == 2) {
+                    p.part[((static_cast<long long>(split) * 2 + 0) * B + b) * p.N + n] = gsum[j] * 0x1p64f;
+                    p.part[((static_cast<long long>(split) * 2 + 1) * B + b) * p.N + n] = v[j] * 0x1p64f;
+                } else {
+                    p.part[(static_cast<long long>(split) * B + b) * p.N + n] = v[j] * 0x1p64f;
+                }
+            } else {
+                float out;
+                if constexpr (NS == 2) {
+                    const float g = gsum[j] * 0x1p64f;
+                    const float u = v[j] * 0x1p64f;
+                    out = g / (1.0f + expf(-g)) * u;
+                } else {
+                    out = v[j] * 0x1p64f;
+                }
+                p.y[static_cast<long long>(b) * p.N + n] = out;
+                if (p.argmax && cand_better(out, n, best_v, best_i)) {
+                    best_v = out;
+                    best_i = n;
                 }
             }
         }
@@ -449,14 +482,15 @@ Q4KPlan q4k_plan(long long N, int K, int B, int NS, int soa, int sm_count, int s
 {
     Q4KPlan pl{};
     const int nb = K / kQ4KBlockElems;
-    const int misc = 128 /*argmax scratch*/ + 256 /*barriers*/;
+    const int misc = 256 /*argmax scratch, 16 B per warp*/ + 256 /*barriers*/;
     // SoA groups are 16 super-blocks, so SoA always walks K in 16-block chunks.
     const int lpr_opts[2] = {(soa || nb % 16 == 0) ? 16 : 4, 4};
     const int n_opts = (soa || nb % 16 != 0) ? 1 : 2;
     for (int oi = 0; oi < n_opts && !pl.ok; ++oi) {
         const int lpr = lpr_opts[oi];
+        const int R = 2;
         const int sb = q4k_slot_bytes(lpr);
-        const int TR = (32 / lpr) * 2;
+        const int TR = (32 / lpr) * R;
         const long long tiles = (N + TR - 1) / TR;
         const int nchunk = (nb + lpr - 1) / lpr;
         for (int warps = kMaxWarps; warps >= 4 && !pl.ok; warps /= 2) {
@@ -489,7 +523,7 @@ Q4KPlan q4k_plan(long long N, int K, int B, int NS, int soa, int sm_count, int s
             if (ctas > max_ctas)
                 ctas = max_ctas;
             pl.lpr = lpr;
-            pl.R = 2;
+            pl.R = R;
             pl.warps = warps;
             pl.tiles = tiles;
             pl.splits = splits;
@@ -497,7 +531,7 @@ Q4KPlan q4k_plan(long long N, int K, int B, int NS, int soa, int sm_count, int s
             pl.depth = depth;
             pl.ctas_per_split = static_cast<int>(ctas);
             pl.grid = pl.ctas_per_split * splits;
-            pl.smem = x_bytes + ((warps * depth * 8 + 127) & ~127) + warps * depth * sb + 128;
+            pl.smem = x_bytes + ((warps * depth * 8 + 127) & ~127) + warps * depth * sb + 256;
             pl.ok = pl.smem <= smem_optin;
         }
     }
@@ -507,7 +541,7 @@ Q4KPlan q4k_plan(long long N, int K, int B, int NS, int soa, int sm_count, int s
 template <int LPR, int B, int NS>
 static cudaError_t launch_one(const Q4KParams &p, const Q4KPlan &pl, cudaStream_t s)
 {
-    auto k = p.soa ? q4k_gemv_kernel<LPR, B, NS, 2, true> : q4k_gemv_kernel<LPR, B, NS, 2, false>;
+    auto k = p.soa ? q4k_gemv_kernel<LPR, B, NS, true> : q4k_gemv_kernel<LPR, B, NS, false>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
     if (e != cudaSuccess)
         return e;
