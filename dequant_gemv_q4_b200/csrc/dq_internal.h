@@ -32,6 +32,7 @@ struct Q4KParams {
 
 struct Q4KPlan {
     bool ok;
+    bool half;             // batch-1 half-block kernel (q4k_gemv_b1_kernel)
     int lpr;               // lanes per row group (4 or 16)
     int R;                 // rows per lane
     int warps;             // warps per CTA

@@ -73,11 +73,10 @@ struct ChunkScales {
     float2 S0, S1, M;
 };
 
-__device__ __forceinline__ ChunkScales chunk_scales(const Hdr &h, int c)
+// Scale pairs of the sub-block pair held in bytes k, k+1 of the scale word scw
+// and min word mnw.
+__device__ __forceinline__ ChunkScales scales_from_words(const Hdr &h, uint32_t scw, uint32_t mnw, uint32_t k)
 {
-    const uint32_t scw = (c < 2) ? h.sc03 : h.sc47;
-    const uint32_t mnw = (c < 2) ? h.mn03 : h.mn47;
-    const uint32_t k = (c & 1) * 2;  // byte of sub-block 2c within the word
     // {2^23 + scale_lo, 2^23 + scale_hi} and the same for the mins
     const float2 fs = f2(__uint_as_float(__byte_perm(scw, kMagic23, 0x7540u + k)),
                          __uint_as_float(__byte_perm(scw, kMagic23, 0x7541u + k)));
@@ -88,6 +87,12 @@ __device__ __forceinline__ ChunkScales chunk_scales(const Hdr &h, int c)
     s.S1 = __ffma2_rn(fs, h.D1, h.N1);
     s.M = __ffma2_rn(fm, h.DN, h.NN);
     return s;
+}
+
+__device__ __forceinline__ ChunkScales chunk_scales(const Hdr &h, int c)
+{
+    // sub-blocks 2c, 2c+1 sit in bytes 2(c%2), 2(c%2)+1 of the 0..3 or 4..7 words
+    return scales_from_words(h, (c < 2) ? h.sc03 : h.sc47, (c < 2) ? h.mn03 : h.mn47, (c & 1) * 2);
 }
 
 // The eight weights of one quant word, times 2^-64: wv[k] = {lo, hi} weights of

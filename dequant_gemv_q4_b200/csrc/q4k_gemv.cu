@@ -62,14 +62,36 @@ constexpr int kMaxWarps = 8;
 // of padding per super-block keep the lanes' reads free of bank conflicts.
 constexpr int kXBlockPitch = 1040;
 
-template <int LPR, int R>
+// Slot geometry.  LPR lanes per row group, RG = 32/LPR row groups per warp, R
+// rows per lane, BPC super-blocks per K-chunk.  A slot is TR = RG*R rows x BPC
+// super-blocks; rows of a row group are contiguous, row groups RG_PITCH apart.
+//   Geo     ("full-block" lanes): lane l owns super-block l of each chunk (BPC = LPR).
+//   GeoHalf ("half-block" lanes): lane l owns chunks 2(l%2), 2(l%2)+1 of super-block
+//           l/2 of each chunk (BPC = LPR/2), so a slot is half as large.
+template <int LPR, int RR>
 struct Geo {
-    static constexpr int RG = 32 / LPR;                       // row groups per warp
-    static constexpr int TR = RG * R;                         // rows per tile
-    static constexpr int ROW_BYTES = LPR * kQ4KBlockBytes;    // one row of a slot
+    static constexpr int R = RR;
+    static constexpr int RG = 32 / LPR;
+    static constexpr int TR = RG * R;
+    static constexpr int BPC = LPR;
+    static constexpr int ROW_BYTES = BPC * kQ4KBlockBytes;
     static constexpr int PAD = (LPR < 8) ? 64 : 0;            // bank-shift between row groups
     static constexpr int RG_PITCH = R * ROW_BYTES + PAD;
     static constexpr int SLOT_BYTES = RG * RG_PITCH;
+    static_assert(SLOT_BYTES % 128 == 0, "slot must keep 128-byte alignment");
+};
+
+template <int LPR>
+struct GeoHalf {
+    static constexpr int RG = 32 / LPR;
+    static constexpr int R = 2;
+    static constexpr int TR = RG * R;
+    static constexpr int BPC = LPR / 2;
+    static constexpr int ROW_BYTES = BPC * kQ4KBlockBytes;
+    static constexpr int PAD = 0;
+    static constexpr int RG_PITCH = R * ROW_BYTES;
+    static constexpr int SLOT_BYTES = RG * RG_PITCH;
+    static_assert(LPR == 32 || LPR == 8, "half-block lanes are laid out for 32 or 8 lanes per row group");
     static_assert(SLOT_BYTES % 128 == 0, "slot must keep 128-byte alignment");
 };
 
@@ -130,33 +152,32 @@ struct Cursor {
 
 // Issues the bulk copies of one slot (K-chunk c_begin + cur.kcl of stream
 // cur.st of the tile at cur.row0) into ring slot `slot`.
-template <int LPR, int R>
+template <class G>
 __device__ __forceinline__ void issue_slot(const Q4KParams &p, const Cursor &cur, int slot, int c_begin,
                                            uint32_t ring_s, uint32_t bars_s)
 {
-    using G = Geo<LPR, R>;
     const long long row_bytes_g = static_cast<long long>(p.nb) * kQ4KBlockBytes;
     const int rows = static_cast<int>(min(static_cast<long long>(G::TR), p.N - cur.row0));
-    const int kb0 = (c_begin + cur.kcl) * LPR;
-    const int nblk = min(LPR, p.nb - kb0);
+    const int kb0 = (c_begin + cur.kcl) * G::BPC;
+    const int nblk = min(G::BPC, p.nb - kb0);
     const uint8_t *src = (cur.st == 0 ? p.w[0] : p.w[1]) + cur.row0 * row_bytes_g + kb0 * kQ4KBlockBytes;
     const uint32_t dst = ring_s + slot * G::SLOT_BYTES;
     const uint32_t bar = bars_s + slot * 8;
     mbar_arrive_expect_tx(bar, static_cast<uint32_t>(rows * nblk * kQ4KBlockBytes));
-    if (nblk == p.nb && p.nb == LPR) {
+    if (nblk == p.nb && p.nb == G::BPC) {
         if (G::PAD == 0) {
             // whole rows of a contiguous tile, laid out without padding: one copy
             bulk_g2s(dst, src, static_cast<uint32_t>(rows * G::ROW_BYTES), bar);
         } else {
-            for (int g = 0; g * R < rows; ++g) {
-                const int gr = min(R, rows - g * R);
-                bulk_g2s(dst + g * G::RG_PITCH, src + static_cast<long long>(g) * R * row_bytes_g,
+            for (int g = 0; g * G::R < rows; ++g) {
+                const int gr = min(G::R, rows - g * G::R);
+                bulk_g2s(dst + g * G::RG_PITCH, src + static_cast<long long>(g) * G::R * row_bytes_g,
                          static_cast<uint32_t>(gr * G::ROW_BYTES), bar);
             }
         }
     } else {
         for (int r = 0; r < rows; ++r)
-            bulk_g2s(dst + (r / R) * G::RG_PITCH + (r % R) * G::ROW_BYTES, src + r * row_bytes_g,
+            bulk_g2s(dst + (r / G::R) * G::RG_PITCH + (r % G::R) * G::ROW_BYTES, src + r * row_bytes_g,
                      static_cast<uint32_t>(nblk * kQ4KBlockBytes), bar);
     }
 }
@@ -232,14 +253,15 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_kernel(const Q4KPa
     }
     for (int s = 0; s < p.depth && issued < total; ++s, ++issued) {
         if (lane == 0)
-            issue_slot<LPR, R>(p, pc, s, c_begin, my_ring_s, my_bars_s);
+            issue_slot<G>(p, pc, s, c_begin, my_ring_s, my_bars_s);
         pc.advance(nch, NS, row_step);
     }
 
     // stage this split's activations in (lo, hi) pairs (fp32, padded per super-block);
-    // each thread keeps kStageBatch loads in flight before storing
+    // each thread keeps kStageBatch loads in flight before storing (one at a
+    // time for large B, whose kernels have no registers to spare)
     {
-        constexpr int kStageBatch = 8;
+        constexpr int kStageBatch = (B <= 2) ? 8 : 1;
         const int per_b = nbs * 64;  // float4 per batch row
         const int n_out = B * per_b;
         for (int base = threadIdx.x; base < n_out; base += kStageBatch * blockDim.x) {
@@ -354,7 +376,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_kernel(const Q4KPa
         if (issued < total) {
             if (lane == 0) {
                 fence_proxy_async_smem();
-                issue_slot<LPR, R>(p, pc, slot, c_begin, my_ring_s, my_bars_s);
+                issue_slot<G>(p, pc, slot, c_begin, my_ring_s, my_bars_s);
             }
             pc.advance(nch, NS, row_step);
             ++issued;
@@ -471,6 +493,281 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_kernel(const Q4KPa
 }
 
 // ---------------------------------------------------------------------------
+// Batch-1 kernel with half-block lanes (GeoHalf): each lane owns two of the
+// four 64-weight chunks of one super-block for two rows, so a slot is 4.5 KB
+// and sixteen warps (four per scheduler) fit beside their two-deep rings.
+// x keeps the (lo, hi) pair staging, with the two 512-byte halves of every
+// super-block kXHalfGap bytes apart and kXHalfPitch bytes per super-block, so
+// the eight lanes of one shared-memory phase read eight distinct bank groups.
+// ---------------------------------------------------------------------------
+constexpr int kB1Warps = 16;
+constexpr int kXHalfPitch = 1056;
+constexpr int kXHalfGap = 528;
+
+template <int LPR, int NS, bool SOA>
+__global__ void __launch_bounds__(kB1Warps * 32, 1) q4k_gemv_b1_kernel(const Q4KParams p)
+{
+    using G = GeoHalf<LPR>;
+    constexpr int R = G::R;
+
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int nwarps = blockDim.x >> 5;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int rg = lane / LPR;
+    const int l = lane % LPR;
+    const int bl = l >> 1;   // super-block of the chunk
+    const int hh = l & 1;    // half: chunks 2*hh and 2*hh + 1
+
+    const int split = blockIdx.x / p.ctas_per_split;
+    const int cj = blockIdx.x % p.ctas_per_split;
+    const int nchunk_total = (p.nb + G::BPC - 1) / G::BPC;
+    const int c_begin = split * p.chunks_per_split;
+    const int c_end = min(c_begin + p.chunks_per_split, nchunk_total);
+    const int nch = c_end - c_begin;
+    const int kb_begin = c_begin * G::BPC;
+    const int nbs = min(nch * G::BPC, p.nb - kb_begin);
+
+    // shared memory: [x staging][barriers][ring][argmax scratch]
+    const int x_bytes = (nbs * kXHalfPitch + 127) & ~127;
+    uint8_t *xs = smem;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + x_bytes);
+    const int bar_bytes = (nwarps * p.depth * 8 + 127) & ~127;
+    uint8_t *ring = smem + x_bytes + bar_bytes;
+    uint8_t *my_ring = ring + static_cast<size_t>(warp) * p.depth * G::SLOT_BYTES;
+    const uint32_t my_ring_s = smem_u32(my_ring);
+    const uint32_t my_bars_s = smem_u32(bars + warp * p.depth);
+    ArgmaxCand *red = reinterpret_cast<ArgmaxCand *>(ring + static_cast<size_t>(nwarps) * p.depth * G::SLOT_BYTES);
+
+    const long long tstride = static_cast<long long>(p.ctas_per_split) * nwarps;
+    const long long t0 = static_cast<long long>(cj) * nwarps + warp;
+    const long long ntiles_w = (t0 < p.tiles) ? (p.tiles - t0 + tstride - 1) / tstride : 0;
+    const long long total = ntiles_w * NS * nch;
+    const long long row_step = tstride * G::TR;
+
+    // After the row-group reduction lane 0 of the group holds row 0's sum and
+    // lane LPR/2 row 1's; the other lanes hold copies.
+    const bool writer = (l & (LPR / 2 - 1)) == 0;
+    const int wrow = (l >= LPR / 2) ? 1 : 0;
+
+    Cursor pc{t0 * G::TR, 0, 0};
+    long long issued = 0;
+    if (lane == 0) {
+        for (int s = 0; s < p.depth; ++s)
+            mbar_init(my_bars_s + s * 8, 1);
+        mbar_fence_init();
+    }
+    for (int s = 0; s < p.depth && issued < total; ++s, ++issued) {
+        if (lane == 0)
+            issue_slot<G>(p, pc, s, c_begin, my_ring_s, my_bars_s);
+        pc.advance(nch, NS, row_step);
+    }
+
+    // stage x in (lo, hi) pairs, 8 loads in flight per thread
+    {
+        constexpr int kStageBatch = 8;
+        const int n_out = nbs * 64;
+        for (int base = threadIdx.x; base < n_out; base += kStageBatch * blockDim.x) {
+            float2 lo[kStageBatch], hi[kStageBatch];
+#pragma unroll
+            for (int u = 0; u < kStageBatch; ++u) {
+                const int idx = base + u * blockDim.x;
+                if (idx < n_out) {
+                    const int kbl = idx >> 6, sl = (idx >> 3) & 7, k = idx & 7;
+                    const float *xb = p.x + static_cast<long long>(kb_begin + kbl) * 256 + 64 * (sl >> 1) +
+                                      16 * (sl & 1) + 2 * k;
+                    lo[u] = __ldg(reinterpret_cast<const float2 *>(xb));
+                    hi[u] = __ldg(reinterpret_cast<const float2 *>(xb + 32));
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kStageBatch; ++u) {
+                const int idx = base + u * blockDim.x;
+                if (idx < n_out) {
+                    const int kbl = idx >> 6, sl = (idx >> 3) & 7, k = idx & 7;
+                    *reinterpret_cast<float4 *>(xs + kbl * kXHalfPitch + (sl >> 2) * kXHalfGap + (sl & 3) * 128 +
+                                                k * 16) = make_float4(lo[u].x, hi[u].x, lo[u].y, hi[u].y);
+                }
+            }
+        }
+    }
+    __syncthreads();
+
+    float best_v = -INFINITY;
+    long long best_i = 0x7fffffffffffffffLL;
+    bool failed = false;
+    long long consumed = 0;
+    float gsum = 0.f;  // stream-0 sum kept for the SwiGLU epilogue
+
+    float2 acc0[R], acc1[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        acc0[r] = f2(0.f, 0.f);
+        acc1[r] = f2(0.f, 0.f);
+    }
+
+    Cursor cc{t0 * G::TR, 0, 0};
+    int slot = 0;
+    uint32_t parity = 0;
+    for (; consumed < total; ++consumed) {
+        const bool ok = mbar_wait_bounded(my_bars_s + slot * 8, parity, p.err);
+        if (!__all_sync(0xffffffffu, ok)) {
+            failed = true;
+            break;
+        }
+        const int kb0 = (c_begin + cc.kcl) * G::BPC;
+        const int nblk = min(G::BPC, p.nb - kb0);
+        if (bl < nblk) {
+            const uint8_t *slot_p = my_ring + slot * G::SLOT_BYTES + rg * G::RG_PITCH;
+            // this lane's header and its first quant slice (slice 4*hh of the super-block)
+            int hdr_off, qs_off0, qs_step;
+            if constexpr (SOA) {
+                hdr_off = 16 * bl;
+                qs_step = 16 * nblk;
+                qs_off0 = 16 * nblk + 4 * hh * qs_step + 16 * bl;
+            } else {
+                hdr_off = kQ4KBlockBytes * bl;
+                qs_step = 16;
+                qs_off0 = hdr_off + 16 + 64 * hh;
+            }
+            Hdr hd[R];
+            uint32_t scw[R], mnw[R];
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                hd[r] = decode_hdr(*reinterpret_cast<const uint4 *>(slot_p + r * G::ROW_BYTES + hdr_off));
+                scw[r] = hh ? hd[r].sc47 : hd[r].sc03;
+                mnw[r] = hh ? hd[r].mn47 : hd[r].mn03;
+            }
+            const uint8_t *xl = xs + (kb0 - kb_begin + bl) * kXHalfPitch + hh * kXHalfGap;
+
+#pragma unroll
+            for (int cp = 0; cp < 2; ++cp) {  // chunk 2*hh + cp
+                ChunkScales cs[R];
+#pragma unroll
+                for (int r = 0; r < R; ++r)
+                    cs[r] = scales_from_words(hd[r], scw[r], mnw[r], cp * 2);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int sl = 2 * cp + h;  // slice within the half
+                    uint4 q[R];
+#pragma unroll
+                    for (int r = 0; r < R; ++r)
+                        q[r] = *reinterpret_cast<const uint4 *>(slot_p + r * G::ROW_BYTES + qs_off0 + sl * qs_step);
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const uint8_t *xq = xl + sl * 128 + 32 * t;
+                        const float4 xa = *reinterpret_cast<const float4 *>(xq);
+                        const float4 xb = *reinterpret_cast<const float4 *>(xq + 16);
+#pragma unroll
+                        for (int r = 0; r < R; ++r) {
+                            const uint32_t wv = (t == 0) ? q[r].x : (t == 1) ? q[r].y : (t == 2) ? q[r].z : q[r].w;
+                            q4_word(wv, cs[r], xa, xb, acc0[r], acc1[r]);
+                        }
+                    }
+                }
+            }
+        }
+
+        __syncwarp();
+        if (issued < total) {
+            if (lane == 0) {
+                fence_proxy_async_smem();
+                issue_slot<G>(p, pc, slot, c_begin, my_ring_s, my_bars_s);
+            }
+            pc.advance(nch, NS, row_step);
+            ++issued;
+        }
+
+        const int cur_st = cc.st;
+        const long long row0 = cc.row0;
+        const bool last_chunk = (cc.kcl == nch - 1);
+        cc.advance(nch, NS, row_step);
+        if (++slot == p.depth) {
+            slot = 0;
+            parity ^= 1u;
+        }
+        if (!last_chunk)
+            continue;
+
+        float v[2];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const float2 a = __fadd2_rn(acc0[r], acc1[r]);
+            v[r] = a.x + a.y;
+            acc0[r] = f2(0.f, 0.f);
+            acc1[r] = f2(0.f, 0.f);
+        }
+        GroupReduce<LPR / 2, 2>::run(v, l);
+        if constexpr (NS == 2) {
+            if (cur_st == 0) {
+                gsum = v[0];
+                continue;
+            }
+        }
+        const long long n = row0 + rg * R + wrow;
+        if (!writer || n >= p.N)
+            continue;
+        if (p.splits > 1) {
+            if constexpr (NS == 2) {
+                p.part[(static_cast<long long>(split) * 2 + 0) * p.N + n] = gsum * 0x1p64f;
+                p.part[(static_cast<long long>(split) * 2 + 1) * p.N + n] = v[0] * 0x1p64f;
+            } else {
+                p.part[static_cast<long long>(split) * p.N + n] = v[0] * 0x1p64f;
+            }
+        } else {
+            float out;
+            if constexpr (NS == 2) {
+                const float g = gsum * 0x1p64f;
+                out = g / (1.0f + expf(-g)) * (v[0] * 0x1p64f);
+            } else {
+                out = v[0] * 0x1p64f;
+            }
+            p.y[n] = out;
+            if (p.argmax && cand_better(out, n, best_v, best_i)) {
+                best_v = out;
+                best_i = n;
+            }
+        }
+    }
+
+    if (failed) {
+        // the copies already issued into this warp's ring must land before the CTA exits
+        for (long long i = consumed; i < issued; ++i) {
+            mbar_wait_bounded(my_bars_s + slot * 8, parity, nullptr);
+            if (++slot == p.depth) {
+                slot = 0;
+                parity ^= 1u;
+            }
+        }
+    }
+
+    if (p.argmax && p.splits == 1) {
+        // CTA-wide (max, lowest index) candidate
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, best_v, o);
+            const long long oi = __shfl_xor_sync(0xffffffffu, best_i, o);
+            if (cand_better(ov, oi, best_v, best_i)) {
+                best_v = ov;
+                best_i = oi;
+            }
+        }
+        if (lane == 0) {
+            red[warp].v = best_v;
+            red[warp].idx = best_i;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            ArgmaxCand c = red[0];
+            for (int w = 1; w < nwarps; ++w)
+                if (cand_better(red[w].v, red[w].idx, c.v, c.idx))
+                    c = red[w];
+            p.cand[blockIdx.x] = c;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 
@@ -478,10 +775,75 @@ int q4k_slot_bytes(int lpr) { return lpr == 16 ? Geo<16, 2>::SLOT_BYTES : Geo<4,
 
 // Launch plan for a shape; the same function sizes the workspace, so the two
 // always agree.
-Q4KPlan q4k_plan(long long N, int K, int B, int NS, int soa, int sm_count, int smem_optin)
+static Q4KPlan q4k_plan_half(long long N, int nb, int NS, int soa, int sm_count, int smem_optin)
 {
     Q4KPlan pl{};
+    const int misc = 256 /*argmax scratch*/ + 512 /*barriers*/;
+    // SoA groups are 16 super-blocks (the whole row when it has fewer), so SoA
+    // takes 16-block chunks unless a row has at most 4 super-blocks.
+    const int lpr = soa ? (nb <= 4 ? 8 : 32) : (nb % 16 == 0 ? 32 : 8);
+    const int bpc = lpr / 2;
+    const int sb = (lpr == 32) ? GeoHalf<32>::SLOT_BYTES : GeoHalf<8>::SLOT_BYTES;
+    const int TR = (32 / lpr) * 2;
+    const long long tiles = (N + TR - 1) / TR;
+    const int nchunk = (nb + bpc - 1) / bpc;
+    for (int warps = kB1Warps; warps >= 4 && !pl.ok; warps /= 2) {
+        int splits = 1, cps = nchunk;
+        for (;;) {
+            cps = (nchunk + splits - 1) / splits;
+            if (cps * bpc * kXHalfPitch + warps * 2 * sb + misc <= smem_optin || cps == 1)
+                break;
+            ++splits;
+        }
+        const long long warps_total = static_cast<long long>(sm_count) * warps;
+        while (tiles * NS * splits * 2 < warps_total && splits < nchunk) {
+            ++splits;
+            cps = (nchunk + splits - 1) / splits;
+        }
+        splits = (nchunk + cps - 1) / cps;
+        const int x_bytes = (cps * bpc * kXHalfPitch + 127) & ~127;
+        int depth = (smem_optin - x_bytes - misc) / (warps * sb);
+        if (depth > 4)
+            depth = 4;
+        if (depth < 2)
+            continue;
+        long long ctas = (tiles + warps - 1) / warps;
+        const long long max_ctas = sm_count / splits > 0 ? sm_count / splits : 1;
+        if (ctas > max_ctas)
+            ctas = max_ctas;
+        pl.half = true;
+        pl.lpr = lpr;
+        pl.R = 2;
+        pl.warps = warps;
+        pl.tiles = tiles;
+        pl.splits = splits;
+        pl.chunks_per_split = cps;
+        pl.depth = depth;
+        pl.ctas_per_split = static_cast<int>(ctas);
+        pl.grid = pl.ctas_per_split * splits;
+        pl.smem = x_bytes + ((warps * depth * 8 + 127) & ~127) + warps * depth * sb + 256;
+        pl.ok = pl.smem <= smem_optin;
+    }
+    return pl;
+}
+
+Q4KPlan q4k_plan(long long N, int K, int B, int NS, int soa, int sm_count, int smem_optin)
+{
     const int nb = K / kQ4KBlockElems;
+    if (B == 1) {
+        // Half-block lanes halve each warp's serial chain of slots (better when
+        // every warp gets only a few slots); full-block lanes spend fewer
+        // instructions per weight (better for long matrices).
+        const int full_lpr = (soa || nb % 16 == 0) ? 16 : 4;
+        const long long full_tiles = (N + (32 / full_lpr) * 2 - 1) / ((32 / full_lpr) * 2);
+        const long long slots = full_tiles * NS * ((nb + full_lpr - 1) / full_lpr);
+        if (slots < 8LL * sm_count * kMaxWarps) {
+            const Q4KPlan ph = q4k_plan_half(N, nb, NS, soa, sm_count, smem_optin);
+            if (ph.ok)
+                return ph;
+        }
+    }
+    Q4KPlan pl{};
     const int misc = 256 /*argmax scratch, 16 B per warp*/ + 256 /*barriers*/;
     // SoA groups are 16 super-blocks, so SoA always walks K in 16-block chunks.
     const int lpr_opts[2] = {(soa || nb % 16 == 0) ? 16 : 4, 4};
@@ -565,8 +927,24 @@ static cudaError_t launch_b(const Q4KParams &p, const Q4KPlan &pl, int B, cudaSt
     }
 }
 
+template <int LPR, int NS>
+static cudaError_t launch_half(const Q4KParams &p, const Q4KPlan &pl, cudaStream_t s)
+{
+    auto k = p.soa ? q4k_gemv_b1_kernel<LPR, NS, true> : q4k_gemv_b1_kernel<LPR, NS, false>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
+    if (e != cudaSuccess)
+        return e;
+    k<<<pl.grid, pl.warps * 32, pl.smem, s>>>(p);
+    return cudaGetLastError();
+}
+
 cudaError_t q4k_gemv_launch(const Q4KParams &p, const Q4KPlan &pl, int B, int NS, cudaStream_t s)
 {
+    if (pl.half) {
+        if (pl.lpr == 32)
+            return NS == 1 ? launch_half<32, 1>(p, pl, s) : launch_half<32, 2>(p, pl, s);
+        return NS == 1 ? launch_half<8, 1>(p, pl, s) : launch_half<8, 2>(p, pl, s);
+    }
     if (pl.lpr == 16)
         return NS == 1 ? launch_b<16, 1>(p, pl, B, s) : launch_b<16, 2>(p, pl, B, s);
     return NS == 1 ? launch_b<4, 1>(p, pl, B, s) : launch_b<4, 2>(p, pl, B, s);

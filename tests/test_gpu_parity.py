@@ -330,3 +330,18 @@ def test_errors_launch_nothing_and_leave_the_stream_usable():
     y2 = dq.q4k_gemv(w, x, N, K)                     # a valid call still works
     torch.cuda.synchronize()
     assert torch.isfinite(y2).all().item()
+
+
+@pytest.mark.parametrize("N,K", [(40000, 4096), (16000, 12288)])
+@pytest.mark.parametrize("layout", ["aos", "soa"])
+def test_q4k_gemv_long_matrices_full_block_lanes(N, K, layout):
+    # enough rows that batch 1 runs on full-block lanes (the LM-head kernel);
+    # the smaller shapes above run on half-block lanes
+    rng = np.random.default_rng(N + K)
+    w = synth.q4k_matrix(rng, N, K)
+    x = synth.activations(rng, 1, K)
+    wl = w if layout == "aos" else oracle.q4k_repack_soa(w, N, K)
+    y = host(dq.q4k_gemv(dev(wl), dev(x), N, K, layout=layout))
+    rows = np.unique(np.concatenate([np.arange(0, N, 7), [N - 1]]))
+    y_ref, a_ref = oracle_rows(lambda rows: oracle.q4k_gemv(w, N, K, x, rows=rows), N, rows)
+    assert_within(y[:, rows], y_ref, a_ref, "N=%d K=%d %s" % (N, K, layout))
