@@ -220,7 +220,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_kernel(const Q4KPa
 
     // this warp's tiles: t0, t0 + tstride, ...
     const long long tstride = static_cast<long long>(p.ctas_per_split) * nwarps;
-    const long long t0 = static_cast<long long>(cj) * nwarps + warp;
+    // warp-major tile order: the last, partial round of tiles spreads over all SMs
+    const long long t0 = static_cast<long long>(warp) * p.ctas_per_split + cj;
     const long long ntiles_w = (t0 < p.tiles) ? (p.tiles - t0 + tstride - 1) / tstride : 0;
     const long long total = ntiles_w * NS * nch;
     const long long row_step = tstride * G::TR;
@@ -540,7 +541,8 @@ __global__ void __launch_bounds__(kB1Warps * 32, 1) q4k_gemv_b1_kernel(const Q4K
     ArgmaxCand *red = reinterpret_cast<ArgmaxCand *>(ring + static_cast<size_t>(nwarps) * p.depth * G::SLOT_BYTES);
 
     const long long tstride = static_cast<long long>(p.ctas_per_split) * nwarps;
-    const long long t0 = static_cast<long long>(cj) * nwarps + warp;
+    // warp-major tile order: the last, partial round of tiles spreads over all SMs
+    const long long t0 = static_cast<long long>(warp) * p.ctas_per_split + cj;
     const long long ntiles_w = (t0 < p.tiles) ? (p.tiles - t0 + tstride - 1) / tstride : 0;
     const long long total = ntiles_w * NS * nch;
     const long long row_step = tstride * G::TR;
@@ -775,6 +777,23 @@ int q4k_slot_bytes(int lpr) { return lpr == 16 ? Geo<16, 2>::SLOT_BYTES : Geo<4,
 
 // Launch plan for a shape; the same function sizes the workspace, so the two
 // always agree.
+// Warps per CTA for `tiles` row tiles on `sm_count` SMs (one CTA per SM):
+// enough to give every SM work and at least one per scheduler; with `round4`
+// a multiple of four, so the four schedulers of an SM carry equal numbers of
+// warps (the full-block kernel skips the rounding when its shared memory
+// would then force a K split).
+static int pick_warps(long long tiles, int sm_count, int max_warps, bool round4)
+{
+    long long w = (tiles + sm_count - 1) / sm_count;
+    if (round4)
+        w = (w + 3) / 4 * 4;
+    if (w < 4)
+        w = 4;
+    if (w > max_warps)
+        w = max_warps;
+    return static_cast<int>(w);
+}
+
 static Q4KPlan q4k_plan_half(long long N, int nb, int NS, int soa, int sm_count, int smem_optin)
 {
     Q4KPlan pl{};
@@ -787,7 +806,8 @@ static Q4KPlan q4k_plan_half(long long N, int nb, int NS, int soa, int sm_count,
     const int TR = (32 / lpr) * 2;
     const long long tiles = (N + TR - 1) / TR;
     const int nchunk = (nb + bpc - 1) / bpc;
-    for (int warps = kB1Warps; warps >= 4 && !pl.ok; warps /= 2) {
+    const int w0 = pick_warps(tiles, sm_count, kB1Warps, true);
+    for (int warps = w0; warps >= 4 && !pl.ok; warps = (warps > 4 && warps / 2 < 4) ? 4 : warps / 2) {
         int splits = 1, cps = nchunk;
         for (;;) {
             cps = (nchunk + splits - 1) / splits;
@@ -855,7 +875,8 @@ Q4KPlan q4k_plan(long long N, int K, int B, int NS, int soa, int sm_count, int s
         const int TR = (32 / lpr) * R;
         const long long tiles = (N + TR - 1) / TR;
         const int nchunk = (nb + lpr - 1) / lpr;
-        for (int warps = kMaxWarps; warps >= 4 && !pl.ok; warps /= 2) {
+        const int w0 = pick_warps(tiles, sm_count, kMaxWarps, false);
+        for (int warps = w0; warps >= 4 && !pl.ok; warps = (warps > 4 && warps / 2 < 4) ? 4 : warps / 2) {
             const int min_ring = warps * 2 * sb;
             // smallest split count whose activations fit beside a two-deep ring
             int splits = 1;
