@@ -83,6 +83,31 @@ def algorithmic_bytes(wl, B=1):
     return nmat * wl.N * (wl.K // elems) * per_block + 4 * B * wl.K
 
 
+def rank_workload(wl, rank: int, world: int):
+    """The workload a rank runs: with several ranks each one gets its own
+    independent problem of the same shape (seed offset by rank)."""
+    from dequant_gemv_q4_b200 import synth
+    if world <= 1:
+        return wl
+    return synth.Workload(wl.name, wl.fmt, wl.op, wl.N, wl.K, wl.batches, wl.seed + 1000 * rank, wl.x_scale)
+
+
+def max_over_ranks(v: float, world: int, device=None) -> float:
+    """Largest value over all ranks (the job's time is its slowest rank's)."""
+    if world <= 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gbps(nbytes_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job GB/s: the bytes every rank processed in one step over the step time."""
+    return nbytes_per_rank * world / (ms_per_step * 1e-3) / 1e9
+
+
 def measured_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -254,9 +279,7 @@ def main():
     if args.rows:
         wl = synth.Workload("%s_rows%d" % (wl.name, args.rows), wl.fmt, wl.op, args.rows, wl.K, wl.batches,
                             wl.seed, wl.x_scale)
-    if wl.seed is not None and dist_on:
-        wl = synth.Workload(wl.name, wl.fmt, wl.op, wl.N, wl.K, wl.batches, wl.seed + 1000 * rank,
-                            wl.x_scale)
+    wl = rank_workload(wl, rank, world)
     inp = synth.make_inputs(wl, B=B)
     dev = torch.device("cuda", local_rank)
     argmax = wl.op == "gemv_argmax"
@@ -290,13 +313,6 @@ def main():
             dist.barrier(device_ids=[local_rank])
         torch.cuda.synchronize(dev)
 
-    def max_over_ranks(v):
-        if not dist_on:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     nbytes = algorithmic_bytes(wl, B)
 
     # ---- device-resident steps (the headline value) ----
@@ -312,8 +328,8 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize(dev)
     barrier()
-    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
-    value = nbytes * world / (ms * 1e-3) / 1e9
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    value = job_gbps(nbytes, world, ms)
 
     # ---- dominant kernel alone (one launch per call, no epilogue kernels) ----
     if not split:
@@ -354,8 +370,8 @@ def main():
     h1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    e2e_ms = max_over_ranks(h0.elapsed_time(h1) / args.steps)
-    e2e_value = nbytes * world / (e2e_ms * 1e-3) / 1e9
+    e2e_ms = max_over_ranks(h0.elapsed_time(h1) / args.steps, world, dev)
+    e2e_value = job_gbps(nbytes, world, e2e_ms)
     h2d = x_host.numel() * 4
     d2h = y_host.numel() * 4 + (8 if argmax else 0)
 
