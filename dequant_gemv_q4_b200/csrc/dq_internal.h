@@ -33,6 +33,7 @@ struct Q4KParams {
 struct Q4KPlan {
     bool ok;
     bool half;             // batch-1 half-block kernel (q4k_gemv_b1_kernel)
+    bool fx;               // batch-1 fixed-point-activation kernel (q4k_gemv_fx_kernel)
     int lpr;               // lanes per row group (4 or 16)
     int R;                 // rows per lane
     int warps;             // warps per CTA
@@ -47,6 +48,8 @@ struct Q4KPlan {
 
 Q4KPlan q4k_plan(long long N, int K, int B, int NS, int soa, int sm_count, int smem_optin);
 cudaError_t q4k_gemv_launch(const Q4KParams &p, const Q4KPlan &pl, int B, int NS, cudaStream_t s);
+int q4k_fx_stage_bytes_per_block();
+cudaError_t q4k_gemv_fx_launch(const Q4KParams &p, const Q4KPlan &pl, int NS, cudaStream_t s);
 
 // Q8_0 GEMV
 struct Q8Params {

@@ -37,6 +37,7 @@
 #include "dq_common.cuh"
 #include "dq_internal.h"
 #include "q4k_decode.cuh"
+#include "q4k_stream.cuh"
 
 namespace dq {
 
@@ -54,133 +55,12 @@ __device__ __forceinline__ void q4_word(uint32_t w, const ChunkScales &cs, float
     acc1 = __ffma2_rn(wv[3], f2(xb.z, xb.w), acc1);
 }
 
-constexpr int kMaxWarps = 8;
-
 // x of one super-block is staged as 8 slices x 8 float4, float4 k of slice
 // s = 2c+h holding {x[L+2k], x[H+2k], x[L+2k+1], x[H+2k+1]} (L = 64c+16h,
 // H = L+32): the (lo, hi) weight pairs of quant bytes 2k and 2k+1.  16 bytes
 // of padding per super-block keep the lanes' reads free of bank conflicts.
 constexpr int kXBlockPitch = 1040;
 
-// Slot geometry.  LPR lanes per row group, RG = 32/LPR row groups per warp, R
-// rows per lane, BPC super-blocks per K-chunk.  A slot is TR = RG*R rows x BPC
-// super-blocks; rows of a row group are contiguous, row groups RG_PITCH apart.
-//   Geo     ("full-block" lanes): lane l owns super-block l of each chunk (BPC = LPR).
-//   GeoHalf ("half-block" lanes): lane l owns chunks 2(l%2), 2(l%2)+1 of super-block
-//           l/2 of each chunk (BPC = LPR/2), so a slot is half as large.
-template <int LPR, int RR>
-struct Geo {
-    static constexpr int R = RR;
-    static constexpr int RG = 32 / LPR;
-    static constexpr int TR = RG * R;
-    static constexpr int BPC = LPR;
-    static constexpr int ROW_BYTES = BPC * kQ4KBlockBytes;
-    static constexpr int PAD = (LPR < 8) ? 64 : 0;            // bank-shift between row groups
-    static constexpr int RG_PITCH = R * ROW_BYTES + PAD;
-    static constexpr int SLOT_BYTES = RG * RG_PITCH;
-    static_assert(SLOT_BYTES % 128 == 0, "slot must keep 128-byte alignment");
-};
-
-template <int LPR>
-struct GeoHalf {
-    static constexpr int RG = 32 / LPR;
-    static constexpr int R = 2;
-    static constexpr int TR = RG * R;
-    static constexpr int BPC = LPR / 2;
-    static constexpr int ROW_BYTES = BPC * kQ4KBlockBytes;
-    static constexpr int PAD = 0;
-    static constexpr int RG_PITCH = R * ROW_BYTES;
-    static constexpr int SLOT_BYTES = RG * RG_PITCH;
-    static_assert(LPR == 32 || LPR == 8, "half-block lanes are laid out for 32 or 8 lanes per row group");
-    static_assert(SLOT_BYTES % 128 == 0, "slot must keep 128-byte alignment");
-};
-
-// Transposing butterfly over the LPR lanes of a row group: on entry each lane
-// holds M partial values; on exit lane l holds the sums of a contiguous run of
-// value indices (the kernel recomputes which).  M is a power of two.
-template <int O, int M>
-struct GroupReduce {
-    static __device__ __forceinline__ void run(float *v, int lane)
-    {
-        if constexpr (M > 1) {
-            const bool up = (lane & O) != 0;
-#pragma unroll
-            for (int i = 0; i < M / 2; ++i) {
-                const float send = up ? v[i] : v[i + M / 2];
-                const float keep = up ? v[i + M / 2] : v[i];
-                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, O);
-            }
-            if constexpr (O > 1)
-                GroupReduce<O / 2, M / 2>::run(v, lane);
-        } else {
-            v[0] += __shfl_xor_sync(0xffffffffu, v[0], O);
-            if constexpr (O > 1)
-                GroupReduce<O / 2, 1>::run(v, lane);
-        }
-    }
-};
-
-template <int N>
-struct Pow2Ceil {
-    static constexpr int value = (N <= 1) ? 1 : 2 * Pow2Ceil<(N + 1) / 2>::value;
-};
-template <>
-struct Pow2Ceil<1> {
-    static constexpr int value = 1;
-};
-
-// Position of a warp in its slot sequence: the tile's first row row0, weight
-// stream st, K-chunk kcl (relative to the split's first chunk).  row0 moves by
-// the warp's tile stride once every stream and chunk of a tile are done.
-struct Cursor {
-    long long row0;
-    int st;
-    int kcl;
-    __device__ __forceinline__ bool advance(int nch, int ns, long long row_step)
-    {
-        if (++kcl == nch) {
-            kcl = 0;
-            if (++st == ns) {
-                st = 0;
-                row0 += row_step;
-                return true;
-            }
-        }
-        return false;
-    }
-};
-
-// Issues the bulk copies of one slot (K-chunk c_begin + cur.kcl of stream
-// cur.st of the tile at cur.row0) into ring slot `slot`.
-template <class G>
-__device__ __forceinline__ void issue_slot(const Q4KParams &p, const Cursor &cur, int slot, int c_begin,
-                                           uint32_t ring_s, uint32_t bars_s)
-{
-    const long long row_bytes_g = static_cast<long long>(p.nb) * kQ4KBlockBytes;
-    const int rows = static_cast<int>(min(static_cast<long long>(G::TR), p.N - cur.row0));
-    const int kb0 = (c_begin + cur.kcl) * G::BPC;
-    const int nblk = min(G::BPC, p.nb - kb0);
-    const uint8_t *src = (cur.st == 0 ? p.w[0] : p.w[1]) + cur.row0 * row_bytes_g + kb0 * kQ4KBlockBytes;
-    const uint32_t dst = ring_s + slot * G::SLOT_BYTES;
-    const uint32_t bar = bars_s + slot * 8;
-    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(rows * nblk * kQ4KBlockBytes));
-    if (nblk == p.nb && p.nb == G::BPC) {
-        if (G::PAD == 0) {
-            // whole rows of a contiguous tile, laid out without padding: one copy
-            bulk_g2s(dst, src, static_cast<uint32_t>(rows * G::ROW_BYTES), bar);
-        } else {
-            for (int g = 0; g * G::R < rows; ++g) {
-                const int gr = min(G::R, rows - g * G::R);
-                bulk_g2s(dst + g * G::RG_PITCH, src + static_cast<long long>(g) * G::R * row_bytes_g,
-                         static_cast<uint32_t>(gr * G::ROW_BYTES), bar);
-            }
-        }
-    } else {
-        for (int r = 0; r < rows; ++r)
-            bulk_g2s(dst + (r / G::R) * G::RG_PITCH + (r % G::R) * G::ROW_BYTES, src + r * row_bytes_g,
-                     static_cast<uint32_t>(nblk * kQ4KBlockBytes), bar);
-    }
-}
 
 template <int LPR, int B, int NS, bool SOA>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_kernel(const Q4KParams p)
@@ -847,22 +727,10 @@ static Q4KPlan q4k_plan_half(long long N, int nb, int NS, int soa, int sm_count,
     return pl;
 }
 
-Q4KPlan q4k_plan(long long N, int K, int B, int NS, int soa, int sm_count, int smem_optin)
+// Full-block plan (fp32 kernel for any B, fixed-point kernel for B = 1):
+// `stage_bytes` is the shared memory the staged activations take per super-block.
+static Q4KPlan plan_full_block(long long N, int nb, int NS, int soa, int sm_count, int smem_optin, int stage_bytes)
 {
-    const int nb = K / kQ4KBlockElems;
-    if (B == 1) {
-        // Half-block lanes halve each warp's serial chain of slots (better when
-        // every warp gets only a few slots); full-block lanes spend fewer
-        // instructions per weight (better for long matrices).
-        const int full_lpr = (soa || nb % 16 == 0) ? 16 : 4;
-        const long long full_tiles = (N + (32 / full_lpr) * 2 - 1) / ((32 / full_lpr) * 2);
-        const long long slots = full_tiles * NS * ((nb + full_lpr - 1) / full_lpr);
-        if (slots < 8LL * sm_count * kMaxWarps) {
-            const Q4KPlan ph = q4k_plan_half(N, nb, NS, soa, sm_count, smem_optin);
-            if (ph.ok)
-                return ph;
-        }
-    }
     Q4KPlan pl{};
     const int misc = 256 /*argmax scratch, 16 B per warp*/ + 256 /*barriers*/;
     // SoA groups are 16 super-blocks, so SoA always walks K in 16-block chunks.
@@ -883,7 +751,7 @@ Q4KPlan q4k_plan(long long N, int K, int B, int NS, int soa, int sm_count, int s
             int cps = nchunk;
             for (;;) {
                 cps = (nchunk + splits - 1) / splits;
-                const int xb = B * cps * lpr * kXBlockPitch;
+                const int xb = cps * lpr * stage_bytes;
                 if (xb + min_ring + misc <= smem_optin || cps == 1)
                     break;
                 ++splits;
@@ -895,7 +763,7 @@ Q4KPlan q4k_plan(long long N, int K, int B, int NS, int soa, int sm_count, int s
                 cps = (nchunk + splits - 1) / splits;
             }
             splits = (nchunk + cps - 1) / cps;
-            const int x_bytes = (B * cps * lpr * kXBlockPitch + 127) & ~127;
+            const int x_bytes = (cps * lpr * stage_bytes + 127) & ~127;
             int depth = (smem_optin - x_bytes - misc) / (warps * sb);
             if (depth > 4)
                 depth = 4;
@@ -919,6 +787,31 @@ Q4KPlan q4k_plan(long long N, int K, int B, int NS, int soa, int sm_count, int s
         }
     }
     return pl;
+}
+
+Q4KPlan q4k_plan(long long N, int K, int B, int NS, int soa, int sm_count, int smem_optin)
+{
+    const int nb = K / kQ4KBlockElems;
+    if (B == 1) {
+        // batch 1: integer dot products on fixed-point activations
+        Q4KPlan pf = plan_full_block(N, nb, NS, soa, sm_count, smem_optin, q4k_fx_stage_bytes_per_block());
+        if (pf.ok) {
+            pf.fx = true;
+            return pf;
+        }
+        // Half-block lanes halve each warp's serial chain of slots (better when
+        // every warp gets only a few slots); full-block lanes spend fewer
+        // instructions per weight (better for long matrices).
+        const int full_lpr = (soa || nb % 16 == 0) ? 16 : 4;
+        const long long full_tiles = (N + (32 / full_lpr) * 2 - 1) / ((32 / full_lpr) * 2);
+        const long long slots = full_tiles * NS * ((nb + full_lpr - 1) / full_lpr);
+        if (slots < 8LL * sm_count * kMaxWarps) {
+            const Q4KPlan ph = q4k_plan_half(N, nb, NS, soa, sm_count, smem_optin);
+            if (ph.ok)
+                return ph;
+        }
+    }
+    return plan_full_block(N, nb, NS, soa, sm_count, smem_optin, B * kXBlockPitch);
 }
 
 template <int LPR, int B, int NS>
@@ -961,6 +854,8 @@ static cudaError_t launch_half(const Q4KParams &p, const Q4KPlan &pl, cudaStream
 
 cudaError_t q4k_gemv_launch(const Q4KParams &p, const Q4KPlan &pl, int B, int NS, cudaStream_t s)
 {
+    if (pl.fx)
+        return q4k_gemv_fx_launch(p, pl, NS, s);
     if (pl.half) {
         if (pl.lpr == 32)
             return NS == 1 ? launch_half<32, 1>(p, pl, s) : launch_half<32, 2>(p, pl, s);
