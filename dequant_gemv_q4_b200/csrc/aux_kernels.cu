@@ -35,16 +35,16 @@ int *device_error_flag(int device)
 // ---------------------------------------------------------------------------
 
 // Byte offset within a row of the header (byte < 16) or of quant slice s of
-// super-block kb in the SoA layout (groups of 16 super-blocks; see dqgemv.h).
+// super-block kb in the SoA layout (groups of kQ4KSoaGroup super-blocks; see dqgemv.h).
 __device__ __forceinline__ long long soa_hdr_off(int nb, int kb)
 {
-    const int first = (kb / 16) * 16;
+    const int first = (kb / kQ4KSoaGroup) * kQ4KSoaGroup;
     return static_cast<long long>(first) * kQ4KBlockBytes + 16 * (kb - first);
 }
 __device__ __forceinline__ long long soa_slice_off(int nb, int kb, int s)
 {
-    const int first = (kb / 16) * 16;
-    const int g = min(16, nb - first);
+    const int first = (kb / kQ4KSoaGroup) * kQ4KSoaGroup;
+    const int g = min(kQ4KSoaGroup, nb - first);
     return static_cast<long long>(first) * kQ4KBlockBytes + 16 * g + 16 * g * s + 16 * (kb - first);
 }
 

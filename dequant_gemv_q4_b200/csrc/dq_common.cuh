@@ -13,6 +13,9 @@ namespace dq {
 
 constexpr int kQ4KBlockElems = 256;
 constexpr int kQ4KBlockBytes = 144;
+// Q4_K structure-of-arrays layout: groups of this many super-blocks, each
+// group holding its headers and then its eight 16-byte quant slices.
+constexpr int kQ4KSoaGroup = 4;
 constexpr int kQ8BlockElems = 32;
 constexpr int kQ8BlockBytes = 34;
 

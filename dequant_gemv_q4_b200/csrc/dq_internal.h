@@ -34,7 +34,8 @@ struct Q4KPlan {
     bool ok;
     bool half;             // batch-1 half-block kernel (q4k_gemv_b1_kernel)
     bool fx;               // batch-1 fixed-point-activation kernel (q4k_gemv_fx_kernel)
-    int lpr;               // lanes per row group (4 or 16)
+    bool tma;              // fx kernel: slots moved by TMA tile copies
+    int lpr;               // lanes per row group (4, 8, 16 or 32)
     int R;                 // rows per lane
     int warps;             // warps per CTA
     long long tiles;
@@ -48,7 +49,8 @@ struct Q4KPlan {
 
 Q4KPlan q4k_plan(long long N, int K, int B, int NS, int soa, int sm_count, int smem_optin);
 cudaError_t q4k_gemv_launch(const Q4KParams &p, const Q4KPlan &pl, int B, int NS, cudaStream_t s);
-int q4k_fx_stage_bytes_per_block();
+int q4k_pick_warps(long long tiles, int sm_count, int max_warps, bool round4 = false);
+Q4KPlan q4k_plan_fx(long long N, int nb, int NS, int sm_count, int smem_optin);
 cudaError_t q4k_gemv_fx_launch(const Q4KParams &p, const Q4KPlan &pl, int NS, cudaStream_t s);
 
 // Q8_0 GEMV

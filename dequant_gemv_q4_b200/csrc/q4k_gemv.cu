@@ -206,16 +206,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_kernel(const Q4KPa
         if (l < nblk) {
             const uint8_t *slot_p = my_ring + slot * G::SLOT_BYTES + rg * G::RG_PITCH;
             // byte offsets of this lane's header and quant slices within a row of the slot
-            int hdr_off, qs_off0, qs_step;
-            if constexpr (SOA) {
-                hdr_off = 16 * l;
-                qs_off0 = 16 * nblk + 16 * l;
-                qs_step = 16 * nblk;
-            } else {
-                hdr_off = kQ4KBlockBytes * l;
-                qs_off0 = hdr_off + 16;
-                qs_step = 16;
-            }
+            const BlockOffsets bo = block_offsets<SOA>(l, nblk);
+            const int hdr_off = bo.hdr, qs_off0 = bo.qs0, qs_step = bo.qs_step;
             Hdr hd[R];
 #pragma unroll
             for (int r = 0; r < R; ++r)
@@ -502,16 +494,9 @@ __global__ void __launch_bounds__(kB1Warps * 32, 1) q4k_gemv_b1_kernel(const Q4K
         if (bl < nblk) {
             const uint8_t *slot_p = my_ring + slot * G::SLOT_BYTES + rg * G::RG_PITCH;
             // this lane's header and its first quant slice (slice 4*hh of the super-block)
-            int hdr_off, qs_off0, qs_step;
-            if constexpr (SOA) {
-                hdr_off = 16 * bl;
-                qs_step = 16 * nblk;
-                qs_off0 = 16 * nblk + 4 * hh * qs_step + 16 * bl;
-            } else {
-                hdr_off = kQ4KBlockBytes * bl;
-                qs_step = 16;
-                qs_off0 = hdr_off + 16 + 64 * hh;
-            }
+            const BlockOffsets bo = block_offsets<SOA>(bl, nblk);
+            const int hdr_off = bo.hdr, qs_step = bo.qs_step;
+            const int qs_off0 = bo.qs0 + 4 * hh * bo.qs_step;
             Hdr hd[R];
             uint32_t scw[R], mnw[R];
 #pragma unroll
@@ -662,7 +647,7 @@ int q4k_slot_bytes(int lpr) { return lpr == 16 ? Geo<16, 2>::SLOT_BYTES : Geo<4,
 // a multiple of four, so the four schedulers of an SM carry equal numbers of
 // warps (the full-block kernel skips the rounding when its shared memory
 // would then force a K split).
-static int pick_warps(long long tiles, int sm_count, int max_warps, bool round4)
+int q4k_pick_warps(long long tiles, int sm_count, int max_warps, bool round4)
 {
     long long w = (tiles + sm_count - 1) / sm_count;
     if (round4)
@@ -674,19 +659,19 @@ static int pick_warps(long long tiles, int sm_count, int max_warps, bool round4)
     return static_cast<int>(w);
 }
 
-static Q4KPlan q4k_plan_half(long long N, int nb, int NS, int soa, int sm_count, int smem_optin)
+static Q4KPlan q4k_plan_half(long long N, int nb, int NS, int sm_count, int smem_optin)
 {
     Q4KPlan pl{};
     const int misc = 256 /*argmax scratch*/ + 512 /*barriers*/;
-    // SoA groups are 16 super-blocks (the whole row when it has fewer), so SoA
-    // takes 16-block chunks unless a row has at most 4 super-blocks.
-    const int lpr = soa ? (nb <= 4 ? 8 : 32) : (nb % 16 == 0 ? 32 : 8);
+    // 16-block chunks when they tile the row, else 4-block chunks (both start
+    // at SoA group boundaries)
+    const int lpr = (nb % 16 == 0) ? 32 : 8;
     const int bpc = lpr / 2;
     const int sb = (lpr == 32) ? GeoHalf<32>::SLOT_BYTES : GeoHalf<8>::SLOT_BYTES;
     const int TR = (32 / lpr) * 2;
     const long long tiles = (N + TR - 1) / TR;
     const int nchunk = (nb + bpc - 1) / bpc;
-    const int w0 = pick_warps(tiles, sm_count, kB1Warps, true);
+    const int w0 = q4k_pick_warps(tiles, sm_count, kB1Warps, true);
     for (int warps = w0; warps >= 4 && !pl.ok; warps = (warps > 4 && warps / 2 < 4) ? 4 : warps / 2) {
         int splits = 1, cps = nchunk;
         for (;;) {
@@ -727,15 +712,16 @@ static Q4KPlan q4k_plan_half(long long N, int nb, int NS, int soa, int sm_count,
     return pl;
 }
 
-// Full-block plan (fp32 kernel for any B, fixed-point kernel for B = 1):
-// `stage_bytes` is the shared memory the staged activations take per super-block.
-static Q4KPlan plan_full_block(long long N, int nb, int NS, int soa, int sm_count, int smem_optin, int stage_bytes)
+// Full-block plan of the fp32 kernel: `stage_bytes` is the shared memory the
+// staged activations take per super-block.
+static Q4KPlan plan_full_block(long long N, int nb, int NS, int sm_count, int smem_optin, int stage_bytes)
 {
     Q4KPlan pl{};
     const int misc = 256 /*argmax scratch, 16 B per warp*/ + 256 /*barriers*/;
-    // SoA groups are 16 super-blocks, so SoA always walks K in 16-block chunks.
-    const int lpr_opts[2] = {(soa || nb % 16 == 0) ? 16 : 4, 4};
-    const int n_opts = (soa || nb % 16 != 0) ? 1 : 2;
+    // 16-block chunks when they tile the row, else 4-block chunks (both start
+    // at SoA group boundaries)
+    const int lpr_opts[2] = {(nb % 16 == 0) ? 16 : 4, 4};
+    const int n_opts = (nb % 16 != 0) ? 1 : 2;
     for (int oi = 0; oi < n_opts && !pl.ok; ++oi) {
         const int lpr = lpr_opts[oi];
         const int R = 2;
@@ -743,7 +729,7 @@ static Q4KPlan plan_full_block(long long N, int nb, int NS, int soa, int sm_coun
         const int TR = (32 / lpr) * R;
         const long long tiles = (N + TR - 1) / TR;
         const int nchunk = (nb + lpr - 1) / lpr;
-        const int w0 = pick_warps(tiles, sm_count, kMaxWarps, false);
+        const int w0 = q4k_pick_warps(tiles, sm_count, kMaxWarps, false);
         for (int warps = w0; warps >= 4 && !pl.ok; warps = (warps > 4 && warps / 2 < 4) ? 4 : warps / 2) {
             const int min_ring = warps * 2 * sb;
             // smallest split count whose activations fit beside a two-deep ring
@@ -794,24 +780,22 @@ Q4KPlan q4k_plan(long long N, int K, int B, int NS, int soa, int sm_count, int s
     const int nb = K / kQ4KBlockElems;
     if (B == 1) {
         // batch 1: integer dot products on fixed-point activations
-        Q4KPlan pf = plan_full_block(N, nb, NS, soa, sm_count, smem_optin, q4k_fx_stage_bytes_per_block());
-        if (pf.ok) {
-            pf.fx = true;
+        const Q4KPlan pf = q4k_plan_fx(N, nb, NS, sm_count, smem_optin);
+        if (pf.ok)
             return pf;
-        }
         // Half-block lanes halve each warp's serial chain of slots (better when
         // every warp gets only a few slots); full-block lanes spend fewer
         // instructions per weight (better for long matrices).
-        const int full_lpr = (soa || nb % 16 == 0) ? 16 : 4;
+        const int full_lpr = (nb % 16 == 0) ? 16 : 4;
         const long long full_tiles = (N + (32 / full_lpr) * 2 - 1) / ((32 / full_lpr) * 2);
         const long long slots = full_tiles * NS * ((nb + full_lpr - 1) / full_lpr);
         if (slots < 8LL * sm_count * kMaxWarps) {
-            const Q4KPlan ph = q4k_plan_half(N, nb, NS, soa, sm_count, smem_optin);
+            const Q4KPlan ph = q4k_plan_half(N, nb, NS, sm_count, smem_optin);
             if (ph.ok)
                 return ph;
         }
     }
-    return plan_full_block(N, nb, NS, soa, sm_count, smem_optin, B * kXBlockPitch);
+    return plan_full_block(N, nb, NS, sm_count, smem_optin, B * kXBlockPitch);
 }
 
 template <int LPR, int B, int NS>

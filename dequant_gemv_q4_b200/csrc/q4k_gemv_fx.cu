@@ -33,13 +33,29 @@
 //   i.e. 2^-30 of the largest activation of each super-block.
 //   A super-block of x holding an infinity or a NaN makes the rows' results NaN.
 //
-// Work decomposition: the full-block lanes of the fp32 kernel (lane l of a row
-// group owns super-block l of each K-chunk, two rows per lane) and its
-// per-warp bulk-copy rings; only the staging of x and the per-weight
-// arithmetic differ.
+// Work decomposition ("quarter-warp lanes").  A K-chunk is 4 super-blocks (one
+// SoA group, 576 contiguous bytes of a row in both layouts).  Lane (g, i) =
+// (lane / 8, lane % 8) handles super-block g of each chunk for rows i + 8r
+// (r < R) of a row tile of 8R rows, so the eight lanes of a quarter-warp read
+// the same activation bytes (a shared-memory broadcast) and distinct rows'
+// quants.  A slot is one chunk of one tile, 8R rows x 576 bytes.  Each warp
+// streams its own ring of slots as in the fp32 kernels; the four quarter sums
+// of a row are added with two shuffles.
+//
+// Slot copies.  When a row is a whole number of 64-byte units (K a multiple of
+// 1024) one TMA tile copy moves the slot: the matrix is described to the TMA
+// unit as [N rows][row/64 units][64 bytes] and a box of 16 x 9 x 64 bytes is
+// written with the 64-byte swizzle (16-byte chunk c of each 64-byte unit lands
+// at chunk c ^ ((offset >> 7) & 3)), which places the eight rows a quarter-warp
+// reads at one time in eight distinct bank groups.  Otherwise each row of the
+// slot is its own 1-D bulk copy, at a 592-byte pitch for the same purpose.
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_fp16.h>
 #include <cstdint>
+#include <cstring>
+#include <mutex>
 
 #include "dq_common.cuh"
 #include "dq_internal.h"
@@ -54,6 +70,35 @@ namespace dq {
 // again a distinct bank group per super-block).
 constexpr int kFxLimbPitch = 1040;
 constexpr int kFxAuxPitch = 80;
+
+constexpr int kFxRows = 2;                     // rows per lane (R)
+constexpr int kFxBPC = 4;                      // super-blocks per K-chunk
+constexpr int kFxChunkBytes = kFxBPC * kQ4KBlockBytes;   // 576
+constexpr int kFxTileRows = 8 * kFxRows;
+// slot bytes per row and per slot: padded rows for 1-D copies, dense swizzled rows for TMA
+template <bool TMA>
+struct FxSlot {
+    static constexpr int kRowPitch = TMA ? kFxChunkBytes : kFxChunkBytes + 16;
+    static constexpr int kBytes = kFxTileRows * kRowPitch;
+    // byte offset within the slot of byte `b` of row `row`
+    static __device__ __forceinline__ uint32_t off(int row, int b)
+    {
+        const uint32_t o = static_cast<uint32_t>(row * kRowPitch + b);
+        if constexpr (TMA)
+            return o ^ (((o >> 7) & 3u) << 4);
+        else
+            return o;
+    }
+};
+constexpr int kFxSlotAlign = 1024;   // the swizzle pattern repeats every 512 bytes
+constexpr int kFxMaxWarps = 12;
+static_assert(FxSlot<true>::kBytes % kFxSlotAlign == 0 && FxSlot<false>::kBytes % 128 == 0,
+              "slots must keep the ring aligned");
+
+// TMA descriptors of the (up to two) weight streams.
+struct FxMaps {
+    CUtensorMap m[2];
+};
 
 int q4k_fx_stage_bytes_per_block() { return kFxLimbPitch + kFxAuxPitch; }
 
@@ -144,27 +189,67 @@ __device__ __forceinline__ void fx_slice(const uint4 (&q)[R], const uint8_t *xlo
     }
 }
 
-template <int LPR, int NS, bool SOA>
-__global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_fx_kernel(const Q4KParams p)
+
+// Issues the copies of one slot (K-chunk c_begin + cur.kcl of stream cur.st of
+// the tile at cur.row0).  TMA: lane 0 arms the slot's mbarrier and issues one
+// tile copy (rows past N are filled with zeros and still counted).  Otherwise
+// lane 0 arms the mbarrier with the slot's byte count and lane r copies row r.
+template <bool TMA>
+__device__ __forceinline__ void fx_issue_slot(const Q4KParams &p, const FxMaps &maps, const Cursor &cur, int slot,
+                                              int c_begin, uint32_t ring_s, uint32_t bars_s, int lane)
 {
-    constexpr int R = 2;
-    using G = Geo<LPR, R>;
+    const int kb0 = (c_begin + cur.kcl) * kFxBPC;
+    const uint32_t bar = bars_s + slot * 8;
+    const uint32_t dst = ring_s + slot * FxSlot<TMA>::kBytes;
+    if constexpr (TMA) {
+        if (lane == 0) {
+            mbar_arrive_expect_tx(bar, static_cast<uint32_t>(FxSlot<true>::kBytes));
+            const CUtensorMap *m = cur.st == 0 ? &maps.m[0] : &maps.m[1];
+            asm volatile(
+                "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+                "[%5];" ::"r"(dst),
+                "l"(m), "r"(0), "r"(kb0 / kFxBPC * (kFxChunkBytes / 64)), "r"(static_cast<int>(cur.row0)), "r"(bar)
+                : "memory");
+        }
+    } else {
+        const long long row_bytes_g = static_cast<long long>(p.nb) * kQ4KBlockBytes;
+        const int rows = static_cast<int>(min(static_cast<long long>(kFxTileRows), p.N - cur.row0));
+        const int nblk = min(kFxBPC, p.nb - kb0);
+        const uint32_t bytes = static_cast<uint32_t>(nblk * kQ4KBlockBytes);
+        if (lane == 0)
+            mbar_arrive_expect_tx(bar, static_cast<uint32_t>(rows) * bytes);
+        __syncwarp();
+        if (lane < rows) {
+            const uint8_t *src = (cur.st == 0 ? p.w[0] : p.w[1]) + (cur.row0 + lane) * row_bytes_g +
+                                 static_cast<long long>(kb0) * kQ4KBlockBytes;
+            bulk_g2s(dst + lane * FxSlot<false>::kRowPitch, src, bytes, bar);
+        }
+    }
+}
+
+template <int NS, bool SOA, bool TMA>
+__global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
+    q4k_gemv_fx_kernel(const __grid_constant__ Q4KParams p, const __grid_constant__ FxMaps maps)
+{
+    using S = FxSlot<TMA>;
+    constexpr int R = kFxRows;
+    static_assert(R == 2, "the quarter reduction below is written for two rows per lane");
 
     extern __shared__ __align__(128) uint8_t smem[];
     const int nwarps = blockDim.x >> 5;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int rg = lane / LPR;
-    const int l = lane % LPR;
+    const int g = lane >> 3;   // super-block of each chunk
+    const int i = lane & 7;    // rows i and i + 8 of each tile
 
     const int split = blockIdx.x / p.ctas_per_split;
     const int cj = blockIdx.x % p.ctas_per_split;
-    const int nchunk_total = (p.nb + LPR - 1) / LPR;
+    const int nchunk_total = (p.nb + kFxBPC - 1) / kFxBPC;
     const int c_begin = split * p.chunks_per_split;
     const int c_end = min(c_begin + p.chunks_per_split, nchunk_total);
     const int nch = c_end - c_begin;
-    const int kb_begin = c_begin * LPR;
-    const int nbs = min(nch * LPR, p.nb - kb_begin);  // super-blocks of this split
+    const int kb_begin = c_begin * kFxBPC;
+    const int nbs = min(nch * kFxBPC, p.nb - kb_begin);  // super-blocks of this split
 
     // shared memory: [limb planes][sums and scales][barriers][ring][argmax scratch]
     const int x_bytes = (nbs * (kFxLimbPitch + kFxAuxPitch) + 127) & ~127;
@@ -172,34 +257,37 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_fx_kernel(const Q4
     uint8_t *aux = smem + nbs * kFxLimbPitch;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + x_bytes);
     const int bar_bytes = (nwarps * p.depth * 8 + 127) & ~127;
-    uint8_t *ring = smem + x_bytes + bar_bytes;
-    uint8_t *my_ring = ring + static_cast<size_t>(warp) * p.depth * G::SLOT_BYTES;
+    // the ring starts at the next kFxSlotAlign boundary of the shared window
+    const uint32_t ring_pad = (kFxSlotAlign - ((smem_u32(smem) + x_bytes + bar_bytes) & (kFxSlotAlign - 1))) &
+                              (kFxSlotAlign - 1);
+    uint8_t *ring = smem + x_bytes + bar_bytes + ring_pad;
+    uint8_t *my_ring = ring + static_cast<size_t>(warp) * p.depth * S::kBytes;
     const uint32_t my_ring_s = smem_u32(my_ring);
     const uint32_t my_bars_s = smem_u32(bars + warp * p.depth);
-    ArgmaxCand *red = reinterpret_cast<ArgmaxCand *>(ring + static_cast<size_t>(nwarps) * p.depth * G::SLOT_BYTES);
+    ArgmaxCand *red = reinterpret_cast<ArgmaxCand *>(ring + static_cast<size_t>(nwarps) * p.depth * S::kBytes);
 
     // this warp's tiles: t0, t0 + tstride, ... (warp-major order)
     const long long tstride = static_cast<long long>(p.ctas_per_split) * nwarps;
     const long long t0 = static_cast<long long>(warp) * p.ctas_per_split + cj;
     const long long ntiles_w = (t0 < p.tiles) ? (p.tiles - t0 + tstride - 1) / tstride : 0;
     const long long total = ntiles_w * NS * nch;
-    const long long row_step = tstride * G::TR;
+    const long long row_step = tstride * kFxTileRows;
 
-    // After the row-group reduction of the two row sums, lane 0 of the group
-    // holds row 0 and lane LPR/2 row 1 (LPR >= 2).
-    const bool writer = (l & (LPR / 2 - 1)) == 0;
-    const int wrow = (l >= LPR / 2) ? 1 : 0;
+    // after the quarter reduction lanes of quarters 0, 1 hold row i and
+    // quarters 2, 3 row i + 8; quarters 0 and 2 store
+    const bool writer = (lane & 8) == 0;
+    const int wrow = i + ((lane & 16) ? 8 : 0);
 
-    Cursor pc{t0 * G::TR, 0, 0};
+    Cursor pc{t0 * kFxTileRows, 0, 0};
     long long issued = 0;
     if (lane == 0) {
         for (int s = 0; s < p.depth; ++s)
             mbar_init(my_bars_s + s * 8, 1);
         mbar_fence_init();
     }
+    __syncwarp();
     for (int s = 0; s < p.depth && issued < total; ++s, ++issued) {
-        if (lane == 0)
-            issue_slot<G>(p, pc, s, c_begin, my_ring_s, my_bars_s);
+        fx_issue_slot<TMA>(p, maps, pc, s, c_begin, my_ring_s, my_bars_s, lane);
         pc.advance(nch, NS, row_step);
     }
 
@@ -210,10 +298,13 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_fx_kernel(const Q4
     long long best_i = 0x7fffffffffffffffLL;
     bool failed = false;
     long long consumed = 0;
-    double acc[R] = {0.0, 0.0};
+    double acc[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+        acc[r] = 0.0;
     double gsum = 0.0;  // stream-0 sum kept for the SwiGLU epilogue
 
-    Cursor cc{t0 * G::TR, 0, 0};
+    Cursor cc{t0 * kFxTileRows, 0, 0};
     int slot = 0;
     uint32_t parity = 0;
     for (; consumed < total; ++consumed) {
@@ -222,32 +313,23 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_fx_kernel(const Q4
             failed = true;
             break;
         }
-        const int kb0 = (c_begin + cc.kcl) * LPR;
-        const int nblk = min(LPR, p.nb - kb0);
-        if (l < nblk) {
-            const uint8_t *slot_p = my_ring + slot * G::SLOT_BYTES + rg * G::RG_PITCH;
-            int hdr_off, qs_off0, qs_step;
-            if constexpr (SOA) {
-                hdr_off = 16 * l;
-                qs_off0 = 16 * nblk + 16 * l;
-                qs_step = 16 * nblk;
-            } else {
-                hdr_off = kQ4KBlockBytes * l;
-                qs_off0 = hdr_off + 16;
-                qs_step = 16;
-            }
+        const int kb0 = (c_begin + cc.kcl) * kFxBPC;
+        const int nblk = min(kFxBPC, p.nb - kb0);
+        if (g < nblk) {
+            const uint8_t *slot_p = my_ring + slot * S::kBytes;
+            const BlockOffsets bo = block_offsets<SOA>(g, nblk);
             uint4 hd[R];
             uint32_t sc03[R], sc47[R];
 #pragma unroll
             for (int r = 0; r < R; ++r) {
-                hd[r] = *reinterpret_cast<const uint4 *>(slot_p + r * G::ROW_BYTES + hdr_off);
+                hd[r] = *reinterpret_cast<const uint4 *>(slot_p + S::off(i + 8 * r, bo.hdr));
                 // GGML get_scale_min_k4 packing: scales 0..3 are the low six bits of
                 // bytes 0..3; scales 4..7 take their low four bits from the low nibbles
                 // of bytes 8..11 and their top two bits from bits 6..7 of bytes 0..3
                 sc03[r] = hd[r].y & 0x3F3F3F3Fu;
                 sc47[r] = (hd[r].w & 0x0F0F0F0Fu) | ((hd[r].y >> 2) & 0x30303030u);
             }
-            const uint8_t *xb = limbs + (kb0 - kb_begin + l) * kFxLimbPitch;
+            const uint8_t *xb = limbs + (kb0 - kb_begin + g) * kFxLimbPitch;
 
             int isum[R][4];
 #pragma unroll
@@ -271,7 +353,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_fx_kernel(const Q4
                     uint4 q[R];
 #pragma unroll
                     for (int r = 0; r < R; ++r)
-                        q[r] = *reinterpret_cast<const uint4 *>(slot_p + r * G::ROW_BYTES + qs_off0 + s * qs_step);
+                        q[r] = *reinterpret_cast<const uint4 *>(slot_p + S::off(i + 8 * r, bo.qs0 + s * bo.qs_step));
                     fx_slice<R>(q, xb + 64 * c + 16 * h, xb + 64 * c + 32 + 16 * h, alo, ahi);
                 }
                 // fold the scales of sub-blocks 2c (lo) and 2c+1 (hi)
@@ -287,7 +369,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_fx_kernel(const Q4
             }
 
             // per row: y_sb = 2^-F (d I_s - dmin I_m) in fp64
-            const double *ap = reinterpret_cast<const double *>(aux + (kb0 - kb_begin + l) * kFxAuxPitch);
+            const double *ap = reinterpret_cast<const double *>(aux + (kb0 - kb_begin + g) * kFxAuxPitch);
             double X[8];
 #pragma unroll
             for (int j = 0; j < 8; j += 2) {
@@ -310,8 +392,12 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_fx_kernel(const Q4
                     const uint32_t mw = (j < 4) ? mn03 : mn47;
                     im = fma(static_cast<double>((mw >> (8 * (j & 3))) & 0xFFu), X[j], im);
                 }
-                const double d = static_cast<double>(__half2float(__ushort_as_half(static_cast<unsigned short>(hd[r].x & 0xFFFFu)))) * s2f;
-                const double dm = static_cast<double>(__half2float(__ushort_as_half(static_cast<unsigned short>(hd[r].x >> 16)))) * s2f;
+                const double d =
+                    static_cast<double>(__half2float(__ushort_as_half(static_cast<unsigned short>(hd[r].x & 0xFFFFu)))) *
+                    s2f;
+                const double dm =
+                    static_cast<double>(__half2float(__ushort_as_half(static_cast<unsigned short>(hd[r].x >> 16)))) *
+                    s2f;
                 const double pm = dm * im;            // rounded
                 const double em = fma(dm, im, -pm);   // its exact rounding error
                 acc[r] += fma(d, is, -pm) - em;
@@ -320,10 +406,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_fx_kernel(const Q4
 
         __syncwarp();
         if (issued < total) {
-            if (lane == 0) {
-                fence_proxy_async_smem();
-                issue_slot<G>(p, pc, slot, c_begin, my_ring_s, my_bars_s);
-            }
+            fence_proxy_async_smem();
+            fx_issue_slot<TMA>(p, maps, pc, slot, c_begin, my_ring_s, my_bars_s, lane);
             pc.advance(nch, NS, row_step);
             ++issued;
         }
@@ -339,34 +423,35 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_fx_kernel(const Q4
         if (!last_chunk)
             continue;
 
-        // end of this stream's K range for the tile: reduce across the row group
-        double v[R] = {acc[0], acc[1]};
+        // end of this stream's K range for the tile: add the four quarters' sums
+        const bool up = (lane & 16) != 0;
+        double t = (up ? acc[1] : acc[0]) + __shfl_xor_sync(0xffffffffu, up ? acc[0] : acc[1], 16);
+        t += __shfl_xor_sync(0xffffffffu, t, 8);
         acc[0] = 0.0;
         acc[1] = 0.0;
-        GroupReduce<LPR / 2, R, double>::run(v, l);
         if constexpr (NS == 2) {
             if (cur_st == 0) {
-                gsum = v[0];
+                gsum = t;
                 continue;
             }
         }
-        const long long n = row0 + rg * R + wrow;
+        const long long n = row0 + wrow;
         if (!writer || n >= p.N)
             continue;
         if (p.splits > 1) {
             if constexpr (NS == 2) {
                 p.part[(static_cast<long long>(split) * 2 + 0) * p.N + n] = static_cast<float>(gsum);
-                p.part[(static_cast<long long>(split) * 2 + 1) * p.N + n] = static_cast<float>(v[0]);
+                p.part[(static_cast<long long>(split) * 2 + 1) * p.N + n] = static_cast<float>(t);
             } else {
-                p.part[static_cast<long long>(split) * p.N + n] = static_cast<float>(v[0]);
+                p.part[static_cast<long long>(split) * p.N + n] = static_cast<float>(t);
             }
         } else {
             float out;
             if constexpr (NS == 2) {
-                const float g = static_cast<float>(gsum);
-                out = g / (1.0f + expf(-g)) * static_cast<float>(v[0]);
+                const float gv = static_cast<float>(gsum);
+                out = gv / (1.0f + expf(-gv)) * static_cast<float>(t);
             } else {
-                out = static_cast<float>(v[0]);
+                out = static_cast<float>(t);
             }
             p.y[n] = out;
             if (p.argmax && cand_better(out, n, best_v, best_i)) {
@@ -378,7 +463,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_fx_kernel(const Q4
 
     if (failed) {
         // the copies already issued into this warp's ring must land before the CTA exits
-        for (long long i = consumed; i < issued; ++i) {
+        for (long long k = consumed; k < issued; ++k) {
             mbar_wait_bounded(my_bars_s + slot * 8, parity, nullptr);
             if (++slot == p.depth) {
                 slot = 0;
@@ -413,22 +498,122 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_fx_kernel(const Q4
     }
 }
 
-template <int LPR, int NS>
-static cudaError_t launch_fx(const Q4KParams &p, const Q4KPlan &pl, cudaStream_t s)
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+// The driver's tensor-map encoder, looked up once (null when unavailable).
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 {
-    auto k = p.soa ? q4k_gemv_fx_kernel<LPR, NS, true> : q4k_gemv_fx_kernel<LPR, NS, false>;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+// Launch plan: slot copies by TMA when rows are whole 64-byte units; warps per
+// CTA from the tiles per SM; the fewest K splits whose activations fit beside
+// a two-deep ring per warp (more while fewer than half the warps would have a
+// tile); the deepest ring (up to 4) that fits.
+Q4KPlan q4k_plan_fx(long long N, int nb, int NS, int sm_count, int smem_optin)
+{
+    Q4KPlan pl{};
+    const bool tma = (nb % kFxBPC == 0) && N < 0x7FFFFFFFLL && tensor_map_encoder() != nullptr;
+    const int slot_bytes = tma ? FxSlot<true>::kBytes : FxSlot<false>::kBytes;
+    const int misc = 256 /*argmax scratch, 16 B per warp*/ + 512 /*barriers*/ + kFxSlotAlign /*ring alignment*/;
+    const int stage = kFxLimbPitch + kFxAuxPitch;
+    const long long tiles = (N + kFxTileRows - 1) / kFxTileRows;
+    const int nchunk = (nb + kFxBPC - 1) / kFxBPC;
+    const int w0 = q4k_pick_warps(tiles, sm_count, kFxMaxWarps);
+    for (int warps = w0; warps >= 4 && !pl.ok; --warps) {
+        int splits = 1;
+        int cps = nchunk;
+        for (;;) {
+            cps = (nchunk + splits - 1) / splits;
+            if (cps * kFxBPC * stage + warps * 2 * slot_bytes + misc <= smem_optin || cps == 1)
+                break;
+            ++splits;
+        }
+        const long long warps_total = static_cast<long long>(sm_count) * warps;
+        while (tiles * NS * splits * 2 < warps_total && splits < nchunk) {
+            ++splits;
+            cps = (nchunk + splits - 1) / splits;
+        }
+        splits = (nchunk + cps - 1) / cps;
+        const int x_bytes = (cps * kFxBPC * stage + 127) & ~127;
+        int depth = (smem_optin - x_bytes - misc) / (warps * slot_bytes);
+        if (depth > 4)
+            depth = 4;
+        if (depth < 2)
+            continue;
+        long long ctas = (tiles + warps - 1) / warps;
+        const long long max_ctas = sm_count / splits > 0 ? sm_count / splits : 1;
+        if (ctas > max_ctas)
+            ctas = max_ctas;
+        pl.fx = true;
+        pl.tma = tma;
+        pl.lpr = 8;
+        pl.R = kFxRows;
+        pl.warps = warps;
+        pl.tiles = tiles;
+        pl.splits = splits;
+        pl.chunks_per_split = cps;
+        pl.depth = depth;
+        pl.ctas_per_split = static_cast<int>(ctas);
+        pl.grid = pl.ctas_per_split * splits;
+        pl.smem = x_bytes + ((warps * depth * 8 + 127) & ~127) + kFxSlotAlign + warps * depth * slot_bytes + 256;
+        pl.ok = pl.smem <= smem_optin;
+    }
+    return pl;
+}
+
+// Describes one weight matrix to the TMA unit as [N][row / 64][64 bytes].
+static cudaError_t encode_weight_map(CUtensorMap *m, const uint8_t *w, long long N, int nb)
+{
+    const cuuint64_t row = static_cast<cuuint64_t>(nb) * kQ4KBlockBytes;
+    const cuuint64_t dims[3] = {16, row / 64, static_cast<cuuint64_t>(N)};
+    const cuuint64_t strides[2] = {64, row};
+    const cuuint32_t box[3] = {16, kFxChunkBytes / 64, kFxTileRows};
+    const cuuint32_t es[3] = {1, 1, 1};
+    const CUresult r = tensor_map_encoder()(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint8_t *>(w), dims,
+                                            strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                            CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int NS, bool TMA>
+static cudaError_t launch_fx(const Q4KParams &p, const FxMaps &maps, const Q4KPlan &pl, cudaStream_t s)
+{
+    auto k = p.soa ? q4k_gemv_fx_kernel<NS, true, TMA> : q4k_gemv_fx_kernel<NS, false, TMA>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
     if (e != cudaSuccess)
         return e;
-    k<<<pl.grid, pl.warps * 32, pl.smem, s>>>(p);
+    k<<<pl.grid, pl.warps * 32, pl.smem, s>>>(p, maps);
     return cudaGetLastError();
 }
 
 cudaError_t q4k_gemv_fx_launch(const Q4KParams &p, const Q4KPlan &pl, int NS, cudaStream_t s)
 {
-    if (pl.lpr == 16)
-        return NS == 1 ? launch_fx<16, 1>(p, pl, s) : launch_fx<16, 2>(p, pl, s);
-    return NS == 1 ? launch_fx<4, 1>(p, pl, s) : launch_fx<4, 2>(p, pl, s);
+    FxMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    if (pl.tma) {
+        for (int st = 0; st < NS; ++st) {
+            const cudaError_t e = encode_weight_map(&maps.m[st], p.w[st], p.N, p.nb);
+            if (e != cudaSuccess)
+                return e;
+        }
+        return NS == 1 ? launch_fx<1, true>(p, maps, pl, s) : launch_fx<2, true>(p, maps, pl, s);
+    }
+    return NS == 1 ? launch_fx<1, false>(p, maps, pl, s) : launch_fx<2, false>(p, maps, pl, s);
 }
 
 }  // namespace dq

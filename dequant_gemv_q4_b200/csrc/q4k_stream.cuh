@@ -87,6 +87,28 @@ struct Pow2Ceil<1> {
     static constexpr int value = 1;
 };
 
+// Byte offsets, within one row of a K-chunk of nblk super-blocks that starts
+// at an SoA group boundary, of super-block t's 16-byte header and of its first
+// quant slice, and the distance between its slices.
+struct BlockOffsets {
+    int hdr;
+    int qs0;
+    int qs_step;
+};
+template <bool SOA>
+__device__ __forceinline__ BlockOffsets block_offsets(int t, int nblk)
+{
+    if constexpr (SOA) {
+        const int grp = t / kQ4KSoaGroup;
+        const int tt = t % kQ4KSoaGroup;
+        const int gsz = min(kQ4KSoaGroup, nblk - grp * kQ4KSoaGroup);
+        const int base = grp * kQ4KSoaGroup * kQ4KBlockBytes;
+        return {base + 16 * tt, base + 16 * gsz + 16 * tt, 16 * gsz};
+    } else {
+        return {kQ4KBlockBytes * t, kQ4KBlockBytes * t + 16, 16};
+    }
+}
+
 // Position of a warp in its slot sequence: the tile's first row row0, weight
 // stream st, K-chunk kcl (relative to the split's first chunk).  row0 moves by
 // the warp's tile stride once every stream and chunk of a tile are done.

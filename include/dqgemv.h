@@ -120,8 +120,8 @@ dq_status q4k_swiglu_gemv(const void *w_gate, const void *w_up, int layout, cons
  * library's structure-of-arrays order (qualiaDB cuda_lane:
  * preload_q4k_soa_weights; the pages do not define the SoA layout, this is the
  * library's own).  Every row keeps its byte range and size.  Within a row the
- * super-blocks are taken in groups of 16 (the last group holds the remaining
- * g <= 16); a group of g blocks is stored as g 16-byte headers (d, dmin, 12
+ * super-blocks are taken in groups of 4 (the last group holds the remaining
+ * g <= 4); a group of g blocks is stored as g 16-byte headers (d, dmin, 12
  * scale bytes of block t at 16*t) followed by 8 slices, slice s holding quant
  * bytes 16s..16s+15 of each block t at 16*g + 16*g*s + 16*t.
  *   w_aos, w_soa  N*(K/256)*144 bytes each, 16-byte aligned, not overlapping.

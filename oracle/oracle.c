@@ -42,7 +42,7 @@
 #define Q8_0_BLOCK_BYTES 34
 #define Q4K_BLOCK_ELEMS 256
 #define Q4K_BLOCK_BYTES 144
-#define Q4K_SOA_GROUP 16
+#define Q4K_SOA_GROUP 4
 
 /* ------------------------------------------------------------------------ */
 /* IEEE 754 binary16 -> double.  1 sign bit, 5 exponent bits (bias 15),     */
@@ -143,9 +143,9 @@ void oracle_q8_0_block(const uint8_t *blk, double *w)
 /* Structure-of-arrays layout of Q4_K (this library's definition).          */
 /*                                                                          */
 /* Each row keeps its byte range and its size (144 bytes per super-block).  */
-/* Within the row, the super-blocks are taken in groups of 16 consecutive   */
-/* blocks (the last group of a row holds the remaining g <= 16 blocks).     */
-/* A group of g blocks, starting at byte 144 * 16 * group of the row, is    */
+/* Within the row, the super-blocks are taken in groups of 4 consecutive    */
+/* blocks (the last group of a row holds the remaining g <= 4 blocks).      */
+/* A group of g blocks, starting at byte 144 * 4 * group of the row, is     */
 /* stored as                                                                */
 /*   g headers of 16 bytes:  header t = bytes 0..15 of block t             */
 /*                           (d, dmin, 12 scale bytes)                     */

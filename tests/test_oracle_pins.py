@@ -312,16 +312,16 @@ def test_soa_repack_is_a_row_permutation_and_decodes_identically(N, K):
 
 
 def test_soa_positions_hand_derived():
-    # one row of 20 super-blocks: a full group of 16 and a partial group of 4.
-    N, K = 1, 20 * 256
-    w = np.zeros((1, 20 * 144), np.uint8)
+    # one row of 6 super-blocks: a full group of 4 and a partial group of 2.
+    N, K = 1, 6 * 256
+    w = np.zeros((1, 6 * 144), np.uint8)
     w[0, 1 * 144 + 0] = 11            # block 1, header byte 0
     w[0, 0 * 144 + 16 + 16] = 22      # block 0, quant byte 16 (slice 1, byte 0)
-    w[0, 17 * 144 + 16 + 127] = 33    # block 17 (group 1, t=1, g=4), quant byte 127 (slice 7, byte 15)
+    w[0, 5 * 144 + 16 + 127] = 33     # block 5 (group 1, t=1, g=2), quant byte 127 (slice 7, byte 15)
     soa = oracle.q4k_repack_soa(w, N, K)
-    # group 0: 16 headers (256 B), then slice s of block t at 256 + 256*s + 16*t
+    # group 0: 4 headers (64 B), then slice s of block t at 64 + 64*s + 16*t
     assert soa[0, 16] == 11
-    assert soa[0, 256 + 256 * 1 + 0] == 22
-    # group 1 starts at byte 16*144 = 2304: 4 headers (64 B), slice s of block t at 64 + 64*s + 16*t
-    assert soa[0, 2304 + 64 + 64 * 7 + 16 * 1 + 15] == 33
+    assert soa[0, 64 + 64 * 1 + 0] == 22
+    # group 1 starts at byte 4*144 = 576: 2 headers (32 B), slice s of block t at 32 + 32*s + 16*t
+    assert soa[0, 576 + 32 + 32 * 7 + 16 * 1 + 15] == 33
     assert int(np.count_nonzero(soa)) == 3
