@@ -191,6 +191,8 @@ __global__ void __launch_bounds__(kReduceThreads) splitk_reduce_kernel(const flo
                                                                        int NS, int B, long long N,
                                                                        float *__restrict__ y, ArgmaxCand *cand)
 {
+    pdl_wait();
+    pdl_launch_dependents();
     float best_v = -INFINITY;
     long long best_i = 0x7fffffffffffffffLL;
     const long long total = N * B;
@@ -240,14 +242,15 @@ __global__ void __launch_bounds__(kReduceThreads) splitk_reduce_kernel(const flo
 cudaError_t splitk_reduce_launch(const float *part, int splits, int NS, int B, long long N, float *y,
                                  ArgmaxCand *cand, int grid, cudaStream_t s)
 {
-    splitk_reduce_kernel<<<grid, kReduceThreads, 0, s>>>(part, splits, NS, B, N, y, cand);
-    return cudaGetLastError();
+    return launch_pdl(splitk_reduce_kernel, dim3(grid), dim3(kReduceThreads), 0, s, part, splits, NS, B, N, y, cand);
 }
 
 // One CTA folds all candidates into the final index.
 __global__ void __launch_bounds__(1024) argmax_finalize_kernel(const ArgmaxCand *__restrict__ cand, int ncand,
                                                                long long *out)
 {
+    pdl_wait();
+    pdl_launch_dependents();
     float best_v = -INFINITY;
     long long best_i = 0x7fffffffffffffffLL;
     for (int i = threadIdx.x; i < ncand; i += blockDim.x)
@@ -282,8 +285,7 @@ __global__ void __launch_bounds__(1024) argmax_finalize_kernel(const ArgmaxCand 
 
 cudaError_t argmax_finalize_launch(const ArgmaxCand *cand, int ncand, long long *out, cudaStream_t s)
 {
-    argmax_finalize_kernel<<<1, 1024, 0, s>>>(cand, ncand, out);
-    return cudaGetLastError();
+    return launch_pdl(argmax_finalize_kernel, dim3(1), dim3(1024), 0, s, cand, ncand, out);
 }
 
 }  // namespace dq

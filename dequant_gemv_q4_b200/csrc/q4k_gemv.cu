@@ -65,6 +65,8 @@ constexpr int kXBlockPitch = 1040;
 template <int LPR, int B, int NS, bool SOA>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_kernel(const Q4KParams p)
 {
+    pdl_wait();
+    pdl_launch_dependents();
     constexpr int R = 2;
     using G = Geo<LPR, R>;
     constexpr int MV = R * B;                         // values per lane per stream
@@ -380,6 +382,8 @@ constexpr int kXHalfGap = 528;
 template <int LPR, int NS, bool SOA>
 __global__ void __launch_bounds__(kB1Warps * 32, 1) q4k_gemv_b1_kernel(const Q4KParams p)
 {
+    pdl_wait();
+    pdl_launch_dependents();
     using G = GeoHalf<LPR>;
     constexpr int R = G::R;
 
@@ -805,8 +809,7 @@ static cudaError_t launch_one(const Q4KParams &p, const Q4KPlan &pl, cudaStream_
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
     if (e != cudaSuccess)
         return e;
-    k<<<pl.grid, pl.warps * 32, pl.smem, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(k, dim3(pl.grid), dim3(pl.warps * 32), pl.smem, s, p);
 }
 
 template <int LPR, int NS>
@@ -832,8 +835,7 @@ static cudaError_t launch_half(const Q4KParams &p, const Q4KPlan &pl, cudaStream
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
     if (e != cudaSuccess)
         return e;
-    k<<<pl.grid, pl.warps * 32, pl.smem, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(k, dim3(pl.grid), dim3(pl.warps * 32), pl.smem, s, p);
 }
 
 cudaError_t q4k_gemv_launch(const Q4KParams &p, const Q4KPlan &pl, int B, int NS, cudaStream_t s)

@@ -42,13 +42,13 @@
 // streams its own ring of slots as in the fp32 kernels; the four quarter sums
 // of a row are added with two shuffles.
 //
-// Slot copies.  When a row is a whole number of 64-byte units (K a multiple of
-// 1024) one TMA tile copy moves the slot: the matrix is described to the TMA
-// unit as [N rows][row/64 units][64 bytes] and a box of 16 x 9 x 64 bytes is
-// written with the 64-byte swizzle (16-byte chunk c of each 64-byte unit lands
-// at chunk c ^ ((offset >> 7) & 3)), which places the eight rows a quarter-warp
-// reads at one time in eight distinct bank groups.  Otherwise each row of the
-// slot is its own 1-D bulk copy, at a 592-byte pitch for the same purpose.
+// Slot copies.  Slot rows sit at a 592-byte pitch (576 + 16), which places the
+// eight rows a quarter-warp reads at one time in eight distinct bank groups.
+// One TMA tile copy moves a slot: the matrix is described to the TMA unit as
+// [N rows][row bytes / 4] 32-bit words and a box of 16 rows x 148 words is
+// copied, i.e. each row's chunk plus the next 16 bytes of that row (zeros past
+// its end), so the box itself lays the rows out at the padded pitch.  Without
+// the driver's tensor-map encoder each row is its own 1-D bulk copy instead.
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -64,10 +64,10 @@
 namespace dq {
 
 // Staged activations of one super-block: four limb planes of 256 bytes (plane
-// l, byte k = limb l of xi_k), 16 bytes of padding so that the lanes of one
-// shared-memory phase (eight consecutive super-blocks) hit distinct bank
-// groups; then, in a separate array, X_0..X_7 and 2^-F as fp64 (80-byte pitch,
-// again a distinct bank group per super-block).
+// l, byte k = limb l of xi_k) and 16 bytes of padding, which shifts the bank
+// group from one super-block to the next; then, in a separate array, X_0..X_7
+// and 2^-F as fp64 (80-byte pitch).  The lanes of a quarter-warp read the same
+// super-block, so these reads are broadcasts.
 constexpr int kFxLimbPitch = 1040;
 constexpr int kFxAuxPitch = 80;
 
@@ -75,32 +75,15 @@ constexpr int kFxRows = 2;                     // rows per lane (R)
 constexpr int kFxBPC = 4;                      // super-blocks per K-chunk
 constexpr int kFxChunkBytes = kFxBPC * kQ4KBlockBytes;   // 576
 constexpr int kFxTileRows = 8 * kFxRows;
-// slot bytes per row and per slot: padded rows for 1-D copies, dense swizzled rows for TMA
-template <bool TMA>
-struct FxSlot {
-    static constexpr int kRowPitch = TMA ? kFxChunkBytes : kFxChunkBytes + 16;
-    static constexpr int kBytes = kFxTileRows * kRowPitch;
-    // byte offset within the slot of byte `b` of row `row`
-    static __device__ __forceinline__ uint32_t off(int row, int b)
-    {
-        const uint32_t o = static_cast<uint32_t>(row * kRowPitch + b);
-        if constexpr (TMA)
-            return o ^ (((o >> 7) & 3u) << 4);
-        else
-            return o;
-    }
-};
-constexpr int kFxSlotAlign = 1024;   // the swizzle pattern repeats every 512 bytes
+constexpr int kFxRowPitch = kFxChunkBytes + 16;           // 592
+constexpr int kFxSlotBytes = kFxTileRows * kFxRowPitch;
+static_assert(kFxSlotBytes % 128 == 0, "slots must keep the ring 128-byte aligned");
 constexpr int kFxMaxWarps = 12;
-static_assert(FxSlot<true>::kBytes % kFxSlotAlign == 0 && FxSlot<false>::kBytes % 128 == 0,
-              "slots must keep the ring aligned");
 
 // TMA descriptors of the (up to two) weight streams.
 struct FxMaps {
     CUtensorMap m[2];
 };
-
-int q4k_fx_stage_bytes_per_block() { return kFxLimbPitch + kFxAuxPitch; }
 
 // Converts the activations of super-blocks kb_begin .. kb_begin + nbs - 1 into
 // limb planes and sums; one warp per super-block.
@@ -192,23 +175,25 @@ __device__ __forceinline__ void fx_slice(const uint4 (&q)[R], const uint8_t *xlo
 
 // Issues the copies of one slot (K-chunk c_begin + cur.kcl of stream cur.st of
 // the tile at cur.row0).  TMA: lane 0 arms the slot's mbarrier and issues one
-// tile copy (rows past N are filled with zeros and still counted).  Otherwise
-// lane 0 arms the mbarrier with the slot's byte count and lane r copies row r.
+// tile copy (elements past the matrix are filled with zeros and still counted).
+// Otherwise lane 0 arms the mbarrier with the slot's byte count and lane r
+// copies row r.
 template <bool TMA>
 __device__ __forceinline__ void fx_issue_slot(const Q4KParams &p, const FxMaps &maps, const Cursor &cur, int slot,
                                               int c_begin, uint32_t ring_s, uint32_t bars_s, int lane)
 {
     const int kb0 = (c_begin + cur.kcl) * kFxBPC;
     const uint32_t bar = bars_s + slot * 8;
-    const uint32_t dst = ring_s + slot * FxSlot<TMA>::kBytes;
+    const uint32_t dst = ring_s + slot * kFxSlotBytes;
     if constexpr (TMA) {
         if (lane == 0) {
-            mbar_arrive_expect_tx(bar, static_cast<uint32_t>(FxSlot<true>::kBytes));
+            mbar_arrive_expect_tx(bar, static_cast<uint32_t>(kFxSlotBytes));
             const CUtensorMap *m = cur.st == 0 ? &maps.m[0] : &maps.m[1];
+            // x = kb0 * 36 words: a multiple of 4 words, i.e. of 16 bytes
             asm volatile(
-                "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
-                "[%5];" ::"r"(dst),
-                "l"(m), "r"(0), "r"(kb0 / kFxBPC * (kFxChunkBytes / 64)), "r"(static_cast<int>(cur.row0)), "r"(bar)
+                "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+                "[%4];" ::"r"(dst),
+                "l"(m), "r"(kb0 * (kQ4KBlockBytes / 4)), "r"(static_cast<int>(cur.row0)), "r"(bar)
                 : "memory");
         }
     } else {
@@ -222,7 +207,7 @@ __device__ __forceinline__ void fx_issue_slot(const Q4KParams &p, const FxMaps &
         if (lane < rows) {
             const uint8_t *src = (cur.st == 0 ? p.w[0] : p.w[1]) + (cur.row0 + lane) * row_bytes_g +
                                  static_cast<long long>(kb0) * kQ4KBlockBytes;
-            bulk_g2s(dst + lane * FxSlot<false>::kRowPitch, src, bytes, bar);
+            bulk_g2s(dst + lane * kFxRowPitch, src, bytes, bar);
         }
     }
 }
@@ -231,7 +216,6 @@ template <int NS, bool SOA, bool TMA>
 __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
     q4k_gemv_fx_kernel(const __grid_constant__ Q4KParams p, const __grid_constant__ FxMaps maps)
 {
-    using S = FxSlot<TMA>;
     constexpr int R = kFxRows;
     static_assert(R == 2, "the quarter reduction below is written for two rows per lane");
 
@@ -257,14 +241,13 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
     uint8_t *aux = smem + nbs * kFxLimbPitch;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + x_bytes);
     const int bar_bytes = (nwarps * p.depth * 8 + 127) & ~127;
-    // the ring starts at the next kFxSlotAlign boundary of the shared window
-    const uint32_t ring_pad = (kFxSlotAlign - ((smem_u32(smem) + x_bytes + bar_bytes) & (kFxSlotAlign - 1))) &
-                              (kFxSlotAlign - 1);
+    // TMA writes shared memory at 128-byte aligned addresses: align the ring
+    const uint32_t ring_pad = (128u - ((smem_u32(smem) + x_bytes + bar_bytes) & 127u)) & 127u;
     uint8_t *ring = smem + x_bytes + bar_bytes + ring_pad;
-    uint8_t *my_ring = ring + static_cast<size_t>(warp) * p.depth * S::kBytes;
+    uint8_t *my_ring = ring + static_cast<size_t>(warp) * p.depth * kFxSlotBytes;
     const uint32_t my_ring_s = smem_u32(my_ring);
     const uint32_t my_bars_s = smem_u32(bars + warp * p.depth);
-    ArgmaxCand *red = reinterpret_cast<ArgmaxCand *>(ring + static_cast<size_t>(nwarps) * p.depth * S::kBytes);
+    ArgmaxCand *red = reinterpret_cast<ArgmaxCand *>(ring + static_cast<size_t>(nwarps) * p.depth * kFxSlotBytes);
 
     // this warp's tiles: t0, t0 + tstride, ... (warp-major order)
     const long long tstride = static_cast<long long>(p.ctas_per_split) * nwarps;
@@ -286,6 +269,9 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
         mbar_fence_init();
     }
     __syncwarp();
+    // the weights too may come from the previous kernel (a repack, an upload)
+    pdl_wait();
+    pdl_launch_dependents();
     for (int s = 0; s < p.depth && issued < total; ++s, ++issued) {
         fx_issue_slot<TMA>(p, maps, pc, s, c_begin, my_ring_s, my_bars_s, lane);
         pc.advance(nch, NS, row_step);
@@ -316,13 +302,13 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
         const int kb0 = (c_begin + cc.kcl) * kFxBPC;
         const int nblk = min(kFxBPC, p.nb - kb0);
         if (g < nblk) {
-            const uint8_t *slot_p = my_ring + slot * S::kBytes;
+            const uint8_t *slot_p = my_ring + slot * kFxSlotBytes + i * kFxRowPitch;
             const BlockOffsets bo = block_offsets<SOA>(g, nblk);
             uint4 hd[R];
             uint32_t sc03[R], sc47[R];
 #pragma unroll
             for (int r = 0; r < R; ++r) {
-                hd[r] = *reinterpret_cast<const uint4 *>(slot_p + S::off(i + 8 * r, bo.hdr));
+                hd[r] = *reinterpret_cast<const uint4 *>(slot_p + 8 * r * kFxRowPitch + bo.hdr);
                 // GGML get_scale_min_k4 packing: scales 0..3 are the low six bits of
                 // bytes 0..3; scales 4..7 take their low four bits from the low nibbles
                 // of bytes 8..11 and their top two bits from bits 6..7 of bytes 0..3
@@ -353,7 +339,8 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
                     uint4 q[R];
 #pragma unroll
                     for (int r = 0; r < R; ++r)
-                        q[r] = *reinterpret_cast<const uint4 *>(slot_p + S::off(i + 8 * r, bo.qs0 + s * bo.qs_step));
+                        q[r] = *reinterpret_cast<const uint4 *>(slot_p + 8 * r * kFxRowPitch + bo.qs0 +
+                                                                s * bo.qs_step);
                     fx_slice<R>(q, xb + 64 * c + 16 * h, xb + 64 * c + 32 + 16 * h, alo, ahi);
                 }
                 // fold the scales of sub-blocks 2c (lo) and 2c+1 (hi)
@@ -386,12 +373,14 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
                 is = fma(is, 256.0, static_cast<double>(isum[r][0]));
                 const uint32_t mn03 = hd[r].z & 0x3F3F3F3Fu;
                 const uint32_t mn47 = ((hd[r].w >> 4) & 0x0F0F0F0Fu) | ((hd[r].z >> 2) & 0x30303030u);
-                double im = 0.0;
+                // I_m as a tree of exact products and sums (integers below 2^53)
+                double pmn[8];
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const uint32_t mw = (j < 4) ? mn03 : mn47;
-                    im = fma(static_cast<double>((mw >> (8 * (j & 3))) & 0xFFu), X[j], im);
+                    pmn[j] = static_cast<double>((mw >> (8 * (j & 3))) & 0xFFu) * X[j];
                 }
+                const double im = ((pmn[0] + pmn[1]) + (pmn[2] + pmn[3])) + ((pmn[4] + pmn[5]) + (pmn[6] + pmn[7]));
                 const double d =
                     static_cast<double>(__half2float(__ushort_as_half(static_cast<unsigned short>(hd[r].x & 0xFFFFu)))) *
                     s2f;
@@ -519,37 +508,33 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
     return fn;
 }
 
-// Launch plan: slot copies by TMA when rows are whole 64-byte units; warps per
-// CTA from the tiles per SM; the fewest K splits whose activations fit beside
-// a two-deep ring per warp (more while fewer than half the warps would have a
-// tile); the deepest ring (up to 4) that fits.
+// Launch plan.  Slot copies by TMA when the driver's encoder is available.  K
+// is split until there are about eight tile tasks per SM (or each split is one
+// chunk), warps per CTA follow from the tasks per SM, and K is split further
+// if the activations would not fit beside a two-deep ring per warp; the ring
+// is as deep as shared memory allows, up to 4 slots.
 Q4KPlan q4k_plan_fx(long long N, int nb, int NS, int sm_count, int smem_optin)
 {
     Q4KPlan pl{};
-    const bool tma = (nb % kFxBPC == 0) && N < 0x7FFFFFFFLL && tensor_map_encoder() != nullptr;
-    const int slot_bytes = tma ? FxSlot<true>::kBytes : FxSlot<false>::kBytes;
-    const int misc = 256 /*argmax scratch, 16 B per warp*/ + 512 /*barriers*/ + kFxSlotAlign /*ring alignment*/;
+    const bool tma = N < 0x7FFFFFFFLL && tensor_map_encoder() != nullptr;
+    const int misc = 256 /*argmax scratch, 16 B per warp*/ + 512 /*barriers*/ + 128 /*ring alignment*/;
     const int stage = kFxLimbPitch + kFxAuxPitch;
     const long long tiles = (N + kFxTileRows - 1) / kFxTileRows;
     const int nchunk = (nb + kFxBPC - 1) / kFxBPC;
-    const int w0 = q4k_pick_warps(tiles, sm_count, kFxMaxWarps);
+    int splits_par = 1;
+    while (tiles * splits_par < 8LL * sm_count && splits_par < nchunk)
+        ++splits_par;
+    const int w0 = q4k_pick_warps(tiles * splits_par, sm_count, kFxMaxWarps);
     for (int warps = w0; warps >= 4 && !pl.ok; --warps) {
-        int splits = 1;
-        int cps = nchunk;
-        for (;;) {
-            cps = (nchunk + splits - 1) / splits;
-            if (cps * kFxBPC * stage + warps * 2 * slot_bytes + misc <= smem_optin || cps == 1)
-                break;
-            ++splits;
-        }
-        const long long warps_total = static_cast<long long>(sm_count) * warps;
-        while (tiles * NS * splits * 2 < warps_total && splits < nchunk) {
+        int splits = splits_par;
+        int cps = (nchunk + splits - 1) / splits;
+        while (cps * kFxBPC * stage + warps * 2 * kFxSlotBytes + misc > smem_optin && cps > 1) {
             ++splits;
             cps = (nchunk + splits - 1) / splits;
         }
         splits = (nchunk + cps - 1) / cps;
         const int x_bytes = (cps * kFxBPC * stage + 127) & ~127;
-        int depth = (smem_optin - x_bytes - misc) / (warps * slot_bytes);
+        int depth = (smem_optin - x_bytes - misc) / (warps * kFxSlotBytes);
         if (depth > 4)
             depth = 4;
         if (depth < 2)
@@ -569,24 +554,24 @@ Q4KPlan q4k_plan_fx(long long N, int nb, int NS, int sm_count, int smem_optin)
         pl.depth = depth;
         pl.ctas_per_split = static_cast<int>(ctas);
         pl.grid = pl.ctas_per_split * splits;
-        pl.smem = x_bytes + ((warps * depth * 8 + 127) & ~127) + kFxSlotAlign + warps * depth * slot_bytes + 256;
+        pl.smem = x_bytes + ((warps * depth * 8 + 127) & ~127) + 128 + warps * depth * kFxSlotBytes + 256;
         pl.ok = pl.smem <= smem_optin;
     }
     return pl;
 }
 
-// Describes one weight matrix to the TMA unit as [N][row / 64][64 bytes].
+// Describes one weight matrix to the TMA unit as [N][row bytes / 4] 32-bit words
+// with a box of one slot: 16 rows x (576 + 16) bytes.
 static cudaError_t encode_weight_map(CUtensorMap *m, const uint8_t *w, long long N, int nb)
 {
     const cuuint64_t row = static_cast<cuuint64_t>(nb) * kQ4KBlockBytes;
-    const cuuint64_t dims[3] = {16, row / 64, static_cast<cuuint64_t>(N)};
-    const cuuint64_t strides[2] = {64, row};
-    const cuuint32_t box[3] = {16, kFxChunkBytes / 64, kFxTileRows};
-    const cuuint32_t es[3] = {1, 1, 1};
-    const CUresult r = tensor_map_encoder()(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint8_t *>(w), dims,
-                                            strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                                            CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    const cuuint64_t dims[2] = {row / 4, static_cast<cuuint64_t>(N)};
+    const cuuint64_t strides[1] = {row};
+    const cuuint32_t box[2] = {kFxRowPitch / 4, kFxTileRows};
+    const cuuint32_t es[2] = {1, 1};
+    const CUresult r = tensor_map_encoder()(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint8_t *>(w), dims,
+                                            strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
@@ -597,8 +582,7 @@ static cudaError_t launch_fx(const Q4KParams &p, const FxMaps &maps, const Q4KPl
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
     if (e != cudaSuccess)
         return e;
-    k<<<pl.grid, pl.warps * 32, pl.smem, s>>>(p, maps);
-    return cudaGetLastError();
+    return launch_pdl(k, dim3(pl.grid), dim3(pl.warps * 32), pl.smem, s, p, maps);
 }
 
 cudaError_t q4k_gemv_fx_launch(const Q4KParams &p, const Q4KPlan &pl, int NS, cudaStream_t s)

@@ -50,6 +50,8 @@ struct WarpReduceT {
 template <int B>
 __global__ void __launch_bounds__(kQ8Threads) q8_0_gemv_kernel(const Q8Params p)
 {
+    pdl_wait();
+    pdl_launch_dependents();
     constexpr int MV = kQ8RowsPerWarp * B;
     constexpr int MP = (MV <= 2) ? 2 : (MV <= 4) ? 4 : (MV <= 8) ? 8 : 16;
     __shared__ __align__(16) uint8_t tile[kQ8Rows * kQ8RowPitch];
@@ -201,17 +203,16 @@ Q8Plan q8_plan(long long N, int K, int B, int sm_count, int smem_optin)
 cudaError_t q8_0_gemv_launch(const Q8Params &p, const Q8Plan &pl, int B, cudaStream_t s)
 {
     switch (B) {
-    case 1: q8_0_gemv_kernel<1><<<pl.grid, pl.block, 0, s>>>(p); break;
-    case 2: q8_0_gemv_kernel<2><<<pl.grid, pl.block, 0, s>>>(p); break;
-    case 3: q8_0_gemv_kernel<3><<<pl.grid, pl.block, 0, s>>>(p); break;
-    case 4: q8_0_gemv_kernel<4><<<pl.grid, pl.block, 0, s>>>(p); break;
-    case 5: q8_0_gemv_kernel<5><<<pl.grid, pl.block, 0, s>>>(p); break;
-    case 6: q8_0_gemv_kernel<6><<<pl.grid, pl.block, 0, s>>>(p); break;
-    case 7: q8_0_gemv_kernel<7><<<pl.grid, pl.block, 0, s>>>(p); break;
-    case 8: q8_0_gemv_kernel<8><<<pl.grid, pl.block, 0, s>>>(p); break;
+    case 1: return launch_pdl(q8_0_gemv_kernel<1>, dim3(pl.grid), dim3(pl.block), 0, s, p);
+    case 2: return launch_pdl(q8_0_gemv_kernel<2>, dim3(pl.grid), dim3(pl.block), 0, s, p);
+    case 3: return launch_pdl(q8_0_gemv_kernel<3>, dim3(pl.grid), dim3(pl.block), 0, s, p);
+    case 4: return launch_pdl(q8_0_gemv_kernel<4>, dim3(pl.grid), dim3(pl.block), 0, s, p);
+    case 5: return launch_pdl(q8_0_gemv_kernel<5>, dim3(pl.grid), dim3(pl.block), 0, s, p);
+    case 6: return launch_pdl(q8_0_gemv_kernel<6>, dim3(pl.grid), dim3(pl.block), 0, s, p);
+    case 7: return launch_pdl(q8_0_gemv_kernel<7>, dim3(pl.grid), dim3(pl.block), 0, s, p);
+    case 8: return launch_pdl(q8_0_gemv_kernel<8>, dim3(pl.grid), dim3(pl.block), 0, s, p);
     default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
 
 }  // namespace dq
