@@ -66,10 +66,11 @@ struct Q4KWorkspace {
 Q4KWorkspace q4k_ws(const dq::Q4KPlan &pl, long long N, int B, int NS, bool argmax)
 {
     Q4KWorkspace ws{};
-    if (pl.splits > 1)
+    const bool reduce_kernel = pl.splits > 1 && !pl.cluster;
+    if (reduce_kernel)
         ws.part_bytes = round_up(static_cast<size_t>(pl.splits) * NS * B * N * sizeof(float), 256);
     if (argmax) {
-        ws.ncand = (pl.splits > 1) ? dq::reduce_grid(N, B) : pl.grid;
+        ws.ncand = reduce_kernel ? dq::reduce_grid(N, B) : pl.grid;
         ws.cand_bytes = round_up(static_cast<size_t>(ws.ncand) * sizeof(dq::ArgmaxCand), 256);
     }
     return ws;
@@ -117,7 +118,7 @@ dq_status q4k_common(const void *w0, const void *w1, int layout, const float *x,
     p.w[1] = static_cast<const uint8_t *>(NS == 2 ? w1 : w0);
     p.x = x;
     p.y = y;
-    p.part = pl.splits > 1 ? reinterpret_cast<float *>(wsb) : nullptr;
+    p.part = (pl.splits > 1 && !pl.cluster) ? reinterpret_cast<float *>(wsb) : nullptr;
     p.cand = argmax_out ? reinterpret_cast<dq::ArgmaxCand *>(wsb + ws.part_bytes) : nullptr;
     p.err = dq::device_error_flag(di.device);
     p.N = N;
@@ -130,11 +131,12 @@ dq_status q4k_common(const void *w0, const void *w1, int layout, const float *x,
     p.soa = layout == DQ_LAYOUT_SOA;
     p.argmax = argmax_out != nullptr;
     p.tiles = pl.tiles;
+    p.cluster = pl.cluster ? 1 : 0;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = dq::q4k_gemv_launch(p, pl, B, NS, s);
     if (e != cudaSuccess)
         return cuda_fail(e);
-    if (pl.splits > 1) {
+    if (pl.splits > 1 && !pl.cluster) {
         e = dq::splitk_reduce_launch(p.part, pl.splits, NS, B, N, y, p.cand, dq::reduce_grid(N, B), s);
         if (e != cudaSuccess)
             return cuda_fail(e);

@@ -28,6 +28,7 @@ struct Q4KParams {
     int soa;
     int argmax;
     long long tiles;       // row tiles
+    int cluster;           // fx kernel: split partials are added inside each cluster of `splits` CTAs
 };
 
 struct Q4KPlan {
@@ -35,6 +36,7 @@ struct Q4KPlan {
     bool half;             // batch-1 half-block kernel (q4k_gemv_b1_kernel)
     bool fx;               // batch-1 fixed-point-activation kernel (q4k_gemv_fx_kernel)
     bool tma;              // fx kernel: slots moved by TMA tile copies
+    bool cluster;          // fx kernel: K splits reduced in-kernel across a CTA cluster (no workspace)
     int lpr;               // lanes per row group (4, 8, 16 or 32)
     int R;                 // rows per lane
     int warps;             // warps per CTA

@@ -50,6 +50,7 @@
 // its end), so the box itself lays the rows out at the padded pitch.  Without
 // the driver's tensor-map encoder each row is its own 1-D bulk copy instead.
 
+#include <cooperative_groups.h>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_fp16.h>
@@ -79,6 +80,9 @@ constexpr int kFxRowPitch = kFxChunkBytes + 16;           // 592
 constexpr int kFxSlotBytes = kFxTileRows * kFxRowPitch;
 static_assert(kFxSlotBytes % 128 == 0, "slots must keep the ring 128-byte aligned");
 constexpr int kFxMaxWarps = 12;
+// In-cluster split reduction: per warp and stream, the 16 row partials (fp64).
+constexpr int kFxClusterPartBytes = 2 * kFxTileRows * 8;
+constexpr int kFxMaxCluster = 8;
 
 // TMA descriptors of the (up to two) weight streams.
 struct FxMaps {
@@ -226,8 +230,10 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
     const int g = lane >> 3;   // super-block of each chunk
     const int i = lane & 7;    // rows i and i + 8 of each tile
 
-    const int split = blockIdx.x / p.ctas_per_split;
-    const int cj = blockIdx.x % p.ctas_per_split;
+    // the splits of one CTA column are consecutive blocks (one cluster when the
+    // splits are reduced in-kernel)
+    const int split = blockIdx.x % p.splits;
+    const int cj = blockIdx.x / p.splits;
     const int nchunk_total = (p.nb + kFxBPC - 1) / kFxBPC;
     const int c_begin = split * p.chunks_per_split;
     const int c_end = min(c_begin + p.chunks_per_split, nchunk_total);
@@ -248,6 +254,7 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
     const uint32_t my_ring_s = smem_u32(my_ring);
     const uint32_t my_bars_s = smem_u32(bars + warp * p.depth);
     ArgmaxCand *red = reinterpret_cast<ArgmaxCand *>(ring + static_cast<size_t>(nwarps) * p.depth * kFxSlotBytes);
+    double *cpart = reinterpret_cast<double *>(reinterpret_cast<uint8_t *>(red) + 256);
 
     // this warp's tiles: t0, t0 + tstride, ... (warp-major order)
     const long long tstride = static_cast<long long>(p.ctas_per_split) * nwarps;
@@ -425,6 +432,14 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
             }
         }
         const long long n = row0 + wrow;
+        if (p.cluster) {
+            // this warp's only tile: keep its partials for the cluster reduction
+            if (writer) {
+                cpart[(warp * 2 + 0) * kFxTileRows + wrow] = (NS == 2) ? gsum : t;
+                cpart[(warp * 2 + 1) * kFxTileRows + wrow] = t;
+            }
+            continue;
+        }
         if (!writer || n >= p.N)
             continue;
         if (p.splits > 1) {
@@ -461,7 +476,40 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
         }
     }
 
-    if (p.argmax && p.splits == 1) {
+    if (p.cluster) {
+        // Splits of a CTA column are one cluster and their warps hold the same
+        // tiles: each tile is finished by the CTA whose rank is the warp index
+        // modulo the split count, adding the partials of ranks 0, 1, ... in order.
+        namespace cg = cooperative_groups;
+        cg::cluster_group cl = cg::this_cluster();
+        cl.sync();
+        if (warp % p.splits == split && t0 < p.tiles && lane < kFxTileRows) {
+            double g = 0.0, u = 0.0;
+            for (int r = 0; r < p.splits; ++r) {
+                const double *rp = cl.map_shared_rank(cpart, r);
+                g += rp[(warp * 2 + 0) * kFxTileRows + lane];
+                u += rp[(warp * 2 + 1) * kFxTileRows + lane];
+            }
+            const long long n = t0 * kFxTileRows + lane;
+            if (n < p.N) {
+                float out;
+                if constexpr (NS == 2) {
+                    const float gv = static_cast<float>(g);
+                    out = gv / (1.0f + expf(-gv)) * static_cast<float>(u);
+                } else {
+                    out = static_cast<float>(g);
+                }
+                p.y[n] = out;
+                if (p.argmax && cand_better(out, n, best_v, best_i)) {
+                    best_v = out;
+                    best_i = n;
+                }
+            }
+        }
+        cl.sync();  // no CTA leaves while another reads its shared memory
+    }
+
+    if (p.argmax && (p.splits == 1 || p.cluster)) {
         // CTA-wide (max, lowest index) candidate
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) {
@@ -555,6 +603,12 @@ Q4KPlan q4k_plan_fx(long long N, int nb, int NS, int sm_count, int smem_optin)
         pl.ctas_per_split = static_cast<int>(ctas);
         pl.grid = pl.ctas_per_split * splits;
         pl.smem = x_bytes + ((warps * depth * 8 + 127) & ~127) + 128 + warps * depth * kFxSlotBytes + 256;
+        // splits of at most one tile per warp are added inside a cluster
+        pl.cluster = splits > 1 && splits <= kFxMaxCluster &&
+                     tiles <= static_cast<long long>(pl.ctas_per_split) * warps &&
+                     pl.smem + warps * kFxClusterPartBytes <= smem_optin;
+        if (pl.cluster)
+            pl.smem += warps * kFxClusterPartBytes;
         pl.ok = pl.smem <= smem_optin;
     }
     return pl;
@@ -582,7 +636,23 @@ static cudaError_t launch_fx(const Q4KParams &p, const FxMaps &maps, const Q4KPl
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
     if (e != cudaSuccess)
         return e;
-    return launch_pdl(k, dim3(pl.grid), dim3(pl.warps * 32), pl.smem, s, p, maps);
+    if (!pl.cluster)
+        return launch_pdl(k, dim3(pl.grid), dim3(pl.warps * 32), pl.smem, s, p, maps);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(pl.grid);
+    cfg.blockDim = dim3(pl.warps * 32);
+    cfg.dynamicSmemBytes = pl.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = pl.splits;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, k, p, maps);
 }
 
 cudaError_t q4k_gemv_fx_launch(const Q4KParams &p, const Q4KPlan &pl, int NS, cudaStream_t s)
