@@ -10,9 +10,9 @@
 // is what bounds the kernel.  Forming each fp32 weight (an AND to isolate the
 // quant, an fma with scale and min) and then an fma with x costs three
 // instructions per weight on two half-rate pipes.  Here four quants at a time
-// are unpacked into bytes (one AND for the four low nibbles of a word, a shift
-// and an AND for the four high nibbles) and multiplied against four bytes of x
-// by one dp4a (four 8-bit products summed into an int32).
+// are unpacked into bytes (one AND for the four low nibbles of a word, one AND
+// for the four high nibbles, left in place as 16 q) and multiplied against four
+// bytes of x by one dp4a (four 8-bit products summed into an int32).
 //
 // Arithmetic.
 //   x, per super-block sb of 256 activations: with e the exponent of the
@@ -21,7 +21,8 @@
 //   signed bytes (signed digits) xi = l0 + 2^8 l1 + 2^16 l2 + 2^24 l3.  X_j is
 //   the exact sum of xi over sub-block j.
 //   Per row and sub-block j: A_l = sum_k q_k l_{l,k} (dp4a, exact), folded as
-//   I_l += scale_j * A_l (exact, |I_l| < 2^25).  Per row and super-block, in
+//   I_l += scale_j * A_l (exact, |I_l| < 2^25; kept as 16 I_l < 2^29 because
+//   the high nibbles enter dp4a as 16 q).  Per row and super-block, in
 //   fp64: I_s = sum_l 2^(8l) I_l (exact, < 2^49), I_m = sum_j min_j X_j (exact,
 //   < 2^44) and y_sb = 2^-F (d I_s - dmin I_m), evaluated with an error-free
 //   product so that the rounding is relative to y_sb itself, even when the
@@ -146,8 +147,18 @@ __device__ __forceinline__ void fx_stage(const float *x, int kb_begin, int nbs, 
     }
 }
 
+// dp4a with unsigned bytes in a (quants) and signed bytes in b (activation limbs).
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c)
+{
+    int d;
+    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
 // One 16-byte quant slice of R rows against the limb planes: lo (low nibbles,
-// sub-block 2c) and hi (high nibbles, sub-block 2c+1) sums per limb.
+// sub-block 2c) and hi (high nibbles, sub-block 2c+1) sums per limb.  The high
+// nibbles are used in place, as the bytes 16*q (one AND), so the hi sums are
+// 16 times the sub-block sums.
 template <int R>
 __device__ __forceinline__ void fx_slice(const uint4 (&q)[R], const uint8_t *xlo, const uint8_t *xhi, int (&alo)[R][4],
                                          int (&ahi)[R][4])
@@ -163,19 +174,18 @@ __device__ __forceinline__ void fx_slice(const uint4 (&q)[R], const uint8_t *xlo
 #pragma unroll
         for (int r = 0; r < R; ++r) {
             const uint32_t w = (t == 0) ? q[r].x : (t == 1) ? q[r].y : (t == 2) ? q[r].z : q[r].w;
-            const int lo = static_cast<int>(w & 0x0F0F0F0Fu);
-            const int hi = static_cast<int>((w >> 4) & 0x0F0F0F0Fu);
+            const uint32_t lo = w & 0x0F0F0F0Fu;
+            const uint32_t hi16 = w & 0xF0F0F0F0u;
 #pragma unroll
             for (int l = 0; l < 4; ++l) {
                 const uint32_t x0 = (t == 0) ? xa[l].x : (t == 1) ? xa[l].y : (t == 2) ? xa[l].z : xa[l].w;
                 const uint32_t x1 = (t == 0) ? xb[l].x : (t == 1) ? xb[l].y : (t == 2) ? xb[l].z : xb[l].w;
-                alo[r][l] = __dp4a(lo, static_cast<int>(x0), alo[r][l]);
-                ahi[r][l] = __dp4a(hi, static_cast<int>(x1), ahi[r][l]);
+                alo[r][l] = dp4a_us(lo, x0, alo[r][l]);
+                ahi[r][l] = dp4a_us(hi16, x1, ahi[r][l]);
             }
         }
     }
 }
-
 
 // Issues the copies of one slot (K-chunk c_begin + cur.kcl of stream cur.st of
 // the tile at cur.row0).  TMA: lane 0 arms the slot's mbarrier and issues one
@@ -350,15 +360,16 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
                                                                 s * bo.qs_step);
                     fx_slice<R>(q, xb + 64 * c + 16 * h, xb + 64 * c + 32 + 16 * h, alo, ahi);
                 }
-                // fold the scales of sub-blocks 2c (lo) and 2c+1 (hi)
+                // fold the scales of sub-blocks 2c (lo) and 2c+1 (hi); the sums are
+                // kept 16 times larger (the hi sums already are): |16 I_l| < 2^29
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
                     const uint32_t sw = (c < 2) ? sc03[r] : sc47[r];
-                    const int slo = static_cast<int>((sw >> (16 * (c & 1))) & 0xFFu);
+                    const int slo16 = static_cast<int>((sw >> (16 * (c & 1))) & 0xFFu) << 4;
                     const int shi = static_cast<int>((sw >> (16 * (c & 1) + 8)) & 0xFFu);
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
-                        isum[r][k] += slo * alo[r][k] + shi * ahi[r][k];
+                        isum[r][k] += slo16 * alo[r][k] + shi * ahi[r][k];
                 }
             }
 
@@ -388,9 +399,10 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
                     pmn[j] = static_cast<double>((mw >> (8 * (j & 3))) & 0xFFu) * X[j];
                 }
                 const double im = ((pmn[0] + pmn[1]) + (pmn[2] + pmn[3])) + ((pmn[4] + pmn[5]) + (pmn[6] + pmn[7]));
+                // the 1/16 undoes the scaling of the integer sums (exact)
                 const double d =
                     static_cast<double>(__half2float(__ushort_as_half(static_cast<unsigned short>(hd[r].x & 0xFFFFu)))) *
-                    s2f;
+                    (s2f * 0.0625);
                 const double dm =
                     static_cast<double>(__half2float(__ushort_as_half(static_cast<unsigned short>(hd[r].x >> 16)))) *
                     s2f;
