@@ -56,6 +56,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_fp16.h>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -576,7 +577,10 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 Q4KPlan q4k_plan_fx(long long N, int nb, int NS, int sm_count, int smem_optin)
 {
     Q4KPlan pl{};
-    const bool tma = N < 0x7FFFFFFFLL && tensor_map_encoder() != nullptr;
+    // DQGEMV_NO_TMA=1 selects the per-row bulk copies (same shared-memory
+    // layout, bit-identical results), for comparing the two copy paths
+    const char *no_tma = getenv("DQGEMV_NO_TMA");
+    const bool tma = N < 0x7FFFFFFFLL && tensor_map_encoder() != nullptr && !(no_tma && no_tma[0] == '1');
     const int misc = 256 /*argmax scratch, 16 B per warp*/ + 512 /*barriers*/ + 128 /*ring alignment*/;
     const int stage = kFxLimbPitch + kFxAuxPitch;
     const long long tiles = (N + kFxTileRows - 1) / kFxTileRows;

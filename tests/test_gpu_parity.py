@@ -345,3 +345,92 @@ def test_q4k_gemv_long_matrices_full_block_lanes(N, K, layout):
     rows = np.unique(np.concatenate([np.arange(0, N, 7), [N - 1]]))
     y_ref, a_ref = oracle_rows(lambda rows: oracle.q4k_gemv(w, N, K, x, rows=rows), N, rows)
     assert_within(y[:, rows], y_ref, a_ref, "N=%d K=%d %s" % (N, K, layout))
+
+
+# --- the batch-1 fixed-point path: its own error bound, special values, copy paths ------
+
+def _fx_bound(wd, x):
+    """The batch-1 kernel's stated bound: sum over super-blocks of 2^(e_sb - 30) * sum |w|,
+    e_sb the exponent of the super-block's largest |x| (2^e <= max < 2^(e+1))."""
+    N, K = wd.shape
+    xb = np.abs(x.astype(np.float64)).reshape(K // 256, 256)
+    mx = xb.max(axis=1)
+    _, E = np.frexp(mx)
+    unit = np.where(mx > 0, np.ldexp(1.0, E - 1 - 30), 0.0)           # 2^(e - 30)
+    wsum = np.abs(wd.astype(np.float64)).reshape(N, K // 256, 256).sum(axis=2)
+    return wsum @ unit
+
+
+def test_fixed_point_activations_within_their_stated_bound():
+    # wide dynamic range inside super-blocks: outliers, tiny values, a zero block,
+    # subnormals; the result must stay within 2^-30 of each block's largest |x|
+    N, K = 640, 4096
+    rng = np.random.default_rng(31)
+    w = synth.q4k_matrix(rng, N, K)
+    x = synth.activations(rng, 1, K)[0].astype(np.float32)
+    x[7] = 3.0e4
+    x[300] = -1.0e4
+    x[1000:1010] = 1e-7
+    x[2 * 256:3 * 256] = 0.0
+    x[5 * 256:6 * 256] *= np.float32(1e-40)          # subnormal activations
+    y = host(dq.q4k_gemv(dev(w), dev(x[None, :]), N, K))[0].astype(np.float64)
+    y_ref, a_ref = oracle.q4k_gemv(w, N, K, x[None, :])
+    y_ref = y_ref[0]
+    wd = oracle.q4k_dequant(w, N, K)
+    bound = _fx_bound(wd, x) + 2.0 ** -24 * np.abs(y_ref) + 1e-30
+    err = np.abs(y - y_ref)
+    assert np.all(np.isfinite(y))
+    assert np.all(err <= bound), "worst err/bound %.3g" % (err / bound).max()
+    assert_within(y[None, :], y_ref[None, :], a_ref, "wide-range x")
+
+
+@pytest.mark.parametrize("scale", [1e-30, 1e30, 1e34])
+def test_extreme_activation_scales(scale):
+    # the per-super-block exponent covers the fp32 range: results scale with x
+    N, K = 256, 2048
+    rng = np.random.default_rng(34)
+    w = synth.q4k_matrix(rng, N, K)
+    x = (synth.activations(rng, 1, K) * np.float32(scale)).astype(np.float32)
+    y = host(dq.q4k_gemv(dev(w), dev(x), N, K))
+    y_ref, a_ref = oracle.q4k_gemv(w, N, K, x)
+    tol = 1e-4 * a_ref + 1e-6 * scale                 # the absolute term scales with x here
+    assert np.all(np.isfinite(y))
+    assert np.all(np.abs(y.astype(np.float64) - y_ref) <= tol)
+
+
+@pytest.mark.parametrize("bad", [np.inf, -np.inf, np.nan])
+def test_non_finite_activations_give_nan_rows(bad):
+    N, K = 64, 1024
+    rng = np.random.default_rng(32)
+    w = synth.q4k_matrix(rng, N, K)
+    x = synth.activations(rng, 1, K)
+    x[0, 300] = bad
+    y = host(dq.q4k_gemv(dev(w), dev(x), N, K))
+    assert np.all(np.isnan(y))
+
+
+def test_per_row_copy_path_is_bitwise_equal_to_tma():
+    # DQGEMV_NO_TMA=1 moves the same slots with one bulk copy per row
+    import subprocess
+    import sys
+    N, K = 1000, 5120
+    rng = np.random.default_rng(33)
+    w = synth.q4k_matrix(rng, N, K)
+    x = synth.activations(rng, 1, K)
+    y_tma = host(dq.q4k_gemv(dev(w), dev(x), N, K))
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = (
+        "import sys, numpy as np, torch\n"
+        "sys.path.insert(0, %r)\n"
+        "import dequant_gemv_q4_b200 as dq\n"
+        "from dequant_gemv_q4_b200 import synth\n"
+        "rng = np.random.default_rng(33)\n"
+        "w = synth.q4k_matrix(rng, %d, %d); x = synth.activations(rng, 1, %d)\n"
+        "y = dq.q4k_gemv(torch.from_numpy(w).cuda(), torch.from_numpy(x).cuda(), %d, %d)\n"
+        "torch.cuda.synchronize(); sys.stdout.buffer.write(y.cpu().numpy().tobytes())\n"
+    ) % (root, N, K, K, N, K)
+    env = dict(os.environ, DQGEMV_NO_TMA="1")
+    out = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, timeout=300)
+    assert out.returncode == 0, out.stderr.decode()[-2000:]
+    y_rows = np.frombuffer(out.stdout, dtype=np.float32).reshape(1, N)
+    assert np.array_equal(y_rows.view(np.uint32), y_tma.view(np.uint32))
