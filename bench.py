@@ -3,16 +3,17 @@
 
 One step = one q4k_gemv call (+ argmax epilogue) over the Q4_K LM-head
 workload (N = 248320 vocab rows x K = 4096, batch 1, ~572 MB of blocks; seed
-4; x ~ N(0,1)/64): block streaming, header decode, scale/min and quant unpack,
-dequant-MAC, reduction, logits + argmax.  The matrix is larger than the 126 MB
-L2, so no flush is needed between steps.
+4; x ~ N(0,1)/64): activation staging (per-super-block fixed point), block
+streaming, header decode, quant unpack, integer dot products, scale/min
+combine in fp64, reduction, logits + argmax.  The matrix is larger than the
+126 MB L2, so no flush is needed between steps.
 
 Metric: effective HBM GB/s = (weight bytes + activation bytes) / time.
   value  - device time of K steps (CUDA events, inputs resident in HBM), max over ranks
   e2e    - the same metric through the same C-ABI call, with each step's x copied
            host->device from pinned memory and its logits + argmax copied back
            (weights stay resident, as a decode loop keeps them)
-  roofline - dominant kernel (q4k_gemv_kernel) timed alone with CUDA events on its
+  roofline - dominant kernel (q4k_gemv_fx_kernel) timed alone with CUDA events on its
            stream, against the measured HBM copy bandwidth in MEASURED_PEAKS.json
   cpu_baseline - the CPU oracle timed on this host (rank 0, N = 1)
 
@@ -46,15 +47,15 @@ UNIT = "GB/s"
 WORKLOAD = "q4k_lmhead_248320x4096"
 FALLBACK_HBM_GBS = 6650.0
 
-# DRAM bytes (read + write) per launch of q4k_gemv_kernel on this workload, from
-# one ncu capture, valid only for the kernel sources whose hash is recorded.
-NCU_TRAFFIC = {"sources_sha1": "ca1e4f2d7a3c06439108472ac3a72795845a4c09",
-               "bytes_per_launch": 572.21e6 + 4.20e6}   # profiles/q4k_gemv_kernel_248320x4096_dram.md
+# DRAM bytes (read + write) per launch of q4k_gemv_fx_kernel on this workload,
+# from one ncu capture, valid only for the kernel sources whose hash is recorded.
+NCU_TRAFFIC = {"sources_sha1": "d2937bcf73647018c79c1b6fabef0f0a4d3ddd0b",
+               "bytes_per_launch": 572196608 + 4256768}   # profiles/q4k_gemv_fx_kernel_248320x4096_dram.md
 
 
 def kernel_sources_sha1() -> str:
     h = hashlib.sha1()
-    for f in ("q4k_gemv.cu", "q4k_decode.cuh", "dq_common.cuh"):
+    for f in ("q4k_gemv_fx.cu", "q4k_stream.cuh", "dq_common.cuh"):
         with open(os.path.join(ROOT, "dequant_gemv_q4_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
@@ -384,7 +385,7 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "vs_baseline": None, "dtype": "s8xu8->s32 dp4a, f64 combine", "data": "synthetic",
         "config": {"workload": wl.name, "N": wl.N, "K": wl.K, "B": B,
                    "format": "Q4_K" if wl.fmt == "q4k" else "Q8_0", "layout": "aos",
                    "epilogue": "argmax" if argmax else ("swiglu" if wl.op == "swiglu" else "none"),
@@ -394,7 +395,7 @@ def main():
                    "parallelism": "replicas x%d (independent problems, no collective)" % world},
         "pct_of_peak_hbm": 100.0 * value / world / peak,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
-                     "traffic": traffic, "kernel": "q4k_gemv_kernel", "kernel_ms": kms,
+                     "traffic": traffic, "kernel": "q4k_gemv_fx_kernel", "kernel_ms": kms,
                      "peak_kind": peak_kind + " (MEASURED_PEAKS.json hbm_gbs, burst)" if peak_kind == "measured"
                      else "fallback"},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
