@@ -20,11 +20,23 @@
  *   A row is K/32 (Q8_0) or K/256 (Q4_K) consecutive blocks; rows follow each
  *   other without padding, so W occupies N*K*34/32 or N*K*144/256 bytes.
  *
- * Numerics.  Every weight is formed exactly as the fp32 value nearest to its
- * exact dequantized value (the same bits the *_dequant entry points return)
- * and the products are accumulated in fp32.  Results satisfy
+ * Numerics.  Results satisfy
  *     |y - y_exact| <= 1e-4 * sum_k |W[n][k] * x[k]| + 1e-6
- * for finite inputs.
+ * (y_exact: the exact sum over the exact dequantized weights) for finite
+ * inputs, up to fp32 overflow of the result.
+ *   - Q8_0 and Q4_K with B >= 2: every weight is formed exactly as the fp32
+ *     value nearest to its dequantized value (the bits the *_dequant entry
+ *     points return) and the products are accumulated in fp32.
+ *   - Q4_K with B == 1 (q4k_gemv, q4k_swiglu_gemv): each activation is rounded
+ *     to a 30-bit fixed point shared by its super-block of 256 activations;
+ *     the dot products over the exact quants, scales and mins are then exact
+ *     (integers, fp64), rounded once to fp32.  The error is at most
+ *     sum over super-blocks of 2^(e - 30) * sum |W[n][k]| over the block, where
+ *     2^e <= (largest |x| of the block) < 2^(e+1).  An infinity or NaN in x
+ *     makes every result that reads it NaN.
+ *   - Environment: DQGEMV_NO_TMA=1 makes the batch-1 kernel fill its shared
+ *     memory with per-row bulk copies instead of TMA tile copies (bitwise
+ *     identical results; a debugging aid).
  *
  * Conventions shared by every entry point:
  *   - All data pointers are DEVICE pointers owned by the caller (for example
