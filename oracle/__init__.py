@@ -69,10 +69,11 @@ def _load():
             lib.oracle_swiglu.argtypes = [p, p, i64, p]
             lib.oracle_swiglu.restype = None
             lib.oracle_argmax.argtypes = [p, i64]
+            lib.oracle_split_qg.argtypes = [p, i64, i64, i64, p, p]
             lib.oracle_argmax.restype = i64
             for name in ("oracle_q4k_repack_soa", "oracle_q8_0_dequant", "oracle_q4k_dequant",
                          "oracle_q4k_dequant_f32", "oracle_q8_0_dequant_f32",
-                         "oracle_q4k_gemv_rows", "oracle_q8_0_gemv_rows"):
+                         "oracle_q4k_gemv_rows", "oracle_q8_0_gemv_rows", "oracle_split_qg"):
                 getattr(lib, name).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -232,6 +233,19 @@ def swiglu(g, u) -> np.ndarray:
 def argmax(v) -> int:
     v = np.ascontiguousarray(np.asarray(v, dtype=np.float64).reshape(-1))
     return int(_load().oracle_argmax(_ptr(v), v.size))
+
+
+def split_qg(y, head_dim: int):
+    """De-interleave a q-projection-with-gate output (B x N, per head head_dim Q
+    values then head_dim gate values) into contiguous Q and G (B x N/2 each);
+    Doppler 0.1.8, split_qg.wgsl."""
+    y = np.ascontiguousarray(np.asarray(y, dtype=np.float64))
+    y2 = y.reshape(-1, y.shape[-1])
+    B, N = y2.shape
+    q = np.empty((B, N // 2), np.float64)
+    g = np.empty((B, N // 2), np.float64)
+    _check(_load().oracle_split_qg(_ptr(y2), B, N, head_dim, _ptr(q), _ptr(g)), "split_qg")
+    return q, g
 
 
 # --- tolerance rules ----------------------------------------------------------

@@ -345,6 +345,25 @@ void oracle_swiglu(const double *g, const double *u, int64_t n, double *out)
         out[i] = g[i] / (1.0 + exp(-g[i])) * u[i];
 }
 
+/* De-interleave of a q-projection-with-gate output (Doppler 0.1.8,
+ * split_qg.wgsl).  Each of the B rows of y holds, per head h, head_dim Q values
+ * followed by head_dim gate values; Q and G receive them contiguously:
+ *   q[b][h*hd + d] = y[b][h*2*hd + d],  g[b][h*hd + d] = y[b][h*2*hd + hd + d].
+ * N (the row length of y) must be a positive multiple of 2*hd. */
+int oracle_split_qg(const double *y, int64_t B, int64_t N, int64_t hd, double *q, double *g)
+{
+    if (B < 0 || N <= 0 || hd <= 0 || N % (2 * hd) != 0)
+        return -1;
+    int64_t qsize = N / 2;
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t h = 0; h < N / (2 * hd); ++h)
+            for (int64_t d = 0; d < hd; ++d) {
+                q[b * qsize + h * hd + d] = y[b * N + h * 2 * hd + d];
+                g[b * qsize + h * hd + d] = y[b * N + h * 2 * hd + hd + d];
+            }
+    return 0;
+}
+
 /* Index of the largest value; among equal largest values the lowest index. */
 int64_t oracle_argmax(const double *v, int64_t n)
 {

@@ -325,3 +325,33 @@ def test_soa_positions_hand_derived():
     # group 1 starts at byte 4*144 = 576: 2 headers (32 B), slice s of block t at 32 + 32*s + 16*t
     assert soa[0, 576 + 32 + 32 * 7 + 16 * 1 + 15] == 33
     assert int(np.count_nonzero(soa)) == 3
+
+
+# --- Q/gate de-interleave (Doppler split_qg.wgsl) -------------------------------------
+
+def test_split_qg_hand_derived():
+    # two heads of head_dim 2: row = [Q0 Q0 G0 G0 Q1 Q1 G1 G1]
+    y = np.array([[10, 11, 20, 21, 12, 13, 22, 23]], np.float64)
+    q, g = oracle.split_qg(y, 2)
+    assert q.tolist() == [[10, 11, 12, 13]]
+    assert g.tolist() == [[20, 21, 22, 23]]
+    # head_dim = N/2: one head, Q is the first half, G the second
+    q1, g1 = oracle.split_qg(y, 4)
+    assert q1.tolist() == [[10, 11, 20, 21]] and g1.tolist() == [[12, 13, 22, 23]]
+
+
+def test_split_qg_is_a_per_row_permutation_inverted_by_interleaving():
+    rng = np.random.default_rng(5)
+    B, heads, hd = 3, 5, 8
+    y = rng.standard_normal((B, 2 * heads * hd))
+    q, g = oracle.split_qg(y, hd)
+    # re-interleave by a different route: stack per head and flatten
+    back = np.stack([q.reshape(B, heads, hd), g.reshape(B, heads, hd)], axis=2).reshape(B, -1)
+    assert np.array_equal(back, y)
+    for b in range(B):
+        assert np.array_equal(np.sort(np.concatenate([q[b], g[b]])), np.sort(y[b]))
+
+
+def test_split_qg_rejects_rows_that_are_not_whole_heads():
+    with pytest.raises(Exception):
+        oracle.split_qg(np.zeros((1, 12)), 4)
