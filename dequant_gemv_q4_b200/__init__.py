@@ -31,7 +31,7 @@ Q8_0_BLOCK_ELEMS, Q8_0_BLOCK_BYTES = 32, 34
 
 EXPORTED = ("q8_0_gemv", "q4k_gemv", "q4k_swiglu_gemv", "q4k_repack_soa", "dq_workspace_bytes",
             "q8_0_dequant", "q4k_dequant", "dq_status_string", "dq_last_cuda_error",
-            "dq_device_error", "q4k_gemv_noalloc", "dq_noalloc_scratch_bytes")
+            "dq_device_error", "q4k_gemv_noalloc", "dq_noalloc_scratch_bytes", "q4k_gemv_split_qg")
 
 
 class DQError(RuntimeError):
@@ -71,6 +71,7 @@ def load_library(path: str = LIB_PATH):
             "q4k_dequant": [p, i32, p, i64, i64, p],
             "dq_device_error": [p, i32, p],
             "q4k_gemv_noalloc": [p, i32, p, p, i64, i64, i32, p, p],
+            "q4k_gemv_split_qg": [p, i32, p, p, p, i64, i64, i32, i64, p, sz, p],
         }
         for name, args in sigs.items():
             f = getattr(lib, name)
@@ -232,6 +233,35 @@ def q4k_gemv_noalloc(w, x, N: int, K: int, layout="aos", y=None, argmax: bool = 
 
 def dq_noalloc_scratch_bytes() -> int:
     return int(load_library().dq_noalloc_scratch_bytes())
+
+
+def q4k_gemv_split_qg(w, x, N: int, K: int, head_dim: int, layout="aos", q=None, g=None, workspace=None,
+                      stream=None):
+    """y = W x for a q-projection-with-gate matrix, stored de-interleaved:
+    per head, head_dim Q rows then head_dim gate rows of y go to Q and G
+    (each (B, N/2), or (N/2,) for 1-D x).  Returns (Q, G)."""
+    torch = _torch()
+    lib = load_library()
+    one_d = x.dim() == 1
+    x2 = _x2d(x, K)
+    B = x2.shape[0]
+    wp = _weights(w, "w", N, K, Q4K_BLOCK_ELEMS, Q4K_BLOCK_BYTES)
+    half = N // 2
+    if q is None:
+        q = torch.empty((B, half), dtype=torch.float32, device=x.device)
+    if g is None:
+        g = torch.empty((B, half), dtype=torch.float32, device=x.device)
+    qp = _dev(q, "q", torch.float32)
+    gp = _dev(g, "g", torch.float32)
+    if q.numel() != B * half or g.numel() != B * half:
+        raise ValueError("q and g must hold B*N/2 floats each")
+    need = dq_workspace_bytes(DQ_OP_Q4K_GEMV, N, K, B)
+    wsp, wsn, _keep = _workspace(workspace, need, x.device)
+    _check("q4k_gemv_split_qg", lib.q4k_gemv_split_qg(wp, _layout(layout), ctypes.c_void_p(x2.data_ptr()), qp, gp,
+                                                      N, K, B, head_dim, wsp, wsn, _stream(stream)))
+    if one_d:
+        return q.view(half), g.view(half)
+    return q.view(B, half), g.view(B, half)
 
 
 def q4k_swiglu_gemv(w_gate, w_up, x, N: int, K: int, layout="aos", out=None, workspace=None,

@@ -84,7 +84,8 @@ dq_status check_q4k_shape(int64_t N, int64_t K, int B)
 }
 
 dq_status q4k_common(const void *w0, const void *w1, int layout, const float *x, float *y, int64_t N, int64_t K,
-                     int B, int NS, int64_t *argmax_out, void *workspace, size_t ws_bytes, void *stream)
+                     int B, int NS, int64_t *argmax_out, void *workspace, size_t ws_bytes, void *stream,
+                     float *g_out = nullptr, int64_t qg_hd = 0)
 {
     if (!w0 || (NS == 2 && !w1) || !x || !y)
         return DQ_ERR_NULL;
@@ -118,6 +119,8 @@ dq_status q4k_common(const void *w0, const void *w1, int layout, const float *x,
     p.w[1] = static_cast<const uint8_t *>(NS == 2 ? w1 : w0);
     p.x = x;
     p.y = y;
+    p.g = g_out;
+    p.qg_hd = static_cast<int>(qg_hd);
     p.part = (pl.splits > 1 && !pl.cluster) ? reinterpret_cast<float *>(wsb) : nullptr;
     p.cand = argmax_out ? reinterpret_cast<dq::ArgmaxCand *>(wsb + ws.part_bytes) : nullptr;
     p.err = dq::device_error_flag(di.device);
@@ -137,7 +140,7 @@ dq_status q4k_common(const void *w0, const void *w1, int layout, const float *x,
     if (e != cudaSuccess)
         return cuda_fail(e);
     if (pl.splits > 1 && !pl.cluster) {
-        e = dq::splitk_reduce_launch(p.part, pl.splits, NS, B, N, y, p.cand, dq::reduce_grid(N, B), s);
+        e = dq::splitk_reduce_launch(p.part, pl.splits, NS, B, N, y, p.g, p.qg_hd, p.cand, dq::reduce_grid(N, B), s);
         if (e != cudaSuccess)
             return cuda_fail(e);
     }
@@ -208,6 +211,23 @@ dq_status q4k_gemv(const void *w, int layout, const float *x, float *y, int64_t 
                    int64_t *argmax_out, void *workspace, size_t ws_bytes, void *stream)
 {
     return q4k_common(w, nullptr, layout, x, y, N, K, B, 1, argmax_out, workspace, ws_bytes, stream);
+}
+
+dq_status q4k_gemv_split_qg(const void *w, int layout, const float *x, float *q, float *g, int64_t N, int64_t K,
+                            int B, int64_t head_dim, void *workspace, size_t ws_bytes, void *stream)
+{
+    if (!q || !g)
+        return DQ_ERR_NULL;
+    if (head_dim < 1 || N < 2 || N % (2 * head_dim) != 0 || head_dim > (1LL << 30))
+        return DQ_ERR_SHAPE;
+    if (!aligned(g, 4))
+        return DQ_ERR_ALIGN;
+    // Q and G must not overlap: each is B x N/2 floats
+    const uintptr_t qa = reinterpret_cast<uintptr_t>(q), ga = reinterpret_cast<uintptr_t>(g);
+    const uintptr_t span = static_cast<uintptr_t>(B > 0 ? B : 0) * static_cast<uintptr_t>(N / 2) * sizeof(float);
+    if (qa < ga + span && ga < qa + span)
+        return DQ_ERR_ARG;
+    return q4k_common(w, nullptr, layout, x, q, N, K, B, 1, nullptr, workspace, ws_bytes, stream, g, head_dim);
 }
 
 dq_status q4k_swiglu_gemv(const void *w_gate, const void *w_up, int layout, const float *x, float *out, int64_t N,

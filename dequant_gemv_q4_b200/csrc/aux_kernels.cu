@@ -189,7 +189,8 @@ int reduce_grid(long long N, int B)
 
 __global__ void __launch_bounds__(kReduceThreads) splitk_reduce_kernel(const float *__restrict__ part, int splits,
                                                                        int NS, int B, long long N,
-                                                                       float *__restrict__ y, ArgmaxCand *cand)
+                                                                       float *__restrict__ y, float *__restrict__ g_out,
+                                                                       int qg_hd, ArgmaxCand *cand)
 {
     pdl_wait();
     pdl_launch_dependents();
@@ -207,7 +208,7 @@ __global__ void __launch_bounds__(kReduceThreads) splitk_reduce_kernel(const flo
                 u += part[((static_cast<long long>(s) * NS + 1) * B + b) * N + n];
         }
         const float out = (NS == 2) ? g / (1.0f + expf(-g)) * u : g;
-        y[i] = out;
+        *gemv_out_addr(y, g_out, qg_hd, N, b, n) = out;
         if (cand && cand_better(out, n, best_v, best_i)) {
             best_v = out;
             best_i = n;
@@ -239,10 +240,11 @@ __global__ void __launch_bounds__(kReduceThreads) splitk_reduce_kernel(const flo
     }
 }
 
-cudaError_t splitk_reduce_launch(const float *part, int splits, int NS, int B, long long N, float *y,
-                                 ArgmaxCand *cand, int grid, cudaStream_t s)
+cudaError_t splitk_reduce_launch(const float *part, int splits, int NS, int B, long long N, float *y, float *g,
+                                 int qg_hd, ArgmaxCand *cand, int grid, cudaStream_t s)
 {
-    return launch_pdl(splitk_reduce_kernel, dim3(grid), dim3(kReduceThreads), 0, s, part, splits, NS, B, N, y, cand);
+    return launch_pdl(splitk_reduce_kernel, dim3(grid), dim3(kReduceThreads), 0, s, part, splits, NS, B, N, y, g,
+                      qg_hd, cand);
 }
 
 // One CTA folds all candidates into the final index.

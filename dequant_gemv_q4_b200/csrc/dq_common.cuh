@@ -19,6 +19,21 @@ constexpr int kQ4KSoaGroup = 4;
 constexpr int kQ8BlockElems = 32;
 constexpr int kQ8BlockBytes = 34;
 
+// Address of GEMV output (b, n) for rows of length N: y[b][n]; or, with the
+// fused Q/gate split (hd > 0; Doppler split_qg.wgsl), the de-interleaved place
+// in Q (= y) or G, each B x N/2: row n = h*2*hd + d goes to Q[b][h*hd + d] when
+// d < hd and to G[b][h*hd + d - hd] otherwise.
+__device__ __forceinline__ float *gemv_out_addr(float *y, float *g, int hd, long long N, int b, long long n)
+{
+    if (hd == 0)
+        return y + static_cast<long long>(b) * N + n;
+    const long long hd2 = 2LL * hd;
+    const long long h = n / hd2;
+    const long long d = n - h * hd2;
+    const long long base = static_cast<long long>(b) * (N / 2) + h * hd;
+    return d < hd ? y + base + d : g + base + (d - hd);
+}
+
 // Error codes written to the device error flag.
 constexpr int kDevErrWaitTimeout = 1;
 

@@ -321,7 +321,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_kernel(const Q4KPa
                 } else {
                     out = v[j] * 0x1p64f;
                 }
-                p.y[static_cast<long long>(b) * p.N + n] = out;
+                *gemv_out_addr(p.y, p.g, p.qg_hd, p.N, b, n) = out;
                 if (p.argmax && cand_better(out, n, best_v, best_i)) {
                     best_v = out;
                     best_i = n;
@@ -593,7 +593,7 @@ __global__ void __launch_bounds__(kB1Warps * 32, 1) q4k_gemv_b1_kernel(const Q4K
             } else {
                 out = v[0] * 0x1p64f;
             }
-            p.y[n] = out;
+            *gemv_out_addr(p.y, p.g, p.qg_hd, p.N, 0, n) = out;
             if (p.argmax && cand_better(out, n, best_v, best_i)) {
                 best_v = out;
                 best_i = n;

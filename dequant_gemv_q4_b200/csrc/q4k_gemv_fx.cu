@@ -470,7 +470,7 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
             } else {
                 out = static_cast<float>(t);
             }
-            p.y[n] = out;
+            *gemv_out_addr(p.y, p.g, p.qg_hd, p.N, 0, n) = out;
             if (p.argmax && cand_better(out, n, best_v, best_i)) {
                 best_v = out;
                 best_i = n;
@@ -512,7 +512,7 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
                 } else {
                     out = static_cast<float>(g);
                 }
-                p.y[n] = out;
+                *gemv_out_addr(p.y, p.g, p.qg_hd, p.N, 0, n) = out;
                 if (p.argmax && cand_better(out, n, best_v, best_i)) {
                     best_v = out;
                     best_i = n;

@@ -115,6 +115,23 @@ dq_status q4k_gemv(const void *w, int layout, const float *x, float *y, int64_t 
                    int B, int64_t *argmax_out, void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * Q4_K GEMV of a q-projection-with-gate matrix with the Q/gate de-interleave
+ * fused into the store (Doppler 0.1.8, split_qg.wgsl: "attentionOutputGate"
+ * models interleave, per head, head_dim Q rows and head_dim gate rows):
+ *   with y = W x (B x N) and h, d such that n = h*2*head_dim + d,
+ *     q[b][h*head_dim + d]            = y[b][n]  for d <  head_dim,
+ *     g[b][h*head_dim + d - head_dim] = y[b][n]  for d >= head_dim.
+ *   q, g      B x N/2 fp32 each, 4-byte aligned, not overlapping (q takes the
+ *             place of y; x as for q4k_gemv).
+ *   N         a positive multiple of 2*head_dim.
+ *   workspace at least dq_workspace_bytes(DQ_OP_Q4K_GEMV, N, K, B, 0) bytes.
+ * The values are exactly those q4k_gemv writes for the same call, stored in
+ * the split order; no argmax.
+ */
+dq_status q4k_gemv_split_qg(const void *w, int layout, const float *x, float *q, float *g, int64_t N, int64_t K,
+                            int B, int64_t head_dim, void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * Fused gate/up SwiGLU GEMV (qualiaDB cuda_lane: try_q4k_soa_fused_swiglu;
  * trueno WgslForwardPass: silu_mul_shader, here fused into the GEMV):
  *   out[b][n] = silu(g) * u,  g = (W_gate x_b)[n],  u = (W_up x_b)[n],

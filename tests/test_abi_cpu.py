@@ -116,3 +116,16 @@ def test_binding_raises_loudly_without_the_library(tmp_path):
             dq.load_library(missing)
     finally:
         dq._lib = saved
+
+
+def test_split_qg_rejects_on_host(lib):
+    f = lib.q4k_gemv_split_qg
+    A16b = P((1 << 20) + (1 << 16))
+    # null outputs, a head that does not divide N, an unaligned G, overlapping Q and G
+    assert f(A16, 0, A16, None, A16b, 512, 256, 1, 64, None, 0, None) == DQ_ERR_NULL
+    assert f(A16, 0, A16, A16, A16b, 512, 256, 1, 96, None, 0, None) == DQ_ERR_SHAPE
+    assert f(A16, 0, A16, A16, A16b, 512, 256, 1, 0, None, 0, None) == DQ_ERR_SHAPE
+    assert f(A16, 0, A16, A16, P((1 << 20) + (1 << 16) + 2), 512, 256, 1, 64, None, 0, None) == DQ_ERR_ALIGN
+    assert f(A16, 0, A16, A16, P((1 << 20) + 512), 512, 256, 1, 64, None, 0, None) == DQ_ERR_ARG
+    # and the shared Q4_K checks still apply (K not a multiple of 256)
+    assert f(A16, 0, A16, A16, A16b, 512, 100, 1, 64, None, 0, None) == DQ_ERR_SHAPE

@@ -434,3 +434,31 @@ def test_per_row_copy_path_is_bitwise_equal_to_tma():
     assert out.returncode == 0, out.stderr.decode()[-2000:]
     y_rows = np.frombuffer(out.stdout, dtype=np.float32).reshape(1, N)
     assert np.array_equal(y_rows.view(np.uint32), y_tma.view(np.uint32))
+
+
+# --- fused Q/gate de-interleave (Doppler split_qg.wgsl) ---------------------------------
+
+@pytest.mark.parametrize("N,K,B,hd,layout", [
+    (4096, 1024, 1, 128, "aos"),     # the q-projection-with-gate workload, 16 heads of 128
+    (4096, 1024, 1, 128, "soa"),
+    (512, 12288, 1, 64, "aos"),      # K splits (reduced in a CTA cluster)
+    (1040, 4096, 3, 8, "aos"),       # batch 3: the fp32 kernel
+    (200, 65536, 2, 50, "aos"),      # many K splits, a second-kernel reduction
+])
+def test_q4k_gemv_split_qg_is_the_plain_gemv_deinterleaved(N, K, B, hd, layout):
+    rng = np.random.default_rng(N + K + B)
+    w = synth.q4k_matrix(rng, N, K)
+    x = synth.activations(rng, B, K)
+    wl = w if layout == "aos" else oracle.q4k_repack_soa(w, N, K)
+    wd, xd = dev(wl), dev(x)
+    y = host(dq.q4k_gemv(wd, xd, N, K, layout=layout))
+    q, g = dq.q4k_gemv_split_qg(wd, xd, N, K, hd, layout=layout)
+    q, g = host(q), host(g)
+    q_ref, g_ref = oracle.split_qg(y.astype(np.float64), hd)
+    # the same arithmetic, only stored in the split order
+    assert np.array_equal(q.astype(np.float64), q_ref) and np.array_equal(g.astype(np.float64), g_ref)
+    # and against the oracle's exact GEMV, split by the oracle
+    y_ref, a_ref = oracle.q4k_gemv(w, N, K, x)
+    tq, tg = oracle.split_qg(oracle.gemv_tolerance(a_ref), hd)
+    yq, yg = oracle.split_qg(y_ref, hd)
+    assert np.all(np.abs(q - yq) <= tq) and np.all(np.abs(g - yg) <= tg)
