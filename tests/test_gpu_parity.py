@@ -462,3 +462,57 @@ def test_q4k_gemv_split_qg_is_the_plain_gemv_deinterleaved(N, K, B, hd, layout):
     tq, tg = oracle.split_qg(oracle.gemv_tolerance(a_ref), hd)
     yq, yg = oracle.split_qg(y_ref, hd)
     assert np.all(np.abs(q - yq) <= tq) and np.all(np.abs(g - yg) <= tg)
+
+
+# --- capture of a decode step's GEMV sequence in a CUDA graph ---------------------------
+
+def test_ffn_and_qproj_sequence_replays_from_a_cuda_graph():
+    # q-projection with the Q/gate split, then the FFN: SwiGLU (gate/up 12288 x 4096)
+    # feeding the down projection (4096 x 12288); captured once, replayed twice
+    rng = np.random.default_rng(41)
+    H, F, NQ, KQ = 4096, 12288, 4096, 1024
+    wq = synth.q4k_matrix(rng, NQ, KQ)
+    wg = synth.q4k_matrix(rng, F, H)
+    wu = synth.q4k_matrix(rng, F, H)
+    wdn = synth.q4k_matrix(rng, H, F)
+    xq = dev(synth.activations(rng, 1, KQ))
+    x = dev(synth.activations(rng, 1, H))
+    dwq, dwg, dwu, dwd = dev(wq), dev(wg), dev(wu), dev(wdn)
+    q = torch.empty((1, NQ // 2), device="cuda")
+    gq = torch.empty((1, NQ // 2), device="cuda")
+    h = torch.empty((1, F), device="cuda")
+    out = torch.empty((1, H), device="cuda")
+    wsz = max(dq.dq_workspace_bytes(dq.DQ_OP_Q4K_GEMV, NQ, KQ, 1), dq.dq_workspace_bytes(dq.DQ_OP_Q4K_SWIGLU, F, H, 1),
+              dq.dq_workspace_bytes(dq.DQ_OP_Q4K_GEMV, H, F, 1), 16)
+    ws = torch.empty(wsz, dtype=torch.uint8, device="cuda")
+
+    def step():
+        dq.q4k_gemv_split_qg(dwq, xq, NQ, KQ, 128, q=q, g=gq, workspace=ws)
+        dq.q4k_swiglu_gemv(dwg, dwu, x, F, H, out=h, workspace=ws)
+        dq.q4k_gemv(dwd, h, H, F, y=out, workspace=ws)
+
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        step()                                  # warm-up outside the capture
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        step()
+    for tensor in (q, gq, h, out):
+        tensor.fill_(float("nan"))
+    graph.replay()
+    graph.replay()
+    torch.cuda.synchronize()
+    qv, gv, hv, ov = host(q), host(gq), host(h), host(out)
+
+    yq_ref, aq = oracle.q4k_gemv(wq, NQ, KQ, host(xq))
+    qr, gr = oracle.split_qg(yq_ref, 128)
+    tq, tg = oracle.split_qg(oracle.gemv_tolerance(aq), 128)
+    assert np.all(np.abs(qv - qr) <= tq) and np.all(np.abs(gv - gr) <= tg)
+    xh = host(x)
+    g_ref, a_g = oracle_rows(lambda rows: oracle.q4k_gemv(wg, F, H, xh, rows=rows), F, np.arange(F))
+    u_ref, a_u = oracle_rows(lambda rows: oracle.q4k_gemv(wu, F, H, xh, rows=rows), F, np.arange(F))
+    assert np.all(np.abs(hv - oracle.swiglu(g_ref, u_ref)) <= oracle.swiglu_tolerance(g_ref, u_ref, a_g, a_u))
+    # the down projection of the GPU's own SwiGLU output
+    y_ref, a_ref = oracle_rows(lambda rows: oracle.q4k_gemv(wdn, H, F, hv, rows=rows), H, np.arange(H))
+    assert_within(ov, y_ref, a_ref, "down projection replayed from the graph")
