@@ -330,6 +330,29 @@ def graph_table():
         del ws
         torch.cuda.empty_cache()
 
+    # Q, K and V projections of a hidden-4096 layer (8 KV heads of 128): one grouped
+    # launch, and three separate calls
+    rng = np.random.default_rng(43)
+    Hq, Ns = 4096, (4096, 1024, 1024)
+    per_set = sum(n * (Hq // 256) * 144 for n in Ns)
+    copies = min(64, max(1, int(np.ceil(1.3 * l2 / per_set))))
+    qkv = [[torch.from_numpy(synth.q4k_matrix(rng, n, Hq)).cuda() for n in Ns]]
+    for _ in range(1, copies):
+        qkv.append([t.clone() for t in qkv[0]])
+    xq = torch.from_numpy(synth.activations(rng, 1, Hq)).cuda()
+    outs = [torch.empty(n, device="cuda") for n in Ns]
+    scratch = torch.empty(1 << 24, dtype=torch.uint8, device="cuda")
+    timed("qkv_4096+1024+1024x4096:group", lambda i: dq.q4k_gemv_group(qkv[i], xq[0], list(Ns), Hq, ys=outs,
+                                                                       workspace=scratch), per_set + 4 * Hq, copies)
+
+    def separate(i):
+        for m, n in enumerate(Ns):
+            dq.q4k_gemv(qkv[i][m], xq, n, Hq, y=outs[m].view(1, n), workspace=scratch)
+
+    timed("qkv_4096+1024+1024x4096:separate", separate, per_set + 4 * Hq, copies)
+    del qkv
+    torch.cuda.empty_cache()
+
     # one decode step's GEMV sequence: q-projection with the Q/gate split (16 heads of
     # 128), SwiGLU 2 x 12288 x 4096, and the down projection 4096 x 12288 of its output
     rng = np.random.default_rng(41)

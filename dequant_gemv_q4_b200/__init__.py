@@ -31,7 +31,8 @@ Q8_0_BLOCK_ELEMS, Q8_0_BLOCK_BYTES = 32, 34
 
 EXPORTED = ("q8_0_gemv", "q4k_gemv", "q4k_swiglu_gemv", "q4k_repack_soa", "dq_workspace_bytes",
             "q8_0_dequant", "q4k_dequant", "dq_status_string", "dq_last_cuda_error",
-            "dq_device_error", "q4k_gemv_noalloc", "dq_noalloc_scratch_bytes", "q4k_gemv_split_qg")
+            "dq_device_error", "q4k_gemv_noalloc", "dq_noalloc_scratch_bytes", "q4k_gemv_split_qg",
+            "q4k_gemv_group")
 
 
 class DQError(RuntimeError):
@@ -72,6 +73,7 @@ def load_library(path: str = LIB_PATH):
             "dq_device_error": [p, i32, p],
             "q4k_gemv_noalloc": [p, i32, p, p, i64, i64, i32, p, p],
             "q4k_gemv_split_qg": [p, i32, p, p, p, i64, i64, i32, i64, p, sz, p],
+            "q4k_gemv_group": [i32, p, p, p, i32, p, i64, p, sz, p],
         }
         for name, args in sigs.items():
             f = getattr(lib, name)
@@ -262,6 +264,40 @@ def q4k_gemv_split_qg(w, x, N: int, K: int, head_dim: int, layout="aos", q=None,
     if one_d:
         return q.view(half), g.view(half)
     return q.view(B, half), g.view(B, half)
+
+
+MAX_GROUP = 4
+
+
+def q4k_gemv_group(ws, x, Ns, K: int, layout="aos", ys=None, workspace=None, stream=None):
+    """Batch-1 GEMVs of up to four Q4_K matrices sharing x, in one launch.
+
+    ws: list of weight tensors (N_m x K each); Ns: their row counts; x: (K,)
+    fp32.  Returns the list of outputs (N_m,) (or fills ``ys``)."""
+    torch = _torch()
+    lib = load_library()
+    count = len(ws)
+    if not 1 <= count <= MAX_GROUP or len(Ns) != count:
+        raise ValueError("1 to %d matrices, one row count each" % MAX_GROUP)
+    x2 = _x2d(x, K)
+    if x2.shape[0] != 1:
+        raise ValueError("a grouped GEMV takes one activation vector")
+    wps = [_weights(w, "w[%d]" % m, int(n), K, Q4K_BLOCK_ELEMS, Q4K_BLOCK_BYTES) for m, (w, n) in enumerate(zip(ws, Ns))]
+    if ys is None:
+        ys = [torch.empty(int(n), dtype=torch.float32, device=x.device) for n in Ns]
+    yps = [_dev(yv, "y[%d]" % m, torch.float32) for m, yv in enumerate(ys)]
+    for yv, n in zip(ys, Ns):
+        if yv.numel() != int(n):
+            raise ValueError("each output must hold N[m] floats")
+    padded = sum((int(n) + 15) // 16 * 16 for n in Ns)
+    need = dq_workspace_bytes(DQ_OP_Q4K_GEMV, padded, K, 1)
+    wsp, wsn, _keep = _workspace(workspace, need, x.device)
+    arr_w = (ctypes.c_void_p * count)(*[wp.value for wp in wps])
+    arr_n = (ctypes.c_int64 * count)(*[int(n) for n in Ns])
+    arr_y = (ctypes.c_void_p * count)(*[yp.value for yp in yps])
+    _check("q4k_gemv_group", lib.q4k_gemv_group(count, arr_w, arr_n, arr_y, _layout(layout),
+                                                ctypes.c_void_p(x2.data_ptr()), K, wsp, wsn, _stream(stream)))
+    return ys
 
 
 def q4k_swiglu_gemv(w_gate, w_up, x, N: int, K: int, layout="aos", out=None, workspace=None,

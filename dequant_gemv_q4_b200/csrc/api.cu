@@ -55,6 +55,7 @@ dq_status dev_info(DevInfo &di)
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+
 // Workspace layout of the Q4_K GEMV for a plan: [split partials][argmax candidates].
 struct Q4KWorkspace {
     size_t part_bytes;
@@ -85,7 +86,8 @@ dq_status check_q4k_shape(int64_t N, int64_t K, int B)
 
 dq_status q4k_common(const void *w0, const void *w1, int layout, const float *x, float *y, int64_t N, int64_t K,
                      int B, int NS, int64_t *argmax_out, void *workspace, size_t ws_bytes, void *stream,
-                     float *g_out = nullptr, int64_t qg_hd = 0)
+                     float *g_out = nullptr, int64_t qg_hd = 0, const dq::GroupOut *grp = nullptr,
+                     const void *const *gw = nullptr)
 {
     if (!w0 || (NS == 2 && !w1) || !x || !y)
         return DQ_ERR_NULL;
@@ -105,7 +107,7 @@ dq_status q4k_common(const void *w0, const void *w1, int layout, const float *x,
         return st;
     const dq::Q4KPlan pl = dq::q4k_plan(N, static_cast<int>(K), B, NS, layout == DQ_LAYOUT_SOA, di.sm_count,
                                         di.smem_optin);
-    if (!pl.ok)
+    if (!pl.ok || (grp && !pl.fx))
         return DQ_ERR_SHAPE;
     const Q4KWorkspace ws = q4k_ws(pl, N, B, NS, argmax_out != nullptr);
     if (ws.total() > 0 && (!workspace || ws_bytes < ws.total()))
@@ -121,6 +123,11 @@ dq_status q4k_common(const void *w0, const void *w1, int layout, const float *x,
     p.y = y;
     p.g = g_out;
     p.qg_hd = static_cast<int>(qg_hd);
+    if (grp) {
+        p.grp = *grp;
+        for (int m = 0; m < grp->n; ++m)
+            p.gw[m] = static_cast<const uint8_t *>(gw[m]);
+    }
     p.part = (pl.splits > 1 && !pl.cluster) ? reinterpret_cast<float *>(wsb) : nullptr;
     p.cand = argmax_out ? reinterpret_cast<dq::ArgmaxCand *>(wsb + ws.part_bytes) : nullptr;
     p.err = dq::device_error_flag(di.device);
@@ -140,7 +147,8 @@ dq_status q4k_common(const void *w0, const void *w1, int layout, const float *x,
     if (e != cudaSuccess)
         return cuda_fail(e);
     if (pl.splits > 1 && !pl.cluster) {
-        e = dq::splitk_reduce_launch(p.part, pl.splits, NS, B, N, y, p.g, p.qg_hd, p.cand, dq::reduce_grid(N, B), s);
+        e = dq::splitk_reduce_launch(p.part, pl.splits, NS, B, N, y, p.g, p.qg_hd, p.grp, p.cand, dq::reduce_grid(N, B),
+                                     s);
         if (e != cudaSuccess)
             return cuda_fail(e);
     }
@@ -228,6 +236,37 @@ dq_status q4k_gemv_split_qg(const void *w, int layout, const float *x, float *q,
     if (qa < ga + span && ga < qa + span)
         return DQ_ERR_ARG;
     return q4k_common(w, nullptr, layout, x, q, N, K, B, 1, nullptr, workspace, ws_bytes, stream, g, head_dim);
+}
+
+dq_status q4k_gemv_group(int count, const void *const *w, const int64_t *N, float *const *y, int layout,
+                         const float *x, int64_t K, void *workspace, size_t ws_bytes, void *stream)
+{
+    if (!w || !N || !y)
+        return DQ_ERR_NULL;
+    if (count < 1 || count > dq::kMaxGroup)
+        return DQ_ERR_ARG;
+    dq::GroupOut grp{};
+    grp.n = count;
+    int64_t total = 0;
+    for (int m = 0; m < count; ++m) {
+        if (!w[m] || !y[m])
+            return DQ_ERR_NULL;
+        if (N[m] < 1 || N[m] > (int64_t(1) << 40))
+            return DQ_ERR_SHAPE;
+        if (!aligned(w[m], 16))
+            return DQ_ERR_ALIGN;
+        if (!aligned(y[m], 4))
+            return DQ_ERR_ALIGN;
+        grp.y[m] = y[m];
+        grp.N[m] = N[m];
+        grp.base[m] = total;
+        // each matrix's rows are padded to the batch-1 kernel's row tile
+        const int64_t tile = dq::q4k_fx_tile_rows();
+        total += (N[m] + tile - 1) / tile * tile;
+    }
+    // y is only a stand-in here: every output goes through the group map
+    return q4k_common(w[0], nullptr, layout, x, y[0], total, K, 1, 1, nullptr, workspace, ws_bytes, stream, nullptr, 0,
+                      &grp, w);
 }
 
 dq_status q4k_swiglu_gemv(const void *w_gate, const void *w_up, int layout, const float *x, float *out, int64_t N,

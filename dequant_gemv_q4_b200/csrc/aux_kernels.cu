@@ -190,7 +190,7 @@ int reduce_grid(long long N, int B)
 __global__ void __launch_bounds__(kReduceThreads) splitk_reduce_kernel(const float *__restrict__ part, int splits,
                                                                        int NS, int B, long long N,
                                                                        float *__restrict__ y, float *__restrict__ g_out,
-                                                                       int qg_hd, ArgmaxCand *cand)
+                                                                       int qg_hd, const GroupOut grp, ArgmaxCand *cand)
 {
     pdl_wait();
     pdl_launch_dependents();
@@ -208,6 +208,20 @@ __global__ void __launch_bounds__(kReduceThreads) splitk_reduce_kernel(const flo
                 u += part[((static_cast<long long>(s) * NS + 1) * B + b) * N + n];
         }
         const float out = (NS == 2) ? g / (1.0f + expf(-g)) * u : g;
+        if (grp.n > 0) {
+            // padded row n of a grouped GEMV: the matrix holding it, and its row there
+            int m = 0;
+#pragma unroll
+            for (int k = 1; k < kMaxGroup; ++k)
+                if (k < grp.n && n >= grp.base[k])
+                    m = k;
+            const long long base = m == 0 ? grp.base[0] : m == 1 ? grp.base[1] : m == 2 ? grp.base[2] : grp.base[3];
+            const long long rows = m == 0 ? grp.N[0] : m == 1 ? grp.N[1] : m == 2 ? grp.N[2] : grp.N[3];
+            float *ym = m == 0 ? grp.y[0] : m == 1 ? grp.y[1] : m == 2 ? grp.y[2] : grp.y[3];
+            if (n - base < rows)
+                ym[n - base] = out;
+            continue;
+        }
         *gemv_out_addr(y, g_out, qg_hd, N, b, n) = out;
         if (cand && cand_better(out, n, best_v, best_i)) {
             best_v = out;
@@ -241,10 +255,10 @@ __global__ void __launch_bounds__(kReduceThreads) splitk_reduce_kernel(const flo
 }
 
 cudaError_t splitk_reduce_launch(const float *part, int splits, int NS, int B, long long N, float *y, float *g,
-                                 int qg_hd, ArgmaxCand *cand, int grid, cudaStream_t s)
+                                 int qg_hd, const GroupOut &grp, ArgmaxCand *cand, int grid, cudaStream_t s)
 {
     return launch_pdl(splitk_reduce_kernel, dim3(grid), dim3(kReduceThreads), 0, s, part, splits, NS, B, N, y, g,
-                      qg_hd, cand);
+                      qg_hd, grp, cand);
 }
 
 // One CTA folds all candidates into the final index.

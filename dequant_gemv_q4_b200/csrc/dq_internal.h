@@ -10,6 +10,18 @@ namespace dq {
 
 struct ArgmaxCand;
 
+constexpr int kMaxGroup = 4;
+
+// Outputs of a grouped GEMV: n > 0 matrices whose row tiles follow each other;
+// matrix m holds padded rows base[m] .. base[m] + N[m] - 1 (base[m] a multiple of
+// the tile height) and writes y[m][0 .. N[m]-1].  n == 0: not a group.
+struct GroupOut {
+    int n;
+    float *y[kMaxGroup];
+    long long N[kMaxGroup];
+    long long base[kMaxGroup];
+};
+
 // Q4_K GEMV kernel arguments (one weight stream, or gate + up for SwiGLU).
 struct Q4KParams {
     const uint8_t *w[2];
@@ -31,6 +43,8 @@ struct Q4KParams {
     int argmax;
     long long tiles;       // row tiles
     int cluster;           // fx kernel: split partials are added inside each cluster of `splits` CTAs
+    GroupOut grp;          // grouped GEMV (fx kernel, batch 1): N is then the padded total
+    const uint8_t *gw[kMaxGroup];   // weights of the grouped matrices
 };
 
 struct Q4KPlan {
@@ -55,6 +69,7 @@ Q4KPlan q4k_plan(long long N, int K, int B, int NS, int soa, int sm_count, int s
 cudaError_t q4k_gemv_launch(const Q4KParams &p, const Q4KPlan &pl, int B, int NS, cudaStream_t s);
 int q4k_pick_warps(long long tiles, int sm_count, int max_warps, bool round4 = false);
 Q4KPlan q4k_plan_fx(long long N, int nb, int NS, int sm_count, int smem_optin);
+int q4k_fx_tile_rows();
 cudaError_t q4k_gemv_fx_launch(const Q4KParams &p, const Q4KPlan &pl, int NS, cudaStream_t s);
 
 // Q8_0 GEMV
@@ -79,7 +94,7 @@ cudaError_t q8_0_gemv_launch(const Q8Params &p, const Q8Plan &pl, int B, cudaStr
 // split-K reduction (+ SwiGLU epilogue, + argmax candidates), argmax finalisation
 int reduce_grid(long long N, int B);
 cudaError_t splitk_reduce_launch(const float *part, int splits, int NS, int B, long long N, float *y, float *g,
-                                 int qg_hd, ArgmaxCand *cand, int grid, cudaStream_t s);
+                                 int qg_hd, const GroupOut &grp, ArgmaxCand *cand, int grid, cudaStream_t s);
 cudaError_t argmax_finalize_launch(const ArgmaxCand *cand, int ncand, long long *out, cudaStream_t s);
 
 // debug dequant, repack

@@ -82,13 +82,15 @@ constexpr int kFxRowPitch = kFxChunkBytes + 16;           // 592
 constexpr int kFxSlotBytes = kFxTileRows * kFxRowPitch;
 static_assert(kFxSlotBytes % 128 == 0, "slots must keep the ring 128-byte aligned");
 constexpr int kFxMaxWarps = 12;
+int q4k_fx_tile_rows() { return kFxTileRows; }
 // In-cluster split reduction: per warp and stream, the 16 row partials (fp64).
 constexpr int kFxClusterPartBytes = 2 * kFxTileRows * 8;
 constexpr int kFxMaxCluster = 8;
 
-// TMA descriptors of the (up to two) weight streams.
+// TMA descriptors of the weight matrices: SwiGLU's gate and up, or one per
+// matrix of a grouped GEMV.
 struct FxMaps {
-    CUtensorMap m[2];
+    CUtensorMap m[kMaxGroup];
 };
 
 // Converts the activations of super-blocks kb_begin .. kb_begin + nbs - 1 into
@@ -188,6 +190,37 @@ __device__ __forceinline__ void fx_slice(const uint4 (&q)[R], const uint8_t *xlo
     }
 }
 
+// The matrix a slot reads and its rows: SwiGLU stream st of the same rows, or,
+// for a grouped GEMV, the matrix holding padded row row0 and the row there.
+struct FxRows {
+    int sel;
+    long long row0;
+    long long nrows;
+};
+__device__ __forceinline__ FxRows fx_rows(const Q4KParams &p, int st, long long row0)
+{
+    if (p.grp.n == 0)
+        return {st, row0, p.N};
+    int m = 0;
+#pragma unroll
+    for (int k = 1; k < kMaxGroup; ++k)
+        if (k < p.grp.n && row0 >= p.grp.base[k])
+            m = k;
+    const long long base = m == 0 ? p.grp.base[0] : m == 1 ? p.grp.base[1] : m == 2 ? p.grp.base[2] : p.grp.base[3];
+    const long long rows = m == 0 ? p.grp.N[0] : m == 1 ? p.grp.N[1] : m == 2 ? p.grp.N[2] : p.grp.N[3];
+    return {m, row0 - base, rows};
+}
+__device__ __forceinline__ const uint8_t *fx_weights(const Q4KParams &p, int sel)
+{
+    if (p.grp.n == 0)
+        return sel == 0 ? p.w[0] : p.w[1];
+    return sel == 0 ? p.gw[0] : sel == 1 ? p.gw[1] : sel == 2 ? p.gw[2] : p.gw[3];
+}
+__device__ __forceinline__ float *fx_group_out(const Q4KParams &p, int sel)
+{
+    return sel == 0 ? p.grp.y[0] : sel == 1 ? p.grp.y[1] : sel == 2 ? p.grp.y[2] : p.grp.y[3];
+}
+
 // Issues the copies of one slot (K-chunk c_begin + cur.kcl of stream cur.st of
 // the tile at cur.row0).  TMA: lane 0 arms the slot's mbarrier and issues one
 // tile copy (elements past the matrix are filled with zeros and still counted).
@@ -200,27 +233,29 @@ __device__ __forceinline__ void fx_issue_slot(const Q4KParams &p, const FxMaps &
     const int kb0 = (c_begin + cur.kcl) * kFxBPC;
     const uint32_t bar = bars_s + slot * 8;
     const uint32_t dst = ring_s + slot * kFxSlotBytes;
+    const FxRows fr = fx_rows(p, cur.st, cur.row0);
     if constexpr (TMA) {
         if (lane == 0) {
             mbar_arrive_expect_tx(bar, static_cast<uint32_t>(kFxSlotBytes));
-            const CUtensorMap *m = cur.st == 0 ? &maps.m[0] : &maps.m[1];
+            const CUtensorMap *m = fr.sel == 0 ? &maps.m[0] : fr.sel == 1 ? &maps.m[1] : fr.sel == 2 ? &maps.m[2]
+                                                                                                      : &maps.m[3];
             // x = kb0 * 36 words: a multiple of 4 words, i.e. of 16 bytes
             asm volatile(
                 "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
                 "[%4];" ::"r"(dst),
-                "l"(m), "r"(kb0 * (kQ4KBlockBytes / 4)), "r"(static_cast<int>(cur.row0)), "r"(bar)
+                "l"(m), "r"(kb0 * (kQ4KBlockBytes / 4)), "r"(static_cast<int>(fr.row0)), "r"(bar)
                 : "memory");
         }
     } else {
         const long long row_bytes_g = static_cast<long long>(p.nb) * kQ4KBlockBytes;
-        const int rows = static_cast<int>(min(static_cast<long long>(kFxTileRows), p.N - cur.row0));
+        const int rows = static_cast<int>(min(static_cast<long long>(kFxTileRows), fr.nrows - fr.row0));
         const int nblk = min(kFxBPC, p.nb - kb0);
         const uint32_t bytes = static_cast<uint32_t>(nblk * kQ4KBlockBytes);
         if (lane == 0)
             mbar_arrive_expect_tx(bar, static_cast<uint32_t>(rows) * bytes);
         __syncwarp();
         if (lane < rows) {
-            const uint8_t *src = (cur.st == 0 ? p.w[0] : p.w[1]) + (cur.row0 + lane) * row_bytes_g +
+            const uint8_t *src = fx_weights(p, fr.sel) + (fr.row0 + lane) * row_bytes_g +
                                  static_cast<long long>(kb0) * kQ4KBlockBytes;
             bulk_g2s(dst + lane * kFxRowPitch, src, bytes, bar);
         }
@@ -445,6 +480,12 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
             }
         }
         const long long n = row0 + wrow;
+        if (p.grp.n > 0 && !p.cluster && p.splits == 1) {
+            const FxRows fr = fx_rows(p, 0, row0);
+            if (writer && fr.row0 + wrow < fr.nrows)
+                fx_group_out(p, fr.sel)[fr.row0 + wrow] = static_cast<float>(t);
+            continue;
+        }
         if (p.cluster) {
             // this warp's only tile: keep its partials for the cluster reduction
             if (writer) {
@@ -504,7 +545,11 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
                 u += rp[(warp * 2 + 1) * kFxTileRows + lane];
             }
             const long long n = t0 * kFxTileRows + lane;
-            if (n < p.N) {
+            const FxRows fr = fx_rows(p, 0, t0 * kFxTileRows);
+            if (p.grp.n > 0) {
+                if (fr.row0 + lane < fr.nrows)
+                    fx_group_out(p, fr.sel)[fr.row0 + lane] = static_cast<float>(g);
+            } else if (n < p.N) {
                 float out;
                 if constexpr (NS == 2) {
                     const float gv = static_cast<float>(g);
@@ -676,10 +721,18 @@ cudaError_t q4k_gemv_fx_launch(const Q4KParams &p, const Q4KPlan &pl, int NS, cu
     FxMaps maps;
     memset(&maps, 0, sizeof(maps));
     if (pl.tma) {
-        for (int st = 0; st < NS; ++st) {
-            const cudaError_t e = encode_weight_map(&maps.m[st], p.w[st], p.N, p.nb);
-            if (e != cudaSuccess)
-                return e;
+        if (p.grp.n > 0) {
+            for (int m = 0; m < p.grp.n; ++m) {
+                const cudaError_t e = encode_weight_map(&maps.m[m], p.gw[m], p.grp.N[m], p.nb);
+                if (e != cudaSuccess)
+                    return e;
+            }
+        } else {
+            for (int st = 0; st < NS; ++st) {
+                const cudaError_t e = encode_weight_map(&maps.m[st], p.w[st], p.N, p.nb);
+                if (e != cudaSuccess)
+                    return e;
+            }
         }
         return NS == 1 ? launch_fx<1, true>(p, maps, pl, s) : launch_fx<2, true>(p, maps, pl, s);
     }

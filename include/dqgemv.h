@@ -132,6 +132,25 @@ dq_status q4k_gemv_split_qg(const void *w, int layout, const float *x, float *q,
                             int B, int64_t head_dim, void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * Grouped batch-1 Q4_K GEMV: up to DQ_MAX_GROUP matrices that share one
+ * activation vector (for example the Q, K and V projections of a layer) in one
+ * launch (qualiaDB cuda_lane: try_q4k_soa_qkv):
+ *   y[m][n] = sum_k W_m[n][k] * x[k],  m < count, n < N[m].
+ *   count       1..DQ_MAX_GROUP.
+ *   w, N, y     HOST arrays of `count` entries, read during the call: device
+ *               pointers to each matrix (N[m] x K Q4_K super-blocks, 16-byte
+ *               aligned, all in `layout`), row counts (>= 1), and device
+ *               outputs of N[m] fp32 (4-byte aligned).
+ *   x           K fp32, 16-byte aligned.   K  positive multiple of 256.
+ *   workspace   at least dq_workspace_bytes(DQ_OP_Q4K_GEMV, P, K, 1, 0) bytes,
+ *               P = sum over m of N[m] rounded up to a multiple of 16.
+ * Numerics as for q4k_gemv with B == 1.
+ */
+#define DQ_MAX_GROUP 4
+dq_status q4k_gemv_group(int count, const void *const *w, const int64_t *N, float *const *y, int layout,
+                         const float *x, int64_t K, void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * Fused gate/up SwiGLU GEMV (qualiaDB cuda_lane: try_q4k_soa_fused_swiglu;
  * trueno WgslForwardPass: silu_mul_shader, here fused into the GEMV):
  *   out[b][n] = silu(g) * u,  g = (W_gate x_b)[n],  u = (W_up x_b)[n],

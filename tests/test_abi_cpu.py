@@ -129,3 +129,19 @@ def test_split_qg_rejects_on_host(lib):
     assert f(A16, 0, A16, A16, P((1 << 20) + 512), 512, 256, 1, 64, None, 0, None) == DQ_ERR_ARG
     # and the shared Q4_K checks still apply (K not a multiple of 256)
     assert f(A16, 0, A16, A16, A16b, 512, 100, 1, 64, None, 0, None) == DQ_ERR_SHAPE
+
+
+def test_group_rejects_on_host(lib):
+    f = lib.q4k_gemv_group
+    W = (P * 2)(A16, A16)
+    Y = (P * 2)(A16, A16)
+    N = (ctypes.c_int64 * 2)(64, 32)
+    assert f(0, W, N, Y, 0, A16, 256, None, 0, None) == DQ_ERR_ARG
+    assert f(5, W, N, Y, 0, A16, 256, None, 0, None) == DQ_ERR_ARG
+    assert f(2, None, N, Y, 0, A16, 256, None, 0, None) == DQ_ERR_NULL
+    assert f(2, (P * 2)(A16, None), N, Y, 0, A16, 256, None, 0, None) == DQ_ERR_NULL
+    assert f(2, W, (ctypes.c_int64 * 2)(64, 0), Y, 0, A16, 256, None, 0, None) == DQ_ERR_SHAPE
+    assert f(2, (P * 2)(A16, A8), N, Y, 0, A16, 256, None, 0, None) == DQ_ERR_ALIGN
+    assert f(2, W, N, (P * 2)(A16, P((1 << 20) + 2)), 0, A16, 256, None, 0, None) == DQ_ERR_ALIGN
+    assert f(2, W, N, Y, 0, A16, 100, None, 0, None) == DQ_ERR_SHAPE
+    assert f(2, W, N, Y, 7, A16, 256, None, 0, None) == DQ_ERR_LAYOUT

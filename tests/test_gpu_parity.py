@@ -516,3 +516,24 @@ def test_ffn_and_qproj_sequence_replays_from_a_cuda_graph():
     # the down projection of the GPU's own SwiGLU output
     y_ref, a_ref = oracle_rows(lambda rows: oracle.q4k_gemv(wdn, H, F, hv, rows=rows), H, np.arange(H))
     assert_within(ov, y_ref, a_ref, "down projection replayed from the graph")
+
+
+# --- grouped batch-1 GEMV (QKV-style projections in one launch) --------------------------
+
+@pytest.mark.parametrize("Ns,K,layout", [
+    ((4096, 1024, 1024), 4096, "aos"),   # Q, K, V of a hidden-4096 layer with 8 KV heads of 128
+    ((4096, 1024, 1024), 4096, "soa"),
+    ((1000, 24, 7, 333), 5120, "aos"),   # ragged row counts, four matrices
+    ((40, 72), 65536, "aos"),            # long K: split into many parts
+    ((3000,), 1024, "aos"),              # a group of one
+])
+def test_q4k_gemv_group_matches_separate_oracle_gemvs(Ns, K, layout):
+    rng = np.random.default_rng(sum(Ns) + K)
+    ws = [synth.q4k_matrix(rng, n, K) for n in Ns]
+    x = synth.activations(rng, 1, K)
+    wls = ws if layout == "aos" else [oracle.q4k_repack_soa(w, n, K) for w, n in zip(ws, Ns)]
+    ys = dq.q4k_gemv_group([dev(w) for w in wls], dev(x[0]), list(Ns), K, layout=layout)
+    for m, (w, n) in enumerate(zip(ws, Ns)):
+        y = host(ys[m])
+        y_ref, a_ref = oracle.q4k_gemv(w, n, K, x)
+        assert_within(y[None, :], y_ref, a_ref, "group matrix %d" % m)
