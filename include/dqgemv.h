@@ -27,7 +27,8 @@
  *   - Q8_0 and Q4_K with B >= 2: every weight is formed exactly as the fp32
  *     value nearest to its dequantized value (the bits the *_dequant entry
  *     points return) and the products are accumulated in fp32.
- *   - Q4_K with B == 1 (q4k_gemv, q4k_swiglu_gemv): each activation is rounded
+ *   - Q4_K with B == 1 (q4k_gemv, q4k_swiglu_gemv, q4k_gemv_split_qg,
+ *     q4k_gemv_group): each activation is rounded
  *     to a 30-bit fixed point shared by its super-block of 256 activations;
  *     the dot products over the exact quants, scales and mins are then exact
  *     (integers, fp64), rounded once to fp32.  The error is at most
