@@ -106,4 +106,62 @@ __device__ __forceinline__ void q4_word_weights(uint32_t w, const ChunkScales &s
     wv[3] = __ffma2_rn(f2(__uint_as_float(u & 0xF00u), __uint_as_float(u & 0xF000u)), s.S1, s.M);
 }
 
+// One quant word (bytes 4t..4t+3 of a 16-byte slice): form its eight weights
+// and accumulate weight*x.  xa = {x[L+4t], x[H+4t], x[L+4t+1], x[H+4t+1]},
+// xb = the same for bytes 4t+2, 4t+3 (x is staged in (lo, hi) pairs).
+__device__ __forceinline__ void q4_word(uint32_t w, const ChunkScales &cs, float4 xa, float4 xb, float2 &acc0,
+                                        float2 &acc1)
+{
+    float2 wv[4];
+    q4_word_weights(w, cs, wv);
+    acc0 = __ffma2_rn(wv[0], f2(xa.x, xa.y), acc0);
+    acc1 = __ffma2_rn(wv[1], f2(xa.z, xa.w), acc1);
+    acc0 = __ffma2_rn(wv[2], f2(xb.x, xb.y), acc0);
+    acc1 = __ffma2_rn(wv[3], f2(xb.z, xb.w), acc1);
+}
+
+// x of one super-block is staged (fp32) as 8 slices x 8 float4, float4 k of
+// slice s = 2c+h holding {x[L+2k], x[H+2k], x[L+2k+1], x[H+2k+1]} (L = 64c+16h,
+// H = L+32): the (lo, hi) weight pairs of quant bytes 2k and 2k+1.  16 bytes of
+// padding per super-block.
+constexpr int kXBlockPitch = 1040;
+
+// Stages activations of super-blocks kb_begin .. kb_begin + nbs - 1 of B rows of
+// x (row b at x + b*K) in that layout, super-block kbl of row b at
+// xs + (b*nbs + kbl)*kXBlockPitch; each thread keeps kBatch loads in flight.
+template <int kBatch>
+__device__ __forceinline__ void stage_x_pairs(const float *x, int K, int B, int kb_begin, int nbs, uint8_t *xs)
+{
+    const int per_b = nbs * 64;  // float4 per batch row
+    const int n_out = B * per_b;
+    for (int base = threadIdx.x; base < n_out; base += kBatch * blockDim.x) {
+        float2 lo[kBatch], hi[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int idx = base + u * blockDim.x;
+            if (idx < n_out) {
+                const int b = idx / per_b;
+                const int rem = idx - b * per_b;
+                const int kbl = rem >> 6;
+                const int sl = (rem >> 3) & 7;    // slice
+                const int k = rem & 7;            // float4 within the slice
+                const float *xb = x + static_cast<long long>(b) * K + static_cast<long long>(kb_begin + kbl) * 256 +
+                                  64 * (sl >> 1) + 16 * (sl & 1) + 2 * k;
+                lo[u] = __ldg(reinterpret_cast<const float2 *>(xb));
+                hi[u] = __ldg(reinterpret_cast<const float2 *>(xb + 32));
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int idx = base + u * blockDim.x;
+            if (idx < n_out) {
+                const int b = idx / per_b;
+                const int rem = idx - b * per_b;
+                *reinterpret_cast<float4 *>(xs + (b * nbs + (rem >> 6)) * kXBlockPitch + ((rem >> 3) & 7) * 128 +
+                                            (rem & 7) * 16) = make_float4(lo[u].x, hi[u].x, lo[u].y, hi[u].y);
+            }
+        }
+    }
+}
+
 }  // namespace dq

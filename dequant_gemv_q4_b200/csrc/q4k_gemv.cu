@@ -41,27 +41,6 @@
 
 namespace dq {
 
-// One quant word (bytes 4t..4t+3 of a 16-byte slice): form its eight weights
-// and accumulate weight*x.  xa = {x[L+4t], x[H+4t], x[L+4t+1], x[H+4t+1]},
-// xb = the same for bytes 4t+2, 4t+3 (x is staged in (lo, hi) pairs).
-__device__ __forceinline__ void q4_word(uint32_t w, const ChunkScales &cs, float4 xa, float4 xb, float2 &acc0,
-                                        float2 &acc1)
-{
-    float2 wv[4];
-    q4_word_weights(w, cs, wv);
-    acc0 = __ffma2_rn(wv[0], f2(xa.x, xa.y), acc0);
-    acc1 = __ffma2_rn(wv[1], f2(xa.z, xa.w), acc1);
-    acc0 = __ffma2_rn(wv[2], f2(xb.x, xb.y), acc0);
-    acc1 = __ffma2_rn(wv[3], f2(xb.z, xb.w), acc1);
-}
-
-// x of one super-block is staged as 8 slices x 8 float4, float4 k of slice
-// s = 2c+h holding {x[L+2k], x[H+2k], x[L+2k+1], x[H+2k+1]} (L = 64c+16h,
-// H = L+32): the (lo, hi) weight pairs of quant bytes 2k and 2k+1.  16 bytes
-// of padding per super-block keep the lanes' reads free of bank conflicts.
-constexpr int kXBlockPitch = 1040;
-
-
 template <int LPR, int B, int NS, bool SOA>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_kernel(const Q4KParams p)
 {
@@ -141,42 +120,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_kernel(const Q4KPa
     }
 
     // stage this split's activations in (lo, hi) pairs (fp32, padded per super-block);
-    // each thread keeps kStageBatch loads in flight before storing (one at a
-    // time for large B, whose kernels have no registers to spare)
-    {
-        constexpr int kStageBatch = (B <= 2) ? 8 : 1;
-        const int per_b = nbs * 64;  // float4 per batch row
-        const int n_out = B * per_b;
-        for (int base = threadIdx.x; base < n_out; base += kStageBatch * blockDim.x) {
-            float2 lo[kStageBatch], hi[kStageBatch];
-#pragma unroll
-            for (int u = 0; u < kStageBatch; ++u) {
-                const int idx = base + u * blockDim.x;
-                if (idx < n_out) {
-                    const int b = idx / per_b;
-                    const int rem = idx - b * per_b;
-                    const int kbl = rem >> 6;
-                    const int sl = (rem >> 3) & 7;    // slice
-                    const int k = rem & 7;            // float4 within the slice
-                    const float *xb = p.x + static_cast<long long>(b) * p.K +
-                                      static_cast<long long>(kb_begin + kbl) * 256 + 64 * (sl >> 1) + 16 * (sl & 1) +
-                                      2 * k;
-                    lo[u] = __ldg(reinterpret_cast<const float2 *>(xb));
-                    hi[u] = __ldg(reinterpret_cast<const float2 *>(xb + 32));
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < kStageBatch; ++u) {
-                const int idx = base + u * blockDim.x;
-                if (idx < n_out) {
-                    const int b = idx / per_b;
-                    const int rem = idx - b * per_b;
-                    *reinterpret_cast<float4 *>(xs + (b * nbs + (rem >> 6)) * kXBlockPitch + ((rem >> 3) & 7) * 128 +
-                                                (rem & 7) * 16) = make_float4(lo[u].x, hi[u].x, lo[u].y, hi[u].y);
-                }
-            }
-        }
-    }
+    // each thread keeps 8 loads in flight before storing (one at a time for
+    // large B, whose kernels have no registers to spare)
+    stage_x_pairs<(B <= 2) ? 8 : 1>(p.x, p.K, B, kb_begin, nbs, xs);
     __syncthreads();
 
     float best_v = -INFINITY;
@@ -782,11 +728,12 @@ static Q4KPlan plan_full_block(long long N, int nb, int NS, int sm_count, int sm
 Q4KPlan q4k_plan(long long N, int K, int B, int NS, int soa, int sm_count, int smem_optin)
 {
     const int nb = K / kQ4KBlockElems;
+    // quarter-warp lanes with TMA slots: integer dot products on fixed-point
+    // activations at batch 1, exact fp32 weights at batch 2..8
+    const Q4KPlan pf = q4k_plan_fx(N, nb, B, NS, sm_count, smem_optin);
+    if (pf.ok)
+        return pf;
     if (B == 1) {
-        // batch 1: integer dot products on fixed-point activations
-        const Q4KPlan pf = q4k_plan_fx(N, nb, NS, sm_count, smem_optin);
-        if (pf.ok)
-            return pf;
         // Half-block lanes halve each warp's serial chain of slots (better when
         // every warp gets only a few slots); full-block lanes spend fewer
         // instructions per weight (better for long matrices).
@@ -841,7 +788,7 @@ static cudaError_t launch_half(const Q4KParams &p, const Q4KPlan &pl, cudaStream
 cudaError_t q4k_gemv_launch(const Q4KParams &p, const Q4KPlan &pl, int B, int NS, cudaStream_t s)
 {
     if (pl.fx)
-        return q4k_gemv_fx_launch(p, pl, NS, s);
+        return q4k_gemv_fx_launch(p, pl, B, NS, s);
     if (pl.half) {
         if (pl.lpr == 32)
             return NS == 1 ? launch_half<32, 1>(p, pl, s) : launch_half<32, 2>(p, pl, s);

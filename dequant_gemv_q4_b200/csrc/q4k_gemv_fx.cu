@@ -62,6 +62,7 @@
 
 #include "dq_common.cuh"
 #include "dq_internal.h"
+#include "q4k_decode.cuh"
 #include "q4k_stream.cuh"
 
 namespace dq {
@@ -594,6 +595,249 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
 }
 
 // ---------------------------------------------------------------------------
+// Batches of 2..8 activation rows: the same quarter-warp lanes, TMA slots and
+// rings, with exact fp32 weights (formed once per weight, used B times) and
+// fp32 accumulation, as in the full-block fp32 kernel.  x is staged in fp32
+// (lo, hi) pairs; each quarter-warp reads its super-block's pairs as a
+// broadcast.
+// ---------------------------------------------------------------------------
+
+// Sums the values of the four quarter-warps (lanes i, i+8, i+16, i+24) with a
+// transposing butterfly over lane bits 4 and 3: on entry every lane holds M
+// values (M a multiple of 4); on exit it holds the totals of indices
+// off .. off + M/4 - 1, off = (bit 4 ? M/2 : 0) + (bit 3 ? M/4 : 0).
+template <int M>
+__device__ __forceinline__ void quarter_sum(float (&v)[M], int lane)
+{
+    static_assert(M % 4 == 0, "four quarter-warps share the values");
+    const bool up16 = (lane & 16) != 0;
+#pragma unroll
+    for (int k = 0; k < M / 2; ++k) {
+        const float send = up16 ? v[k] : v[k + M / 2];
+        const float keep = up16 ? v[k + M / 2] : v[k];
+        v[k] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+    const bool up8 = (lane & 8) != 0;
+#pragma unroll
+    for (int k = 0; k < M / 4; ++k) {
+        const float send = up8 ? v[k] : v[k + M / 4];
+        const float keep = up8 ? v[k + M / 4] : v[k];
+        v[k] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+}
+
+constexpr int kFxbMaxWarps(int B) { return B <= 2 ? 12 : 8; }
+
+template <int B, int NS, bool SOA, bool TMA>
+__global__ void __launch_bounds__(kFxbMaxWarps(B) * 32, 1)
+    q4k_gemv_fxb_kernel(const __grid_constant__ Q4KParams p, const __grid_constant__ FxMaps maps)
+{
+    constexpr int R = kFxRows;
+    constexpr int MV = R * B;                 // values per lane per stream (index r*B + b)
+    constexpr int MP = (MV + 3) / 4 * 4;      // padded for the quarter-warp butterfly
+    constexpr int VPL = MP / 4;               // values per lane after it
+    static_assert(R == 2 && B >= 2 && B <= 8, "two rows per lane, batches of 2 to 8");
+
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int nwarps = blockDim.x >> 5;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int g = lane >> 3;   // super-block of each chunk
+    const int i = lane & 7;    // rows i and i + 8 of each tile
+    const int voff = ((lane & 16) ? MP / 2 : 0) + ((lane & 8) ? MP / 4 : 0);
+
+    const int split = blockIdx.x / p.ctas_per_split;
+    const int cj = blockIdx.x % p.ctas_per_split;
+    const int nchunk_total = (p.nb + kFxBPC - 1) / kFxBPC;
+    const int c_begin = split * p.chunks_per_split;
+    const int c_end = min(c_begin + p.chunks_per_split, nchunk_total);
+    const int nch = c_end - c_begin;
+    const int kb_begin = c_begin * kFxBPC;
+    const int nbs = min(nch * kFxBPC, p.nb - kb_begin);
+
+    // shared memory: [x pairs][barriers][ring]
+    const int x_bytes = (B * nbs * kXBlockPitch + 127) & ~127;
+    uint8_t *xs = smem;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + x_bytes);
+    const int bar_bytes = (nwarps * p.depth * 8 + 127) & ~127;
+    const uint32_t ring_pad = (128u - ((smem_u32(smem) + x_bytes + bar_bytes) & 127u)) & 127u;
+    uint8_t *ring = smem + x_bytes + bar_bytes + ring_pad;
+    uint8_t *my_ring = ring + static_cast<size_t>(warp) * p.depth * kFxSlotBytes;
+    const uint32_t my_ring_s = smem_u32(my_ring);
+    const uint32_t my_bars_s = smem_u32(bars + warp * p.depth);
+
+    const long long tstride = static_cast<long long>(p.ctas_per_split) * nwarps;
+    const long long t0 = static_cast<long long>(warp) * p.ctas_per_split + cj;
+    const long long ntiles_w = (t0 < p.tiles) ? (p.tiles - t0 + tstride - 1) / tstride : 0;
+    const long long total = ntiles_w * NS * nch;
+    const long long row_step = tstride * kFxTileRows;
+
+    Cursor pc{t0 * kFxTileRows, 0, 0};
+    long long issued = 0;
+    if (lane == 0) {
+        for (int s = 0; s < p.depth; ++s)
+            mbar_init(my_bars_s + s * 8, 1);
+        mbar_fence_init();
+    }
+    __syncwarp();
+    pdl_wait();
+    pdl_launch_dependents();
+    for (int s = 0; s < p.depth && issued < total; ++s, ++issued) {
+        fx_issue_slot<TMA>(p, maps, pc, s, c_begin, my_ring_s, my_bars_s, lane);
+        pc.advance(nch, NS, row_step);
+    }
+
+    stage_x_pairs<(B <= 2) ? 4 : 1>(p.x, p.K, B, kb_begin, nbs, xs);
+    __syncthreads();
+
+    bool failed = false;
+    long long consumed = 0;
+    float2 acc0[R][B], acc1[R][B];
+    float gsum[NS == 2 ? VPL : 1];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+            acc0[r][b] = f2(0.f, 0.f);
+            acc1[r][b] = f2(0.f, 0.f);
+        }
+
+    Cursor cc{t0 * kFxTileRows, 0, 0};
+    int slot = 0;
+    uint32_t parity = 0;
+    for (; consumed < total; ++consumed) {
+        const bool ok = mbar_wait_bounded(my_bars_s + slot * 8, parity, p.err);
+        if (!__all_sync(0xffffffffu, ok)) {
+            failed = true;
+            break;
+        }
+        const int kb0 = (c_begin + cc.kcl) * kFxBPC;
+        const int nblk = min(kFxBPC, p.nb - kb0);
+        if (g < nblk) {
+            const uint8_t *slot_p = my_ring + slot * kFxSlotBytes + i * kFxRowPitch;
+            const BlockOffsets bo = block_offsets<SOA>(g, nblk);
+            Hdr hd[R];
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+                hd[r] = decode_hdr(*reinterpret_cast<const uint4 *>(slot_p + 8 * r * kFxRowPitch + bo.hdr));
+            const uint8_t *xblk = xs + (kb0 - kb_begin + g) * kXBlockPitch;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                ChunkScales cs[R];
+#pragma unroll
+                for (int r = 0; r < R; ++r)
+                    cs[r] = chunk_scales(hd[r], c);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int s = 2 * c + h;  // 16-byte quant slice
+                    uint4 q[R];
+#pragma unroll
+                    for (int r = 0; r < R; ++r)
+                        q[r] = *reinterpret_cast<const uint4 *>(slot_p + 8 * r * kFxRowPitch + bo.qs0 +
+                                                                s * bo.qs_step);
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+#pragma unroll
+                        for (int b = 0; b < B; ++b) {
+                            const uint8_t *xq = xblk + b * nbs * kXBlockPitch + s * 128 + 32 * t;
+                            const float4 xa = *reinterpret_cast<const float4 *>(xq);
+                            const float4 xb = *reinterpret_cast<const float4 *>(xq + 16);
+#pragma unroll
+                            for (int r = 0; r < R; ++r) {
+                                const uint32_t wv = (t == 0) ? q[r].x : (t == 1) ? q[r].y : (t == 2) ? q[r].z : q[r].w;
+                                q4_word(wv, cs[r], xa, xb, acc0[r][b], acc1[r][b]);
+                            }
+                        }
+                    }
+                }
+            }
+        }
+
+        __syncwarp();
+        if (issued < total) {
+            fence_proxy_async_smem();
+            fx_issue_slot<TMA>(p, maps, pc, slot, c_begin, my_ring_s, my_bars_s, lane);
+            pc.advance(nch, NS, row_step);
+            ++issued;
+        }
+
+        const int cur_st = cc.st;
+        const long long row0 = cc.row0;
+        const bool last_chunk = (cc.kcl == nch - 1);
+        cc.advance(nch, NS, row_step);
+        if (++slot == p.depth) {
+            slot = 0;
+            parity ^= 1u;
+        }
+        if (!last_chunk)
+            continue;
+
+        // end of this stream's K range for the tile: add the four quarters' sums
+        float v[MP];
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int b = 0; b < B; ++b) {
+                const float2 a = __fadd2_rn(acc0[r][b], acc1[r][b]);
+                v[r * B + b] = a.x + a.y;
+                acc0[r][b] = f2(0.f, 0.f);
+                acc1[r][b] = f2(0.f, 0.f);
+            }
+#pragma unroll
+        for (int k = MV; k < MP; ++k)
+            v[k] = 0.f;
+        quarter_sum<MP>(v, lane);
+        if constexpr (NS == 2) {
+            if (cur_st == 0) {
+#pragma unroll
+                for (int k = 0; k < VPL; ++k)
+                    gsum[k] = v[k];
+                continue;
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < VPL; ++k) {
+            const int idx = voff + k;
+            if (idx >= MV)
+                continue;
+            const int r = idx / B;
+            const int b = idx % B;
+            const long long n = row0 + i + 8 * r;
+            if (n >= p.N)
+                continue;
+            if (p.splits > 1) {
+                if constexpr (NS == 2) {
+                    p.part[((static_cast<long long>(split) * 2 + 0) * B + b) * p.N + n] = gsum[k] * 0x1p64f;
+                    p.part[((static_cast<long long>(split) * 2 + 1) * B + b) * p.N + n] = v[k] * 0x1p64f;
+                } else {
+                    p.part[(static_cast<long long>(split) * B + b) * p.N + n] = v[k] * 0x1p64f;
+                }
+            } else {
+                float out;
+                if constexpr (NS == 2) {
+                    const float gv = gsum[k] * 0x1p64f;
+                    out = gv / (1.0f + expf(-gv)) * (v[k] * 0x1p64f);
+                } else {
+                    out = v[k] * 0x1p64f;
+                }
+                *gemv_out_addr(p.y, p.g, p.qg_hd, p.N, b, n) = out;
+            }
+        }
+    }
+
+    if (failed) {
+        // the copies already issued into this warp's ring must land before the CTA exits
+        for (long long k = consumed; k < issued; ++k) {
+            mbar_wait_bounded(my_bars_s + slot * 8, parity, nullptr);
+            if (++slot == p.depth) {
+                slot = 0;
+                parity ^= 1u;
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 
@@ -619,7 +863,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 // chunk), warps per CTA follow from the tasks per SM, and K is split further
 // if the activations would not fit beside a two-deep ring per warp; the ring
 // is as deep as shared memory allows, up to 4 slots.
-Q4KPlan q4k_plan_fx(long long N, int nb, int NS, int sm_count, int smem_optin)
+Q4KPlan q4k_plan_fx(long long N, int nb, int B, int NS, int sm_count, int smem_optin)
 {
     Q4KPlan pl{};
     // DQGEMV_NO_TMA=1 selects the per-row bulk copies (same shared-memory
@@ -627,13 +871,16 @@ Q4KPlan q4k_plan_fx(long long N, int nb, int NS, int sm_count, int smem_optin)
     const char *no_tma = getenv("DQGEMV_NO_TMA");
     const bool tma = N < 0x7FFFFFFFLL && tensor_map_encoder() != nullptr && !(no_tma && no_tma[0] == '1');
     const int misc = 256 /*argmax scratch, 16 B per warp*/ + 512 /*barriers*/ + 128 /*ring alignment*/;
-    const int stage = kFxLimbPitch + kFxAuxPitch;
+    // staged activations per super-block: limb planes and sums (batch 1), or B
+    // rows of fp32 pairs
+    const int stage = (B == 1) ? kFxLimbPitch + kFxAuxPitch : B * kXBlockPitch;
+    const int max_warps = (B == 1) ? kFxMaxWarps : kFxbMaxWarps(B);
     const long long tiles = (N + kFxTileRows - 1) / kFxTileRows;
     const int nchunk = (nb + kFxBPC - 1) / kFxBPC;
     int splits_par = 1;
     while (tiles * splits_par < 8LL * sm_count && splits_par < nchunk)
         ++splits_par;
-    const int w0 = q4k_pick_warps(tiles * splits_par, sm_count, kFxMaxWarps);
+    const int w0 = q4k_pick_warps(tiles * splits_par, sm_count, max_warps);
     for (int warps = w0; warps >= 4 && !pl.ok; --warps) {
         int splits = splits_par;
         int cps = (nchunk + splits - 1) / splits;
@@ -664,8 +911,8 @@ Q4KPlan q4k_plan_fx(long long N, int nb, int NS, int sm_count, int smem_optin)
         pl.ctas_per_split = static_cast<int>(ctas);
         pl.grid = pl.ctas_per_split * splits;
         pl.smem = x_bytes + ((warps * depth * 8 + 127) & ~127) + 128 + warps * depth * kFxSlotBytes + 256;
-        // splits of at most one tile per warp are added inside a cluster
-        pl.cluster = splits > 1 && splits <= kFxMaxCluster &&
+        // batch-1 splits of at most one tile per warp are added inside a cluster
+        pl.cluster = B == 1 && splits > 1 && splits <= kFxMaxCluster &&
                      tiles <= static_cast<long long>(pl.ctas_per_split) * warps &&
                      pl.smem + warps * kFxClusterPartBytes <= smem_optin;
         if (pl.cluster)
@@ -716,7 +963,33 @@ static cudaError_t launch_fx(const Q4KParams &p, const FxMaps &maps, const Q4KPl
     return cudaLaunchKernelEx(&cfg, k, p, maps);
 }
 
-cudaError_t q4k_gemv_fx_launch(const Q4KParams &p, const Q4KPlan &pl, int NS, cudaStream_t s)
+template <int B, int NS, bool TMA>
+static cudaError_t launch_fxb(const Q4KParams &p, const FxMaps &maps, const Q4KPlan &pl, cudaStream_t s)
+{
+    auto k = p.soa ? q4k_gemv_fxb_kernel<B, NS, true, TMA> : q4k_gemv_fxb_kernel<B, NS, false, TMA>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
+    if (e != cudaSuccess)
+        return e;
+    return launch_pdl(k, dim3(pl.grid), dim3(pl.warps * 32), pl.smem, s, p, maps);
+}
+
+template <int NS, bool TMA>
+static cudaError_t launch_fx_b(const Q4KParams &p, const FxMaps &maps, const Q4KPlan &pl, int B, cudaStream_t s)
+{
+    switch (B) {
+    case 1: return launch_fx<NS, TMA>(p, maps, pl, s);
+    case 2: return launch_fxb<2, NS, TMA>(p, maps, pl, s);
+    case 3: return launch_fxb<3, NS, TMA>(p, maps, pl, s);
+    case 4: return launch_fxb<4, NS, TMA>(p, maps, pl, s);
+    case 5: return launch_fxb<5, NS, TMA>(p, maps, pl, s);
+    case 6: return launch_fxb<6, NS, TMA>(p, maps, pl, s);
+    case 7: return launch_fxb<7, NS, TMA>(p, maps, pl, s);
+    case 8: return launch_fxb<8, NS, TMA>(p, maps, pl, s);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t q4k_gemv_fx_launch(const Q4KParams &p, const Q4KPlan &pl, int B, int NS, cudaStream_t s)
 {
     FxMaps maps;
     memset(&maps, 0, sizeof(maps));
@@ -734,9 +1007,9 @@ cudaError_t q4k_gemv_fx_launch(const Q4KParams &p, const Q4KPlan &pl, int NS, cu
                     return e;
             }
         }
-        return NS == 1 ? launch_fx<1, true>(p, maps, pl, s) : launch_fx<2, true>(p, maps, pl, s);
+        return NS == 1 ? launch_fx_b<1, true>(p, maps, pl, B, s) : launch_fx_b<2, true>(p, maps, pl, B, s);
     }
-    return NS == 1 ? launch_fx<1, false>(p, maps, pl, s) : launch_fx<2, false>(p, maps, pl, s);
+    return NS == 1 ? launch_fx_b<1, false>(p, maps, pl, B, s) : launch_fx_b<2, false>(p, maps, pl, B, s);
 }
 
 }  // namespace dq
