@@ -55,7 +55,7 @@ NCU_TRAFFIC = {"sources_sha1": "d2937bcf73647018c79c1b6fabef0f0a4d3ddd0b",
 
 def kernel_sources_sha1() -> str:
     h = hashlib.sha1()
-    for f in ("q4k_gemv_fx.cu", "q4k_stream.cuh", "dq_common.cuh"):
+    for f in ("q4k_gemv.cu", "q4k_stream.cuh", "dq_common.cuh"):
         with open(os.path.join(ROOT, "dequant_gemv_q4_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()

@@ -107,7 +107,7 @@ dq_status q4k_common(const void *w0, const void *w1, int layout, const float *x,
         return st;
     const dq::Q4KPlan pl = dq::q4k_plan(N, static_cast<int>(K), B, NS, layout == DQ_LAYOUT_SOA, di.sm_count,
                                         di.smem_optin);
-    if (!pl.ok || (grp && !pl.fx))
+    if (!pl.ok)
         return DQ_ERR_SHAPE;
     const Q4KWorkspace ws = q4k_ws(pl, N, B, NS, argmax_out != nullptr);
     if (ws.total() > 0 && (!workspace || ws_bytes < ws.total()))

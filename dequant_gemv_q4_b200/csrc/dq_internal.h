@@ -49,11 +49,8 @@ struct Q4KParams {
 
 struct Q4KPlan {
     bool ok;
-    bool half;             // batch-1 half-block kernel (q4k_gemv_b1_kernel)
-    bool fx;               // quarter-warp kernels: q4k_gemv_fx_kernel (B = 1), q4k_gemv_fxb_kernel (B = 2..8)
-    bool tma;              // fx kernel: slots moved by TMA tile copies
-    bool cluster;          // fx kernel: K splits reduced in-kernel across a CTA cluster (no workspace)
-    int lpr;               // lanes per row group (4, 8, 16 or 32)
+    bool tma;              // slots moved by TMA tile copies (else one bulk copy per row)
+    bool cluster;          // batch 1: K splits reduced in-kernel across a CTA cluster (no workspace)
     int R;                 // rows per lane
     int warps;             // warps per CTA
     long long tiles;
@@ -67,10 +64,7 @@ struct Q4KPlan {
 
 Q4KPlan q4k_plan(long long N, int K, int B, int NS, int soa, int sm_count, int smem_optin);
 cudaError_t q4k_gemv_launch(const Q4KParams &p, const Q4KPlan &pl, int B, int NS, cudaStream_t s);
-int q4k_pick_warps(long long tiles, int sm_count, int max_warps, bool round4 = false);
-Q4KPlan q4k_plan_fx(long long N, int nb, int B, int NS, int sm_count, int smem_optin);
 int q4k_fx_tile_rows();
-cudaError_t q4k_gemv_fx_launch(const Q4KParams &p, const Q4KPlan &pl, int B, int NS, cudaStream_t s);
 
 // Q8_0 GEMV
 struct Q8Params {

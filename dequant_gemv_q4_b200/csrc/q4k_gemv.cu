@@ -1,38 +1,65 @@
-// q4k_gemv.cu -- fused Q4_K dequantize + GEMV (plain, fused SwiGLU, B <= 8,
-// optional argmax) for sm_100a.
+// q4k_gemv.cu -- fused Q4_K dequantize + GEMV for sm_100a: plain, fused
+// SwiGLU, Q/gate split, grouped matrices and argmax at batch 1
+// (q4k_gemv_fx_kernel: integer dot products on fixed-point activations), and
+// batches of 2..8 (q4k_gemv_fxb_kernel: exact fp32 weights).
 //
 // The operation is the pages' fused dequant+GEMV over raw Q4_K bytes (trueno
 // WgslForwardPass: upload_q4k_weight; qualiaDB cuda_lane: try_q4k_soa_gemv,
-// try_q4k_soa_fused_swiglu).  The kernel design below is this library's own.
+// try_q4k_soa_fused_swiglu).  The arithmetic below is this library's own.
 //
-// Work decomposition
-//   A warp owns a set of row tiles.  A row tile is TR = (32/LPR)*R rows; lane
-//   (rg, l) = (lane / LPR, lane % LPR) handles rows rg*R .. rg*R+R-1 of the
-//   tile and, in every K-chunk of LPR super-blocks, super-block l of each of
-//   those rows.  One "slot" is one K-chunk of one tile of one weight stream
-//   (TR rows x LPR super-blocks, 9 KB for R = 2).  Each warp streams its own
-//   ring of `depth` slots: lane 0 issues 1-D bulk copies (cp.async.bulk from
-//   this GPU's global memory into the warp's shared-memory slot, completing on
-//   an mbarrier), the whole warp computes on the oldest slot and lane 0 reuses
-//   it for the slot `depth` steps ahead.  CTAs are persistent: a grid of about
-//   one CTA per SM walks all tiles.  K may be split across CTAs (split-K) when
-//   the activations of all of K do not fit in shared memory or when there are
-//   too few row tiles to occupy the GPU; split partial sums go to the caller's
-//   workspace and a second kernel reduces them in a fixed order.
+// Why integers.  At batch 1 every weight is used once, so the cost per weight
+// is what bounds the kernel.  Forming each fp32 weight (an AND to isolate the
+// quant, an fma with scale and min) and then an fma with x costs three
+// instructions per weight on two half-rate pipes.  Here four quants at a time
+// are unpacked into bytes (one AND for the four low nibbles of a word, one AND
+// for the four high nibbles, left in place as 16 q) and multiplied against four
+// bytes of x by one dp4a (four 8-bit products summed into an int32).
 //
-// Arithmetic (per weight, no factoring of scales or mins)
-//   A quant q at bit position p of a 32-bit word, isolated with one AND, is
-//   the fp32 bit pattern q*2^p, i.e. the subnormal (or smallest-normal) value
-//   q*2^(p-149).  One fma with d*scale*2^(85-p) and -dmin*min*2^-64 then gives
-//   (d*scale*q - dmin*min) * 2^-64 rounded once: exactly the fp32 weight that
-//   q4k_dequant returns, times 2^-64 (all operands are exact: d has 11
-//   significant bits, scale and min 6, q 4).  A second fma accumulates
-//   weight*x.  Sums are taken in units of 2^-64 and scaled back at the end, so
-//   any finite fp32 x is accepted.  Both fmas run as fma.rn.f32x2 on pairs.
-//   Subnormal operands are kept (the library is built without flush-to-zero).
+// Arithmetic.
+//   x, per super-block sb of 256 activations: with e the exponent of the
+//   largest |x_k| (2^e <= max < 2^(e+1)) and F = 29 - e, xi_k = round(x_k 2^F),
+//   so |xi_k| < 2^30 and |x_k - xi_k 2^-F| <= 2^(e-30).  xi is split into four
+//   signed bytes (signed digits) xi = l0 + 2^8 l1 + 2^16 l2 + 2^24 l3.  X_j is
+//   the exact sum of xi over sub-block j.
+//   Per row and sub-block j: A_l = sum_k q_k l_{l,k} (dp4a, exact), folded as
+//   I_l += scale_j * A_l (exact, |I_l| < 2^25; kept as 16 I_l < 2^29 because
+//   the high nibbles enter dp4a as 16 q).  Per row and super-block, in
+//   fp64: I_s = sum_l 2^(8l) I_l (exact, < 2^49), I_m = sum_j min_j X_j (exact,
+//   < 2^44) and y_sb = 2^-F (d I_s - dmin I_m), evaluated with an error-free
+//   product so that the rounding is relative to y_sb itself, even when the
+//   scale and min terms cancel.  Row sums stay in fp64 and are rounded to fp32
+//   once.
+//   So the result is sum_k w_k xi_k 2^-F to fp64 accuracy; the only
+//   approximation is the rounding of x:
+//     |y - sum_k w_k x_k| <= sum_sb 2^(e_sb - 30) sum_{k in sb} |w_k|,
+//   i.e. 2^-30 of the largest activation of each super-block.
+//   A super-block of x holding an infinity or a NaN makes the rows' results NaN.
+//
+// Work decomposition ("quarter-warp lanes").  A K-chunk is 4 super-blocks (one
+// SoA group, 576 contiguous bytes of a row in both layouts).  Lane (g, i) =
+// (lane / 8, lane % 8) handles super-block g of each chunk for rows i + 8r
+// (r < R) of a row tile of 8R rows, so the eight lanes of a quarter-warp read
+// the same activation bytes (a shared-memory broadcast) and distinct rows'
+// quants.  A slot is one chunk of one tile, 8R rows x 576 bytes.  Each warp
+// streams its own ring of slots; the four quarter sums of a row are added with
+// two shuffles.
+//
+// Slot copies.  Slot rows sit at a 592-byte pitch (576 + 16), which places the
+// eight rows a quarter-warp reads at one time in eight distinct bank groups.
+// One TMA tile copy moves a slot: the matrix is described to the TMA unit as
+// [N rows][row bytes / 4] 32-bit words and a box of 16 rows x 148 words is
+// copied, i.e. each row's chunk plus the next 16 bytes of that row (zeros past
+// its end), so the box itself lays the rows out at the padded pitch.  Without
+// the driver's tensor-map encoder each row is its own 1-D bulk copy instead.
 
+#include <cooperative_groups.h>
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_fp16.h>
 #include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
 
 #include "dq_common.cuh"
 #include "dq_internal.h"
@@ -41,106 +68,284 @@
 
 namespace dq {
 
-template <int LPR, int B, int NS, bool SOA>
-__global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_kernel(const Q4KParams p)
+// Staged activations of one super-block: four limb planes of 256 bytes (plane
+// l, byte k = limb l of xi_k) and 16 bytes of padding, which shifts the bank
+// group from one super-block to the next; then, in a separate array, X_0..X_7
+// and 2^-F as fp64 (80-byte pitch).  The lanes of a quarter-warp read the same
+// super-block, so these reads are broadcasts.
+constexpr int kFxLimbPitch = 1040;
+constexpr int kFxAuxPitch = 80;
+
+constexpr int kFxRows = 2;                     // rows per lane (R)
+constexpr int kFxBPC = 4;                      // super-blocks per K-chunk
+constexpr int kFxChunkBytes = kFxBPC * kQ4KBlockBytes;   // 576
+constexpr int kFxTileRows = 8 * kFxRows;
+constexpr int kFxRowPitch = kFxChunkBytes + 16;           // 592
+constexpr int kFxSlotBytes = kFxTileRows * kFxRowPitch;
+static_assert(kFxSlotBytes % 128 == 0, "slots must keep the ring 128-byte aligned");
+constexpr int kFxMaxWarps = 12;
+int q4k_fx_tile_rows() { return kFxTileRows; }
+// In-cluster split reduction: per warp and stream, the 16 row partials (fp64).
+constexpr int kFxClusterPartBytes = 2 * kFxTileRows * 8;
+constexpr int kFxMaxCluster = 8;
+
+// TMA descriptors of the weight matrices: SwiGLU's gate and up, or one per
+// matrix of a grouped GEMV.
+struct FxMaps {
+    CUtensorMap m[kMaxGroup];
+};
+
+// Converts the activations of super-blocks kb_begin .. kb_begin + nbs - 1 into
+// limb planes and sums; one warp per super-block.
+__device__ __forceinline__ void fx_stage(const float *x, int kb_begin, int nbs, uint8_t *limbs, uint8_t *aux,
+                                         int warp, int nwarps, int lane)
 {
-    pdl_wait();
-    pdl_launch_dependents();
-    constexpr int R = 2;
-    using G = Geo<LPR, R>;
-    constexpr int MV = R * B;                         // values per lane per stream
-    constexpr int MP = Pow2Ceil<MV>::value;           // padded to a power of two
-    constexpr int VPL = (MP > LPR) ? MP / LPR : 1;    // values per lane after reduce
+    for (int sb = warp; sb < nbs; sb += nwarps) {
+        const float *xg = x + static_cast<long long>(kb_begin + sb) * 256 + lane * 8;
+        const float4 a = __ldg(reinterpret_cast<const float4 *>(xg));
+        const float4 b = __ldg(reinterpret_cast<const float4 *>(xg + 4));
+        const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        uint32_t m = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            m = max(m, __float_as_uint(v[i]) & 0x7FFFFFFFu);
+        m = __reduce_max_sync(0xffffffffu, m);   // |x| bit patterns order like the values
+        const bool finite = m < 0x7F800000u;
+        int e = 0;
+        if (m >= 0x00800000u)
+            e = static_cast<int>(m >> 23) - 127;
+        else if (m != 0)
+            e = (31 - __clz(static_cast<int>(m))) - 149;
+        const int F = 29 - e;                  // in [-98, 178]
+        const int F1 = F / 2, F2 = F - F1;     // each in [-49, 89]: normal powers of two
+        const float p1 = __int_as_float((127 + F1) << 23);
+        const float p2 = __int_as_float((127 + F2) << 23);
+
+        uint32_t w[4][2] = {};
+        double part = 0.0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            // x * 2^F is exact wherever it is >= 1/2 in magnitude (two power-of-two
+            // products with normal results); smaller values round to 0 either way
+            int t = finite ? __float2int_rn((v[i] * p1) * p2) : 0;
+            part += static_cast<double>(t);
+            // signed digits: the stored byte is t's low byte, the carry rounds t / 256
+#pragma unroll
+            for (int l = 0; l < 4; ++l) {
+                w[l][i >> 2] |= (static_cast<uint32_t>(t) & 0xFFu) << (8 * (i & 3));
+                t = (t + 128) >> 8;
+            }
+        }
+        uint8_t *lp = limbs + sb * kFxLimbPitch + lane * 8;
+#pragma unroll
+        for (int l = 0; l < 4; ++l)
+            *reinterpret_cast<uint2 *>(lp + 256 * l) = make_uint2(w[l][0], w[l][1]);
+        // sub-block j = lanes 4j .. 4j+3; sums of at most 32 values below 2^30 are exact
+        part += __shfl_xor_sync(0xffffffffu, part, 1);
+        part += __shfl_xor_sync(0xffffffffu, part, 2);
+        double *ap = reinterpret_cast<double *>(aux + sb * kFxAuxPitch);
+        if ((lane & 3) == 0)
+            ap[lane >> 2] = part;
+        if (lane == 0)
+            ap[8] = finite ? __longlong_as_double(static_cast<long long>(1023 - F) << 52)
+                           : __longlong_as_double(0x7FF8000000000000LL);
+    }
+}
+
+// dp4a with unsigned bytes in a (quants) and signed bytes in b (activation limbs).
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c)
+{
+    int d;
+    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// One 16-byte quant slice of R rows against the limb planes: lo (low nibbles,
+// sub-block 2c) and hi (high nibbles, sub-block 2c+1) sums per limb.  The high
+// nibbles are used in place, as the bytes 16*q (one AND), so the hi sums are
+// 16 times the sub-block sums.
+template <int R>
+__device__ __forceinline__ void fx_slice(const uint4 (&q)[R], const uint8_t *xlo, const uint8_t *xhi, int (&alo)[R][4],
+                                         int (&ahi)[R][4])
+{
+    uint4 xa[4], xb[4];
+#pragma unroll
+    for (int l = 0; l < 4; ++l) {
+        xa[l] = *reinterpret_cast<const uint4 *>(xlo + 256 * l);
+        xb[l] = *reinterpret_cast<const uint4 *>(xhi + 256 * l);
+    }
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const uint32_t w = (t == 0) ? q[r].x : (t == 1) ? q[r].y : (t == 2) ? q[r].z : q[r].w;
+            const uint32_t lo = w & 0x0F0F0F0Fu;
+            const uint32_t hi16 = w & 0xF0F0F0F0u;
+#pragma unroll
+            for (int l = 0; l < 4; ++l) {
+                const uint32_t x0 = (t == 0) ? xa[l].x : (t == 1) ? xa[l].y : (t == 2) ? xa[l].z : xa[l].w;
+                const uint32_t x1 = (t == 0) ? xb[l].x : (t == 1) ? xb[l].y : (t == 2) ? xb[l].z : xb[l].w;
+                alo[r][l] = dp4a_us(lo, x0, alo[r][l]);
+                ahi[r][l] = dp4a_us(hi16, x1, ahi[r][l]);
+            }
+        }
+    }
+}
+
+// The matrix a slot reads and its rows: SwiGLU stream st of the same rows, or,
+// for a grouped GEMV, the matrix holding padded row row0 and the row there.
+struct FxRows {
+    int sel;
+    long long row0;
+    long long nrows;
+};
+__device__ __forceinline__ FxRows fx_rows(const Q4KParams &p, int st, long long row0)
+{
+    if (p.grp.n == 0)
+        return {st, row0, p.N};
+    int m = 0;
+#pragma unroll
+    for (int k = 1; k < kMaxGroup; ++k)
+        if (k < p.grp.n && row0 >= p.grp.base[k])
+            m = k;
+    const long long base = m == 0 ? p.grp.base[0] : m == 1 ? p.grp.base[1] : m == 2 ? p.grp.base[2] : p.grp.base[3];
+    const long long rows = m == 0 ? p.grp.N[0] : m == 1 ? p.grp.N[1] : m == 2 ? p.grp.N[2] : p.grp.N[3];
+    return {m, row0 - base, rows};
+}
+__device__ __forceinline__ const uint8_t *fx_weights(const Q4KParams &p, int sel)
+{
+    if (p.grp.n == 0)
+        return sel == 0 ? p.w[0] : p.w[1];
+    return sel == 0 ? p.gw[0] : sel == 1 ? p.gw[1] : sel == 2 ? p.gw[2] : p.gw[3];
+}
+__device__ __forceinline__ float *fx_group_out(const Q4KParams &p, int sel)
+{
+    return sel == 0 ? p.grp.y[0] : sel == 1 ? p.grp.y[1] : sel == 2 ? p.grp.y[2] : p.grp.y[3];
+}
+
+// Issues the copies of one slot (K-chunk c_begin + cur.kcl of stream cur.st of
+// the tile at cur.row0).  TMA: lane 0 arms the slot's mbarrier and issues one
+// tile copy (elements past the matrix are filled with zeros and still counted).
+// Otherwise lane 0 arms the mbarrier with the slot's byte count and lane r
+// copies row r.
+template <bool TMA>
+__device__ __forceinline__ void fx_issue_slot(const Q4KParams &p, const FxMaps &maps, const Cursor &cur, int slot,
+                                              int c_begin, uint32_t ring_s, uint32_t bars_s, int lane)
+{
+    const int kb0 = (c_begin + cur.kcl) * kFxBPC;
+    const uint32_t bar = bars_s + slot * 8;
+    const uint32_t dst = ring_s + slot * kFxSlotBytes;
+    const FxRows fr = fx_rows(p, cur.st, cur.row0);
+    if constexpr (TMA) {
+        if (lane == 0) {
+            mbar_arrive_expect_tx(bar, static_cast<uint32_t>(kFxSlotBytes));
+            const CUtensorMap *m = fr.sel == 0 ? &maps.m[0] : fr.sel == 1 ? &maps.m[1] : fr.sel == 2 ? &maps.m[2]
+                                                                                                      : &maps.m[3];
+            // x = kb0 * 36 words: a multiple of 4 words, i.e. of 16 bytes
+            asm volatile(
+                "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+                "[%4];" ::"r"(dst),
+                "l"(m), "r"(kb0 * (kQ4KBlockBytes / 4)), "r"(static_cast<int>(fr.row0)), "r"(bar)
+                : "memory");
+        }
+    } else {
+        const long long row_bytes_g = static_cast<long long>(p.nb) * kQ4KBlockBytes;
+        const int rows = static_cast<int>(min(static_cast<long long>(kFxTileRows), fr.nrows - fr.row0));
+        const int nblk = min(kFxBPC, p.nb - kb0);
+        const uint32_t bytes = static_cast<uint32_t>(nblk * kQ4KBlockBytes);
+        if (lane == 0)
+            mbar_arrive_expect_tx(bar, static_cast<uint32_t>(rows) * bytes);
+        __syncwarp();
+        if (lane < rows) {
+            const uint8_t *src = fx_weights(p, fr.sel) + (fr.row0 + lane) * row_bytes_g +
+                                 static_cast<long long>(kb0) * kQ4KBlockBytes;
+            bulk_g2s(dst + lane * kFxRowPitch, src, bytes, bar);
+        }
+    }
+}
+
+template <int NS, bool SOA, bool TMA>
+__global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
+    q4k_gemv_fx_kernel(const __grid_constant__ Q4KParams p, const __grid_constant__ FxMaps maps)
+{
+    constexpr int R = kFxRows;
+    static_assert(R == 2, "the quarter reduction below is written for two rows per lane");
 
     extern __shared__ __align__(128) uint8_t smem[];
     const int nwarps = blockDim.x >> 5;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int rg = lane / LPR;
-    const int l = lane % LPR;
+    const int g = lane >> 3;   // super-block of each chunk
+    const int i = lane & 7;    // rows i and i + 8 of each tile
 
-    const int split = blockIdx.x / p.ctas_per_split;
-    const int cj = blockIdx.x % p.ctas_per_split;
-    const int nchunk_total = (p.nb + LPR - 1) / LPR;
+    // the splits of one CTA column are consecutive blocks (one cluster when the
+    // splits are reduced in-kernel)
+    const int split = blockIdx.x % p.splits;
+    const int cj = blockIdx.x / p.splits;
+    const int nchunk_total = (p.nb + kFxBPC - 1) / kFxBPC;
     const int c_begin = split * p.chunks_per_split;
     const int c_end = min(c_begin + p.chunks_per_split, nchunk_total);
     const int nch = c_end - c_begin;
-    const int kb_begin = c_begin * LPR;
-    const int nbs = min(nch * LPR, p.nb - kb_begin);  // super-blocks of this split
+    const int kb_begin = c_begin * kFxBPC;
+    const int nbs = min(nch * kFxBPC, p.nb - kb_begin);  // super-blocks of this split
 
-    // shared memory: [x staging][barriers][ring][argmax scratch]
-    const int x_bytes = (B * nbs * kXBlockPitch + 127) & ~127;
-    uint8_t *xs = smem;
+    // shared memory: [limb planes][sums and scales][barriers][ring][argmax scratch]
+    const int x_bytes = (nbs * (kFxLimbPitch + kFxAuxPitch) + 127) & ~127;
+    uint8_t *limbs = smem;
+    uint8_t *aux = smem + nbs * kFxLimbPitch;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + x_bytes);
     const int bar_bytes = (nwarps * p.depth * 8 + 127) & ~127;
-    uint8_t *ring = smem + x_bytes + bar_bytes;
-    uint8_t *my_ring = ring + static_cast<size_t>(warp) * p.depth * G::SLOT_BYTES;
+    // TMA writes shared memory at 128-byte aligned addresses: align the ring
+    const uint32_t ring_pad = (128u - ((smem_u32(smem) + x_bytes + bar_bytes) & 127u)) & 127u;
+    uint8_t *ring = smem + x_bytes + bar_bytes + ring_pad;
+    uint8_t *my_ring = ring + static_cast<size_t>(warp) * p.depth * kFxSlotBytes;
     const uint32_t my_ring_s = smem_u32(my_ring);
     const uint32_t my_bars_s = smem_u32(bars + warp * p.depth);
-    ArgmaxCand *red = reinterpret_cast<ArgmaxCand *>(ring + static_cast<size_t>(nwarps) * p.depth * G::SLOT_BYTES);
+    ArgmaxCand *red = reinterpret_cast<ArgmaxCand *>(ring + static_cast<size_t>(nwarps) * p.depth * kFxSlotBytes);
+    double *cpart = reinterpret_cast<double *>(reinterpret_cast<uint8_t *>(red) + 256);
 
-    // this warp's tiles: t0, t0 + tstride, ...
+    // this warp's tiles: t0, t0 + tstride, ... (warp-major order)
     const long long tstride = static_cast<long long>(p.ctas_per_split) * nwarps;
-    // warp-major tile order: the last, partial round of tiles spreads over all SMs
     const long long t0 = static_cast<long long>(warp) * p.ctas_per_split + cj;
     const long long ntiles_w = (t0 < p.tiles) ? (p.tiles - t0 + tstride - 1) / tstride : 0;
     const long long total = ntiles_w * NS * nch;
-    const long long row_step = tstride * G::TR;
+    const long long row_step = tstride * kFxTileRows;
 
-    // After the row-group reduction this lane holds value indices
-    // off .. off + VPL - 1 (value index = r * B + b); only `writer` lanes store.
-    int off = 0;
-    bool writer = true;
-    {
-        int m = MP;
-#pragma unroll
-        for (int o = LPR / 2; o >= 1; o >>= 1) {
-            if (m > 1) {
-                if (l & o)
-                    off += m / 2;
-                m /= 2;
-            } else if (l & o) {
-                writer = false;
-            }
-        }
-    }
+    // after the quarter reduction lanes of quarters 0, 1 hold row i and
+    // quarters 2, 3 row i + 8; quarters 0 and 2 store
+    const bool writer = (lane & 8) == 0;
+    const int wrow = i + ((lane & 16) ? 8 : 0);
 
-    // producer cursor (used by lane 0, advanced in every lane)
-    Cursor pc{t0 * G::TR, 0, 0};
+    Cursor pc{t0 * kFxTileRows, 0, 0};
     long long issued = 0;
     if (lane == 0) {
         for (int s = 0; s < p.depth; ++s)
             mbar_init(my_bars_s + s * 8, 1);
         mbar_fence_init();
     }
+    __syncwarp();
+    // the weights too may come from the previous kernel (a repack, an upload)
+    pdl_wait();
+    pdl_launch_dependents();
     for (int s = 0; s < p.depth && issued < total; ++s, ++issued) {
-        if (lane == 0)
-            issue_slot<G>(p, pc, s, c_begin, my_ring_s, my_bars_s);
+        fx_issue_slot<TMA>(p, maps, pc, s, c_begin, my_ring_s, my_bars_s, lane);
         pc.advance(nch, NS, row_step);
     }
 
-    // stage this split's activations in (lo, hi) pairs (fp32, padded per super-block);
-    // each thread keeps 8 loads in flight before storing (one at a time for
-    // large B, whose kernels have no registers to spare)
-    stage_x_pairs<(B <= 2) ? 8 : 1>(p.x, p.K, B, kb_begin, nbs, xs);
+    fx_stage(p.x, kb_begin, nbs, limbs, aux, warp, nwarps, lane);
     __syncthreads();
 
     float best_v = -INFINITY;
     long long best_i = 0x7fffffffffffffffLL;
     bool failed = false;
     long long consumed = 0;
-
-    float2 acc0[R][B], acc1[R][B];
-    float gsum[NS == 2 ? VPL : 1];  // stream-0 sums kept for the SwiGLU epilogue
+    double acc[R];
 #pragma unroll
     for (int r = 0; r < R; ++r)
-#pragma unroll
-        for (int b = 0; b < B; ++b) {
-            acc0[r][b] = f2(0.f, 0.f);
-            acc1[r][b] = f2(0.f, 0.f);
-        }
+        acc[r] = 0.0;
+    double gsum = 0.0;  // stream-0 sum kept for the SwiGLU epilogue
 
-    Cursor cc{t0 * G::TR, 0, 0};
+    Cursor cc{t0 * kFxTileRows, 0, 0};
     int slot = 0;
     uint32_t parity = 0;
     for (; consumed < total; ++consumed) {
@@ -149,19 +354,373 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_kernel(const Q4KPa
             failed = true;
             break;
         }
-        const int kb0 = (c_begin + cc.kcl) * LPR;
-        const int nblk = min(LPR, p.nb - kb0);
-        if (l < nblk) {
-            const uint8_t *slot_p = my_ring + slot * G::SLOT_BYTES + rg * G::RG_PITCH;
-            // byte offsets of this lane's header and quant slices within a row of the slot
-            const BlockOffsets bo = block_offsets<SOA>(l, nblk);
-            const int hdr_off = bo.hdr, qs_off0 = bo.qs0, qs_step = bo.qs_step;
+        const int kb0 = (c_begin + cc.kcl) * kFxBPC;
+        const int nblk = min(kFxBPC, p.nb - kb0);
+        if (g < nblk) {
+            const uint8_t *slot_p = my_ring + slot * kFxSlotBytes + i * kFxRowPitch;
+            const BlockOffsets bo = block_offsets<SOA>(g, nblk);
+            uint4 hd[R];
+            uint32_t sc03[R], sc47[R];
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                hd[r] = *reinterpret_cast<const uint4 *>(slot_p + 8 * r * kFxRowPitch + bo.hdr);
+                // GGML get_scale_min_k4 packing: scales 0..3 are the low six bits of
+                // bytes 0..3; scales 4..7 take their low four bits from the low nibbles
+                // of bytes 8..11 and their top two bits from bits 6..7 of bytes 0..3
+                sc03[r] = hd[r].y & 0x3F3F3F3Fu;
+                sc47[r] = (hd[r].w & 0x0F0F0F0Fu) | ((hd[r].y >> 2) & 0x30303030u);
+            }
+            const uint8_t *xb = limbs + (kb0 - kb_begin + g) * kFxLimbPitch;
+
+            int isum[R][4];
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    isum[r][k] = 0;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                int alo[R][4], ahi[R][4];
+#pragma unroll
+                for (int r = 0; r < R; ++r)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        alo[r][k] = 0;
+                        ahi[r][k] = 0;
+                    }
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int s = 2 * c + h;  // 16-byte quant slice
+                    uint4 q[R];
+#pragma unroll
+                    for (int r = 0; r < R; ++r)
+                        q[r] = *reinterpret_cast<const uint4 *>(slot_p + 8 * r * kFxRowPitch + bo.qs0 +
+                                                                s * bo.qs_step);
+                    fx_slice<R>(q, xb + 64 * c + 16 * h, xb + 64 * c + 32 + 16 * h, alo, ahi);
+                }
+                // fold the scales of sub-blocks 2c (lo) and 2c+1 (hi); the sums are
+                // kept 16 times larger (the hi sums already are): |16 I_l| < 2^29
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const uint32_t sw = (c < 2) ? sc03[r] : sc47[r];
+                    const int slo16 = static_cast<int>((sw >> (16 * (c & 1))) & 0xFFu) << 4;
+                    const int shi = static_cast<int>((sw >> (16 * (c & 1) + 8)) & 0xFFu);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        isum[r][k] += slo16 * alo[r][k] + shi * ahi[r][k];
+                }
+            }
+
+            // per row: y_sb = 2^-F (d I_s - dmin I_m) in fp64
+            const double *ap = reinterpret_cast<const double *>(aux + (kb0 - kb_begin + g) * kFxAuxPitch);
+            double X[8];
+#pragma unroll
+            for (int j = 0; j < 8; j += 2) {
+                const double2 t = *reinterpret_cast<const double2 *>(ap + j);
+                X[j] = t.x;
+                X[j + 1] = t.y;
+            }
+            const double s2f = ap[8];
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                double is = static_cast<double>(isum[r][3]);
+                is = fma(is, 256.0, static_cast<double>(isum[r][2]));
+                is = fma(is, 256.0, static_cast<double>(isum[r][1]));
+                is = fma(is, 256.0, static_cast<double>(isum[r][0]));
+                const uint32_t mn03 = hd[r].z & 0x3F3F3F3Fu;
+                const uint32_t mn47 = ((hd[r].w >> 4) & 0x0F0F0F0Fu) | ((hd[r].z >> 2) & 0x30303030u);
+                // I_m as a tree of exact products and sums (integers below 2^53)
+                double pmn[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint32_t mw = (j < 4) ? mn03 : mn47;
+                    pmn[j] = static_cast<double>((mw >> (8 * (j & 3))) & 0xFFu) * X[j];
+                }
+                const double im = ((pmn[0] + pmn[1]) + (pmn[2] + pmn[3])) + ((pmn[4] + pmn[5]) + (pmn[6] + pmn[7]));
+                // the 1/16 undoes the scaling of the integer sums (exact)
+                const double d =
+                    static_cast<double>(__half2float(__ushort_as_half(static_cast<unsigned short>(hd[r].x & 0xFFFFu)))) *
+                    (s2f * 0.0625);
+                const double dm =
+                    static_cast<double>(__half2float(__ushort_as_half(static_cast<unsigned short>(hd[r].x >> 16)))) *
+                    s2f;
+                const double pm = dm * im;            // rounded
+                const double em = fma(dm, im, -pm);   // its exact rounding error
+                acc[r] += fma(d, is, -pm) - em;
+            }
+        }
+
+        __syncwarp();
+        if (issued < total) {
+            fence_proxy_async_smem();
+            fx_issue_slot<TMA>(p, maps, pc, slot, c_begin, my_ring_s, my_bars_s, lane);
+            pc.advance(nch, NS, row_step);
+            ++issued;
+        }
+
+        const int cur_st = cc.st;
+        const long long row0 = cc.row0;
+        const bool last_chunk = (cc.kcl == nch - 1);
+        cc.advance(nch, NS, row_step);
+        if (++slot == p.depth) {
+            slot = 0;
+            parity ^= 1u;
+        }
+        if (!last_chunk)
+            continue;
+
+        // end of this stream's K range for the tile: add the four quarters' sums
+        const bool up = (lane & 16) != 0;
+        double t = (up ? acc[1] : acc[0]) + __shfl_xor_sync(0xffffffffu, up ? acc[0] : acc[1], 16);
+        t += __shfl_xor_sync(0xffffffffu, t, 8);
+        acc[0] = 0.0;
+        acc[1] = 0.0;
+        if constexpr (NS == 2) {
+            if (cur_st == 0) {
+                gsum = t;
+                continue;
+            }
+        }
+        const long long n = row0 + wrow;
+        if (p.grp.n > 0 && !p.cluster && p.splits == 1) {
+            const FxRows fr = fx_rows(p, 0, row0);
+            if (writer && fr.row0 + wrow < fr.nrows)
+                fx_group_out(p, fr.sel)[fr.row0 + wrow] = static_cast<float>(t);
+            continue;
+        }
+        if (p.cluster) {
+            // this warp's only tile: keep its partials for the cluster reduction
+            if (writer) {
+                cpart[(warp * 2 + 0) * kFxTileRows + wrow] = (NS == 2) ? gsum : t;
+                cpart[(warp * 2 + 1) * kFxTileRows + wrow] = t;
+            }
+            continue;
+        }
+        if (!writer || n >= p.N)
+            continue;
+        if (p.splits > 1) {
+            if constexpr (NS == 2) {
+                p.part[(static_cast<long long>(split) * 2 + 0) * p.N + n] = static_cast<float>(gsum);
+                p.part[(static_cast<long long>(split) * 2 + 1) * p.N + n] = static_cast<float>(t);
+            } else {
+                p.part[static_cast<long long>(split) * p.N + n] = static_cast<float>(t);
+            }
+        } else {
+            float out;
+            if constexpr (NS == 2) {
+                const float gv = static_cast<float>(gsum);
+                out = gv / (1.0f + expf(-gv)) * static_cast<float>(t);
+            } else {
+                out = static_cast<float>(t);
+            }
+            *gemv_out_addr(p.y, p.g, p.qg_hd, p.N, 0, n) = out;
+            if (p.argmax && cand_better(out, n, best_v, best_i)) {
+                best_v = out;
+                best_i = n;
+            }
+        }
+    }
+
+    if (failed) {
+        // the copies already issued into this warp's ring must land before the CTA exits
+        for (long long k = consumed; k < issued; ++k) {
+            mbar_wait_bounded(my_bars_s + slot * 8, parity, nullptr);
+            if (++slot == p.depth) {
+                slot = 0;
+                parity ^= 1u;
+            }
+        }
+    }
+
+    if (p.cluster) {
+        // Splits of a CTA column are one cluster and their warps hold the same
+        // tiles: each tile is finished by the CTA whose rank is the warp index
+        // modulo the split count, adding the partials of ranks 0, 1, ... in order.
+        namespace cg = cooperative_groups;
+        cg::cluster_group cl = cg::this_cluster();
+        cl.sync();
+        if (warp % p.splits == split && t0 < p.tiles && lane < kFxTileRows) {
+            double g = 0.0, u = 0.0;
+            for (int r = 0; r < p.splits; ++r) {
+                const double *rp = cl.map_shared_rank(cpart, r);
+                g += rp[(warp * 2 + 0) * kFxTileRows + lane];
+                u += rp[(warp * 2 + 1) * kFxTileRows + lane];
+            }
+            const long long n = t0 * kFxTileRows + lane;
+            const FxRows fr = fx_rows(p, 0, t0 * kFxTileRows);
+            if (p.grp.n > 0) {
+                if (fr.row0 + lane < fr.nrows)
+                    fx_group_out(p, fr.sel)[fr.row0 + lane] = static_cast<float>(g);
+            } else if (n < p.N) {
+                float out;
+                if constexpr (NS == 2) {
+                    const float gv = static_cast<float>(g);
+                    out = gv / (1.0f + expf(-gv)) * static_cast<float>(u);
+                } else {
+                    out = static_cast<float>(g);
+                }
+                *gemv_out_addr(p.y, p.g, p.qg_hd, p.N, 0, n) = out;
+                if (p.argmax && cand_better(out, n, best_v, best_i)) {
+                    best_v = out;
+                    best_i = n;
+                }
+            }
+        }
+        cl.sync();  // no CTA leaves while another reads its shared memory
+    }
+
+    if (p.argmax && (p.splits == 1 || p.cluster)) {
+        // CTA-wide (max, lowest index) candidate
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, best_v, o);
+            const long long oi = __shfl_xor_sync(0xffffffffu, best_i, o);
+            if (cand_better(ov, oi, best_v, best_i)) {
+                best_v = ov;
+                best_i = oi;
+            }
+        }
+        if (lane == 0) {
+            red[warp].v = best_v;
+            red[warp].idx = best_i;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            ArgmaxCand c = red[0];
+            for (int w = 1; w < nwarps; ++w)
+                if (cand_better(red[w].v, red[w].idx, c.v, c.idx))
+                    c = red[w];
+            p.cand[blockIdx.x] = c;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Batches of 2..8 activation rows: the same quarter-warp lanes, TMA slots and
+// rings, with exact fp32 weights (q4k_decode.cuh: formed once per weight, used
+// B times) and fp32 accumulation.  x is staged in fp32 (lo, hi) pairs; each
+// quarter-warp reads its super-block's pairs as a broadcast.
+// ---------------------------------------------------------------------------
+
+// Sums the values of the four quarter-warps (lanes i, i+8, i+16, i+24) with a
+// transposing butterfly over lane bits 4 and 3: on entry every lane holds M
+// values (M a multiple of 4); on exit it holds the totals of indices
+// off .. off + M/4 - 1, off = (bit 4 ? M/2 : 0) + (bit 3 ? M/4 : 0).
+template <int M>
+__device__ __forceinline__ void quarter_sum(float (&v)[M], int lane)
+{
+    static_assert(M % 4 == 0, "four quarter-warps share the values");
+    const bool up16 = (lane & 16) != 0;
+#pragma unroll
+    for (int k = 0; k < M / 2; ++k) {
+        const float send = up16 ? v[k] : v[k + M / 2];
+        const float keep = up16 ? v[k + M / 2] : v[k];
+        v[k] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+    const bool up8 = (lane & 8) != 0;
+#pragma unroll
+    for (int k = 0; k < M / 4; ++k) {
+        const float send = up8 ? v[k] : v[k + M / 4];
+        const float keep = up8 ? v[k + M / 4] : v[k];
+        v[k] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+}
+
+constexpr int kFxbMaxWarps(int B) { return B <= 2 ? 12 : 8; }
+
+template <int B, int NS, bool SOA, bool TMA>
+__global__ void __launch_bounds__(kFxbMaxWarps(B) * 32, 1)
+    q4k_gemv_fxb_kernel(const __grid_constant__ Q4KParams p, const __grid_constant__ FxMaps maps)
+{
+    constexpr int R = kFxRows;
+    constexpr int MV = R * B;                 // values per lane per stream (index r*B + b)
+    constexpr int MP = (MV + 3) / 4 * 4;      // padded for the quarter-warp butterfly
+    constexpr int VPL = MP / 4;               // values per lane after it
+    static_assert(R == 2 && B >= 2 && B <= 8, "two rows per lane, batches of 2 to 8");
+
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int nwarps = blockDim.x >> 5;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int g = lane >> 3;   // super-block of each chunk
+    const int i = lane & 7;    // rows i and i + 8 of each tile
+    const int voff = ((lane & 16) ? MP / 2 : 0) + ((lane & 8) ? MP / 4 : 0);
+
+    const int split = blockIdx.x / p.ctas_per_split;
+    const int cj = blockIdx.x % p.ctas_per_split;
+    const int nchunk_total = (p.nb + kFxBPC - 1) / kFxBPC;
+    const int c_begin = split * p.chunks_per_split;
+    const int c_end = min(c_begin + p.chunks_per_split, nchunk_total);
+    const int nch = c_end - c_begin;
+    const int kb_begin = c_begin * kFxBPC;
+    const int nbs = min(nch * kFxBPC, p.nb - kb_begin);
+
+    // shared memory: [x pairs][barriers][ring]
+    const int x_bytes = (B * nbs * kXBlockPitch + 127) & ~127;
+    uint8_t *xs = smem;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + x_bytes);
+    const int bar_bytes = (nwarps * p.depth * 8 + 127) & ~127;
+    const uint32_t ring_pad = (128u - ((smem_u32(smem) + x_bytes + bar_bytes) & 127u)) & 127u;
+    uint8_t *ring = smem + x_bytes + bar_bytes + ring_pad;
+    uint8_t *my_ring = ring + static_cast<size_t>(warp) * p.depth * kFxSlotBytes;
+    const uint32_t my_ring_s = smem_u32(my_ring);
+    const uint32_t my_bars_s = smem_u32(bars + warp * p.depth);
+
+    const long long tstride = static_cast<long long>(p.ctas_per_split) * nwarps;
+    const long long t0 = static_cast<long long>(warp) * p.ctas_per_split + cj;
+    const long long ntiles_w = (t0 < p.tiles) ? (p.tiles - t0 + tstride - 1) / tstride : 0;
+    const long long total = ntiles_w * NS * nch;
+    const long long row_step = tstride * kFxTileRows;
+
+    Cursor pc{t0 * kFxTileRows, 0, 0};
+    long long issued = 0;
+    if (lane == 0) {
+        for (int s = 0; s < p.depth; ++s)
+            mbar_init(my_bars_s + s * 8, 1);
+        mbar_fence_init();
+    }
+    __syncwarp();
+    pdl_wait();
+    pdl_launch_dependents();
+    for (int s = 0; s < p.depth && issued < total; ++s, ++issued) {
+        fx_issue_slot<TMA>(p, maps, pc, s, c_begin, my_ring_s, my_bars_s, lane);
+        pc.advance(nch, NS, row_step);
+    }
+
+    stage_x_pairs<(B <= 2) ? 4 : 1>(p.x, p.K, B, kb_begin, nbs, xs);
+    __syncthreads();
+
+    bool failed = false;
+    long long consumed = 0;
+    float2 acc0[R][B], acc1[R][B];
+    float gsum[NS == 2 ? VPL : 1];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+            acc0[r][b] = f2(0.f, 0.f);
+            acc1[r][b] = f2(0.f, 0.f);
+        }
+
+    Cursor cc{t0 * kFxTileRows, 0, 0};
+    int slot = 0;
+    uint32_t parity = 0;
+    for (; consumed < total; ++consumed) {
+        const bool ok = mbar_wait_bounded(my_bars_s + slot * 8, parity, p.err);
+        if (!__all_sync(0xffffffffu, ok)) {
+            failed = true;
+            break;
+        }
+        const int kb0 = (c_begin + cc.kcl) * kFxBPC;
+        const int nblk = min(kFxBPC, p.nb - kb0);
+        if (g < nblk) {
+            const uint8_t *slot_p = my_ring + slot * kFxSlotBytes + i * kFxRowPitch;
+            const BlockOffsets bo = block_offsets<SOA>(g, nblk);
             Hdr hd[R];
 #pragma unroll
             for (int r = 0; r < R; ++r)
-                hd[r] = decode_hdr(*reinterpret_cast<const uint4 *>(slot_p + r * G::ROW_BYTES + hdr_off));
-            const uint8_t *xblk = xs + (kb0 - kb_begin + l) * kXBlockPitch;
-
+                hd[r] = decode_hdr(*reinterpret_cast<const uint4 *>(slot_p + 8 * r * kFxRowPitch + bo.hdr));
+            const uint8_t *xblk = xs + (kb0 - kb_begin + g) * kXBlockPitch;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 ChunkScales cs[R];
@@ -174,7 +733,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_kernel(const Q4KPa
                     uint4 q[R];
 #pragma unroll
                     for (int r = 0; r < R; ++r)
-                        q[r] = *reinterpret_cast<const uint4 *>(slot_p + r * G::ROW_BYTES + qs_off0 + s * qs_step);
+                        q[r] = *reinterpret_cast<const uint4 *>(slot_p + 8 * r * kFxRowPitch + bo.qs0 +
+                                                                s * bo.qs_step);
 #pragma unroll
                     for (int t = 0; t < 4; ++t) {
 #pragma unroll
@@ -195,10 +755,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_kernel(const Q4KPa
 
         __syncwarp();
         if (issued < total) {
-            if (lane == 0) {
-                fence_proxy_async_smem();
-                issue_slot<G>(p, pc, slot, c_begin, my_ring_s, my_bars_s);
-            }
+            fence_proxy_async_smem();
+            fx_issue_slot<TMA>(p, maps, pc, slot, c_begin, my_ring_s, my_bars_s, lane);
             pc.advance(nch, NS, row_step);
             ++issued;
         }
@@ -214,7 +772,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_kernel(const Q4KPa
         if (!last_chunk)
             continue;
 
-        // end of this stream's K range for the tile: reduce across the row group
+        // end of this stream's K range for the tile: add the four quarters' sums
         float v[MP];
 #pragma unroll
         for (int r = 0; r < R; ++r)
@@ -226,360 +784,55 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) q4k_gemv_kernel(const Q4KPa
                 acc1[r][b] = f2(0.f, 0.f);
             }
 #pragma unroll
-        for (int j = MV; j < MP; ++j)
-            v[j] = 0.f;
-        if constexpr (LPR > 1)
-            GroupReduce<LPR / 2, MP>::run(v, l);
-
+        for (int k = MV; k < MP; ++k)
+            v[k] = 0.f;
+        quarter_sum<MP>(v, lane);
         if constexpr (NS == 2) {
             if (cur_st == 0) {
 #pragma unroll
-                for (int j = 0; j < VPL; ++j)
-                    gsum[j] = v[j];
+                for (int k = 0; k < VPL; ++k)
+                    gsum[k] = v[k];
                 continue;
             }
         }
-        if (!writer)
-            continue;
 #pragma unroll
-        for (int j = 0; j < VPL; ++j) {
-            const int idx = off + j;
+        for (int k = 0; k < VPL; ++k) {
+            const int idx = voff + k;
             if (idx >= MV)
                 continue;
             const int r = idx / B;
             const int b = idx % B;
-            const long long n = row0 + rg * R + r;
+            const long long n = row0 + i + 8 * r;
             if (n >= p.N)
                 continue;
             if (p.splits > 1) {
                 if constexpr (NS == 2) {
-                    p.part[((static_cast<long long>(split) * 2 + 0) * B + b) * p.N + n] = gsum[j] * 0x1p64f;
-                    p.part[((static_cast<long long>(split) * 2 + 1) * B + b) * p.N + n] = v[j] * 0x1p64f;
+                    p.part[((static_cast<long long>(split) * 2 + 0) * B + b) * p.N + n] = gsum[k] * 0x1p64f;
+                    p.part[((static_cast<long long>(split) * 2 + 1) * B + b) * p.N + n] = v[k] * 0x1p64f;
                 } else {
-                    p.part[(static_cast<long long>(split) * B + b) * p.N + n] = v[j] * 0x1p64f;
+                    p.part[(static_cast<long long>(split) * B + b) * p.N + n] = v[k] * 0x1p64f;
                 }
             } else {
                 float out;
                 if constexpr (NS == 2) {
-                    const float g = gsum[j] * 0x1p64f;
-                    const float u = v[j] * 0x1p64f;
-                    out = g / (1.0f + expf(-g)) * u;
+                    const float gv = gsum[k] * 0x1p64f;
+                    out = gv / (1.0f + expf(-gv)) * (v[k] * 0x1p64f);
                 } else {
-                    out = v[j] * 0x1p64f;
+                    out = v[k] * 0x1p64f;
                 }
                 *gemv_out_addr(p.y, p.g, p.qg_hd, p.N, b, n) = out;
-                if (p.argmax && cand_better(out, n, best_v, best_i)) {
-                    best_v = out;
-                    best_i = n;
-                }
             }
         }
     }
 
     if (failed) {
         // the copies already issued into this warp's ring must land before the CTA exits
-        for (long long i = consumed; i < issued; ++i) {
+        for (long long k = consumed; k < issued; ++k) {
             mbar_wait_bounded(my_bars_s + slot * 8, parity, nullptr);
             if (++slot == p.depth) {
                 slot = 0;
                 parity ^= 1u;
             }
-        }
-    }
-
-    if (p.argmax && p.splits == 1) {
-        // CTA-wide (max, lowest index) candidate
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, best_v, o);
-            const long long oi = __shfl_xor_sync(0xffffffffu, best_i, o);
-            if (cand_better(ov, oi, best_v, best_i)) {
-                best_v = ov;
-                best_i = oi;
-            }
-        }
-        if (lane == 0) {
-            red[warp].v = best_v;
-            red[warp].idx = best_i;
-        }
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            ArgmaxCand c = red[0];
-            for (int w = 1; w < nwarps; ++w)
-                if (cand_better(red[w].v, red[w].idx, c.v, c.idx))
-                    c = red[w];
-            p.cand[blockIdx.x] = c;
-        }
-    }
-}
-
-// ---------------------------------------------------------------------------
-// Batch-1 kernel with half-block lanes (GeoHalf): each lane owns two of the
-// four 64-weight chunks of one super-block for two rows, so a slot is 4.5 KB
-// and sixteen warps (four per scheduler) fit beside their two-deep rings.
-// x keeps the (lo, hi) pair staging, with the two 512-byte halves of every
-// super-block kXHalfGap bytes apart and kXHalfPitch bytes per super-block, so
-// the eight lanes of one shared-memory phase read eight distinct bank groups.
-// ---------------------------------------------------------------------------
-constexpr int kB1Warps = 16;
-constexpr int kXHalfPitch = 1056;
-constexpr int kXHalfGap = 528;
-
-template <int LPR, int NS, bool SOA>
-__global__ void __launch_bounds__(kB1Warps * 32, 1) q4k_gemv_b1_kernel(const Q4KParams p)
-{
-    pdl_wait();
-    pdl_launch_dependents();
-    using G = GeoHalf<LPR>;
-    constexpr int R = G::R;
-
-    extern __shared__ __align__(128) uint8_t smem[];
-    const int nwarps = blockDim.x >> 5;
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int rg = lane / LPR;
-    const int l = lane % LPR;
-    const int bl = l >> 1;   // super-block of the chunk
-    const int hh = l & 1;    // half: chunks 2*hh and 2*hh + 1
-
-    const int split = blockIdx.x / p.ctas_per_split;
-    const int cj = blockIdx.x % p.ctas_per_split;
-    const int nchunk_total = (p.nb + G::BPC - 1) / G::BPC;
-    const int c_begin = split * p.chunks_per_split;
-    const int c_end = min(c_begin + p.chunks_per_split, nchunk_total);
-    const int nch = c_end - c_begin;
-    const int kb_begin = c_begin * G::BPC;
-    const int nbs = min(nch * G::BPC, p.nb - kb_begin);
-
-    // shared memory: [x staging][barriers][ring][argmax scratch]
-    const int x_bytes = (nbs * kXHalfPitch + 127) & ~127;
-    uint8_t *xs = smem;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + x_bytes);
-    const int bar_bytes = (nwarps * p.depth * 8 + 127) & ~127;
-    uint8_t *ring = smem + x_bytes + bar_bytes;
-    uint8_t *my_ring = ring + static_cast<size_t>(warp) * p.depth * G::SLOT_BYTES;
-    const uint32_t my_ring_s = smem_u32(my_ring);
-    const uint32_t my_bars_s = smem_u32(bars + warp * p.depth);
-    ArgmaxCand *red = reinterpret_cast<ArgmaxCand *>(ring + static_cast<size_t>(nwarps) * p.depth * G::SLOT_BYTES);
-
-    const long long tstride = static_cast<long long>(p.ctas_per_split) * nwarps;
-    // warp-major tile order: the last, partial round of tiles spreads over all SMs
-    const long long t0 = static_cast<long long>(warp) * p.ctas_per_split + cj;
-    const long long ntiles_w = (t0 < p.tiles) ? (p.tiles - t0 + tstride - 1) / tstride : 0;
-    const long long total = ntiles_w * NS * nch;
-    const long long row_step = tstride * G::TR;
-
-    // After the row-group reduction lane 0 of the group holds row 0's sum and
-    // lane LPR/2 row 1's; the other lanes hold copies.
-    const bool writer = (l & (LPR / 2 - 1)) == 0;
-    const int wrow = (l >= LPR / 2) ? 1 : 0;
-
-    Cursor pc{t0 * G::TR, 0, 0};
-    long long issued = 0;
-    if (lane == 0) {
-        for (int s = 0; s < p.depth; ++s)
-            mbar_init(my_bars_s + s * 8, 1);
-        mbar_fence_init();
-    }
-    for (int s = 0; s < p.depth && issued < total; ++s, ++issued) {
-        if (lane == 0)
-            issue_slot<G>(p, pc, s, c_begin, my_ring_s, my_bars_s);
-        pc.advance(nch, NS, row_step);
-    }
-
-    // stage x in (lo, hi) pairs, 8 loads in flight per thread
-    {
-        constexpr int kStageBatch = 8;
-        const int n_out = nbs * 64;
-        for (int base = threadIdx.x; base < n_out; base += kStageBatch * blockDim.x) {
-            float2 lo[kStageBatch], hi[kStageBatch];
-#pragma unroll
-            for (int u = 0; u < kStageBatch; ++u) {
-                const int idx = base + u * blockDim.x;
-                if (idx < n_out) {
-                    const int kbl = idx >> 6, sl = (idx >> 3) & 7, k = idx & 7;
-                    const float *xb = p.x + static_cast<long long>(kb_begin + kbl) * 256 + 64 * (sl >> 1) +
-                                      16 * (sl & 1) + 2 * k;
-                    lo[u] = __ldg(reinterpret_cast<const float2 *>(xb));
-                    hi[u] = __ldg(reinterpret_cast<const float2 *>(xb + 32));
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < kStageBatch; ++u) {
-                const int idx = base + u * blockDim.x;
-                if (idx < n_out) {
-                    const int kbl = idx >> 6, sl = (idx >> 3) & 7, k = idx & 7;
-                    *reinterpret_cast<float4 *>(xs + kbl * kXHalfPitch + (sl >> 2) * kXHalfGap + (sl & 3) * 128 +
-                                                k * 16) = make_float4(lo[u].x, hi[u].x, lo[u].y, hi[u].y);
-                }
-            }
-        }
-    }
-    __syncthreads();
-
-    float best_v = -INFINITY;
-    long long best_i = 0x7fffffffffffffffLL;
-    bool failed = false;
-    long long consumed = 0;
-    float gsum = 0.f;  // stream-0 sum kept for the SwiGLU epilogue
-
-    float2 acc0[R], acc1[R];
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-        acc0[r] = f2(0.f, 0.f);
-        acc1[r] = f2(0.f, 0.f);
-    }
-
-    Cursor cc{t0 * G::TR, 0, 0};
-    int slot = 0;
-    uint32_t parity = 0;
-    for (; consumed < total; ++consumed) {
-        const bool ok = mbar_wait_bounded(my_bars_s + slot * 8, parity, p.err);
-        if (!__all_sync(0xffffffffu, ok)) {
-            failed = true;
-            break;
-        }
-        const int kb0 = (c_begin + cc.kcl) * G::BPC;
-        const int nblk = min(G::BPC, p.nb - kb0);
-        if (bl < nblk) {
-            const uint8_t *slot_p = my_ring + slot * G::SLOT_BYTES + rg * G::RG_PITCH;
-            // this lane's header and its first quant slice (slice 4*hh of the super-block)
-            const BlockOffsets bo = block_offsets<SOA>(bl, nblk);
-            const int hdr_off = bo.hdr, qs_step = bo.qs_step;
-            const int qs_off0 = bo.qs0 + 4 * hh * bo.qs_step;
-            Hdr hd[R];
-            uint32_t scw[R], mnw[R];
-#pragma unroll
-            for (int r = 0; r < R; ++r) {
-                hd[r] = decode_hdr(*reinterpret_cast<const uint4 *>(slot_p + r * G::ROW_BYTES + hdr_off));
-                scw[r] = hh ? hd[r].sc47 : hd[r].sc03;
-                mnw[r] = hh ? hd[r].mn47 : hd[r].mn03;
-            }
-            const uint8_t *xl = xs + (kb0 - kb_begin + bl) * kXHalfPitch + hh * kXHalfGap;
-
-#pragma unroll
-            for (int cp = 0; cp < 2; ++cp) {  // chunk 2*hh + cp
-                ChunkScales cs[R];
-#pragma unroll
-                for (int r = 0; r < R; ++r)
-                    cs[r] = scales_from_words(hd[r], scw[r], mnw[r], cp * 2);
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int sl = 2 * cp + h;  // slice within the half
-                    uint4 q[R];
-#pragma unroll
-                    for (int r = 0; r < R; ++r)
-                        q[r] = *reinterpret_cast<const uint4 *>(slot_p + r * G::ROW_BYTES + qs_off0 + sl * qs_step);
-#pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        const uint8_t *xq = xl + sl * 128 + 32 * t;
-                        const float4 xa = *reinterpret_cast<const float4 *>(xq);
-                        const float4 xb = *reinterpret_cast<const float4 *>(xq + 16);
-#pragma unroll
-                        for (int r = 0; r < R; ++r) {
-                            const uint32_t wv = (t == 0) ? q[r].x : (t == 1) ? q[r].y : (t == 2) ? q[r].z : q[r].w;
-                            q4_word(wv, cs[r], xa, xb, acc0[r], acc1[r]);
-                        }
-                    }
-                }
-            }
-        }
-
-        __syncwarp();
-        if (issued < total) {
-            if (lane == 0) {
-                fence_proxy_async_smem();
-                issue_slot<G>(p, pc, slot, c_begin, my_ring_s, my_bars_s);
-            }
-            pc.advance(nch, NS, row_step);
-            ++issued;
-        }
-
-        const int cur_st = cc.st;
-        const long long row0 = cc.row0;
-        const bool last_chunk = (cc.kcl == nch - 1);
-        cc.advance(nch, NS, row_step);
-        if (++slot == p.depth) {
-            slot = 0;
-            parity ^= 1u;
-        }
-        if (!last_chunk)
-            continue;
-
-        float v[2];
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-            const float2 a = __fadd2_rn(acc0[r], acc1[r]);
-            v[r] = a.x + a.y;
-            acc0[r] = f2(0.f, 0.f);
-            acc1[r] = f2(0.f, 0.f);
-        }
-        GroupReduce<LPR / 2, 2>::run(v, l);
-        if constexpr (NS == 2) {
-            if (cur_st == 0) {
-                gsum = v[0];
-                continue;
-            }
-        }
-        const long long n = row0 + rg * R + wrow;
-        if (!writer || n >= p.N)
-            continue;
-        if (p.splits > 1) {
-            if constexpr (NS == 2) {
-                p.part[(static_cast<long long>(split) * 2 + 0) * p.N + n] = gsum * 0x1p64f;
-                p.part[(static_cast<long long>(split) * 2 + 1) * p.N + n] = v[0] * 0x1p64f;
-            } else {
-                p.part[static_cast<long long>(split) * p.N + n] = v[0] * 0x1p64f;
-            }
-        } else {
-            float out;
-            if constexpr (NS == 2) {
-                const float g = gsum * 0x1p64f;
-                out = g / (1.0f + expf(-g)) * (v[0] * 0x1p64f);
-            } else {
-                out = v[0] * 0x1p64f;
-            }
-            *gemv_out_addr(p.y, p.g, p.qg_hd, p.N, 0, n) = out;
-            if (p.argmax && cand_better(out, n, best_v, best_i)) {
-                best_v = out;
-                best_i = n;
-            }
-        }
-    }
-
-    if (failed) {
-        // the copies already issued into this warp's ring must land before the CTA exits
-        for (long long i = consumed; i < issued; ++i) {
-            mbar_wait_bounded(my_bars_s + slot * 8, parity, nullptr);
-            if (++slot == p.depth) {
-                slot = 0;
-                parity ^= 1u;
-            }
-        }
-    }
-
-    if (p.argmax && p.splits == 1) {
-        // CTA-wide (max, lowest index) candidate
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, best_v, o);
-            const long long oi = __shfl_xor_sync(0xffffffffu, best_i, o);
-            if (cand_better(ov, oi, best_v, best_i)) {
-                best_v = ov;
-                best_i = oi;
-            }
-        }
-        if (lane == 0) {
-            red[warp].v = best_v;
-            red[warp].idx = best_i;
-        }
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            ArgmaxCand c = red[0];
-            for (int w = 1; w < nwarps; ++w)
-                if (cand_better(red[w].v, red[w].idx, c.v, c.idx))
-                    c = red[w];
-            p.cand[blockIdx.x] = c;
         }
     }
 }
@@ -588,20 +841,11 @@ __global__ void __launch_bounds__(kB1Warps * 32, 1) q4k_gemv_b1_kernel(const Q4K
 // host side
 // ---------------------------------------------------------------------------
 
-int q4k_slot_bytes(int lpr) { return lpr == 16 ? Geo<16, 2>::SLOT_BYTES : Geo<4, 2>::SLOT_BYTES; }
-
-// Launch plan for a shape; the same function sizes the workspace, so the two
-// always agree.
 // Warps per CTA for `tiles` row tiles on `sm_count` SMs (one CTA per SM):
-// enough to give every SM work and at least one per scheduler; with `round4`
-// a multiple of four, so the four schedulers of an SM carry equal numbers of
-// warps (the full-block kernel skips the rounding when its shared memory
-// would then force a K split).
-int q4k_pick_warps(long long tiles, int sm_count, int max_warps, bool round4)
+// enough to give every SM work and at least one per scheduler.
+static int pick_warps(long long tiles, int sm_count, int max_warps)
 {
     long long w = (tiles + sm_count - 1) / sm_count;
-    if (round4)
-        w = (w + 3) / 4 * 4;
     if (w < 4)
         w = 4;
     if (w > max_warps)
@@ -609,35 +853,56 @@ int q4k_pick_warps(long long tiles, int sm_count, int max_warps, bool round4)
     return static_cast<int>(w);
 }
 
-static Q4KPlan q4k_plan_half(long long N, int nb, int NS, int sm_count, int smem_optin)
+// The driver's tensor-map encoder, looked up once (null when unavailable).
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+// Launch plan.  Slot copies by TMA when the driver's encoder is available.  K
+// is split until there are about eight tile tasks per SM (or each split is one
+// chunk), warps per CTA follow from the tasks per SM, and K is split further
+// if the activations would not fit beside a two-deep ring per warp; the ring
+// is as deep as shared memory allows, up to 4 slots.
+static Q4KPlan plan_quarter_warp(long long N, int nb, int B, int NS, int sm_count, int smem_optin)
 {
     Q4KPlan pl{};
-    const int misc = 256 /*argmax scratch*/ + 512 /*barriers*/;
-    // 16-block chunks when they tile the row, else 4-block chunks (both start
-    // at SoA group boundaries)
-    const int lpr = (nb % 16 == 0) ? 32 : 8;
-    const int bpc = lpr / 2;
-    const int sb = (lpr == 32) ? GeoHalf<32>::SLOT_BYTES : GeoHalf<8>::SLOT_BYTES;
-    const int TR = (32 / lpr) * 2;
-    const long long tiles = (N + TR - 1) / TR;
-    const int nchunk = (nb + bpc - 1) / bpc;
-    const int w0 = q4k_pick_warps(tiles, sm_count, kB1Warps, true);
-    for (int warps = w0; warps >= 4 && !pl.ok; warps = (warps > 4 && warps / 2 < 4) ? 4 : warps / 2) {
-        int splits = 1, cps = nchunk;
-        for (;;) {
-            cps = (nchunk + splits - 1) / splits;
-            if (cps * bpc * kXHalfPitch + warps * 2 * sb + misc <= smem_optin || cps == 1)
-                break;
-            ++splits;
-        }
-        const long long warps_total = static_cast<long long>(sm_count) * warps;
-        while (tiles * NS * splits * 2 < warps_total && splits < nchunk) {
+    // DQGEMV_NO_TMA=1 selects the per-row bulk copies (same shared-memory
+    // layout, bit-identical results), for comparing the two copy paths
+    const char *no_tma = getenv("DQGEMV_NO_TMA");
+    const bool tma = N < 0x7FFFFFFFLL && tensor_map_encoder() != nullptr && !(no_tma && no_tma[0] == '1');
+    const int misc = 256 /*argmax scratch, 16 B per warp*/ + 512 /*barriers*/ + 128 /*ring alignment*/;
+    // staged activations per super-block: limb planes and sums (batch 1), or B
+    // rows of fp32 pairs
+    const int stage = (B == 1) ? kFxLimbPitch + kFxAuxPitch : B * kXBlockPitch;
+    const int max_warps = (B == 1) ? kFxMaxWarps : kFxbMaxWarps(B);
+    const long long tiles = (N + kFxTileRows - 1) / kFxTileRows;
+    const int nchunk = (nb + kFxBPC - 1) / kFxBPC;
+    int splits_par = 1;
+    while (tiles * splits_par < 8LL * sm_count && splits_par < nchunk)
+        ++splits_par;
+    const int w0 = pick_warps(tiles * splits_par, sm_count, max_warps);
+    for (int warps = w0; warps >= 4 && !pl.ok; --warps) {
+        int splits = splits_par;
+        int cps = (nchunk + splits - 1) / splits;
+        while (cps * kFxBPC * stage + warps * 2 * kFxSlotBytes + misc > smem_optin && cps > 1) {
             ++splits;
             cps = (nchunk + splits - 1) / splits;
         }
         splits = (nchunk + cps - 1) / cps;
-        const int x_bytes = (cps * bpc * kXHalfPitch + 127) & ~127;
-        int depth = (smem_optin - x_bytes - misc) / (warps * sb);
+        const int x_bytes = (cps * kFxBPC * stage + 127) & ~127;
+        int depth = (smem_optin - x_bytes - misc) / (warps * kFxSlotBytes);
         if (depth > 4)
             depth = 4;
         if (depth < 2)
@@ -646,9 +911,8 @@ static Q4KPlan q4k_plan_half(long long N, int nb, int NS, int sm_count, int smem
         const long long max_ctas = sm_count / splits > 0 ? sm_count / splits : 1;
         if (ctas > max_ctas)
             ctas = max_ctas;
-        pl.half = true;
-        pl.lpr = lpr;
-        pl.R = 2;
+        pl.tma = tma;
+        pl.R = kFxRows;
         pl.warps = warps;
         pl.tiles = tiles;
         pl.splits = splits;
@@ -656,147 +920,112 @@ static Q4KPlan q4k_plan_half(long long N, int nb, int NS, int sm_count, int smem
         pl.depth = depth;
         pl.ctas_per_split = static_cast<int>(ctas);
         pl.grid = pl.ctas_per_split * splits;
-        pl.smem = x_bytes + ((warps * depth * 8 + 127) & ~127) + warps * depth * sb + 256;
+        pl.smem = x_bytes + ((warps * depth * 8 + 127) & ~127) + 128 + warps * depth * kFxSlotBytes + 256;
+        // batch-1 splits of at most one tile per warp are added inside a cluster
+        pl.cluster = B == 1 && splits > 1 && splits <= kFxMaxCluster &&
+                     tiles <= static_cast<long long>(pl.ctas_per_split) * warps &&
+                     pl.smem + warps * kFxClusterPartBytes <= smem_optin;
+        if (pl.cluster)
+            pl.smem += warps * kFxClusterPartBytes;
         pl.ok = pl.smem <= smem_optin;
     }
     return pl;
 }
 
-// Full-block plan of the fp32 kernel: `stage_bytes` is the shared memory the
-// staged activations take per super-block.
-static Q4KPlan plan_full_block(long long N, int nb, int NS, int sm_count, int smem_optin, int stage_bytes)
+// Describes one weight matrix to the TMA unit as [N][row bytes / 4] 32-bit words
+// with a box of one slot: 16 rows x (576 + 16) bytes.
+static cudaError_t encode_weight_map(CUtensorMap *m, const uint8_t *w, long long N, int nb)
 {
-    Q4KPlan pl{};
-    const int misc = 256 /*argmax scratch, 16 B per warp*/ + 256 /*barriers*/;
-    // 16-block chunks when they tile the row, else 4-block chunks (both start
-    // at SoA group boundaries)
-    const int lpr_opts[2] = {(nb % 16 == 0) ? 16 : 4, 4};
-    const int n_opts = (nb % 16 != 0) ? 1 : 2;
-    for (int oi = 0; oi < n_opts && !pl.ok; ++oi) {
-        const int lpr = lpr_opts[oi];
-        const int R = 2;
-        const int sb = q4k_slot_bytes(lpr);
-        const int TR = (32 / lpr) * R;
-        const long long tiles = (N + TR - 1) / TR;
-        const int nchunk = (nb + lpr - 1) / lpr;
-        const int w0 = q4k_pick_warps(tiles, sm_count, kMaxWarps, false);
-        for (int warps = w0; warps >= 4 && !pl.ok; warps = (warps > 4 && warps / 2 < 4) ? 4 : warps / 2) {
-            const int min_ring = warps * 2 * sb;
-            // smallest split count whose activations fit beside a two-deep ring
-            int splits = 1;
-            int cps = nchunk;
-            for (;;) {
-                cps = (nchunk + splits - 1) / splits;
-                const int xb = cps * lpr * stage_bytes;
-                if (xb + min_ring + misc <= smem_optin || cps == 1)
-                    break;
-                ++splits;
-            }
-            // split K further while fewer than half of the warps would have a tile
-            const long long warps_total = static_cast<long long>(sm_count) * warps;
-            while (tiles * NS * splits * 2 < warps_total && splits < nchunk) {
-                ++splits;
-                cps = (nchunk + splits - 1) / splits;
-            }
-            splits = (nchunk + cps - 1) / cps;
-            const int x_bytes = (cps * lpr * stage_bytes + 127) & ~127;
-            int depth = (smem_optin - x_bytes - misc) / (warps * sb);
-            if (depth > 4)
-                depth = 4;
-            if (depth < 2)
-                continue;
-            long long ctas = (tiles + warps - 1) / warps;
-            const long long max_ctas = sm_count / splits > 0 ? sm_count / splits : 1;
-            if (ctas > max_ctas)
-                ctas = max_ctas;
-            pl.lpr = lpr;
-            pl.R = R;
-            pl.warps = warps;
-            pl.tiles = tiles;
-            pl.splits = splits;
-            pl.chunks_per_split = cps;
-            pl.depth = depth;
-            pl.ctas_per_split = static_cast<int>(ctas);
-            pl.grid = pl.ctas_per_split * splits;
-            pl.smem = x_bytes + ((warps * depth * 8 + 127) & ~127) + warps * depth * sb + 256;
-            pl.ok = pl.smem <= smem_optin;
-        }
-    }
-    return pl;
+    const cuuint64_t row = static_cast<cuuint64_t>(nb) * kQ4KBlockBytes;
+    const cuuint64_t dims[2] = {row / 4, static_cast<cuuint64_t>(N)};
+    const cuuint64_t strides[1] = {row};
+    const cuuint32_t box[2] = {kFxRowPitch / 4, kFxTileRows};
+    const cuuint32_t es[2] = {1, 1};
+    const CUresult r = tensor_map_encoder()(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint8_t *>(w), dims,
+                                            strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-Q4KPlan q4k_plan(long long N, int K, int B, int NS, int soa, int sm_count, int smem_optin)
+template <int NS, bool TMA>
+static cudaError_t launch_fx(const Q4KParams &p, const FxMaps &maps, const Q4KPlan &pl, cudaStream_t s)
 {
-    const int nb = K / kQ4KBlockElems;
-    // quarter-warp lanes with TMA slots: integer dot products on fixed-point
-    // activations at batch 1, exact fp32 weights at batch 2..8
-    const Q4KPlan pf = q4k_plan_fx(N, nb, B, NS, sm_count, smem_optin);
-    if (pf.ok)
-        return pf;
-    if (B == 1) {
-        // Half-block lanes halve each warp's serial chain of slots (better when
-        // every warp gets only a few slots); full-block lanes spend fewer
-        // instructions per weight (better for long matrices).
-        const int full_lpr = (nb % 16 == 0) ? 16 : 4;
-        const long long full_tiles = (N + (32 / full_lpr) * 2 - 1) / ((32 / full_lpr) * 2);
-        const long long slots = full_tiles * NS * ((nb + full_lpr - 1) / full_lpr);
-        if (slots < 8LL * sm_count * kMaxWarps) {
-            const Q4KPlan ph = q4k_plan_half(N, nb, NS, sm_count, smem_optin);
-            if (ph.ok)
-                return ph;
-        }
-    }
-    return plan_full_block(N, nb, NS, sm_count, smem_optin, B * kXBlockPitch);
-}
-
-template <int LPR, int B, int NS>
-static cudaError_t launch_one(const Q4KParams &p, const Q4KPlan &pl, cudaStream_t s)
-{
-    auto k = p.soa ? q4k_gemv_kernel<LPR, B, NS, true> : q4k_gemv_kernel<LPR, B, NS, false>;
+    auto k = p.soa ? q4k_gemv_fx_kernel<NS, true, TMA> : q4k_gemv_fx_kernel<NS, false, TMA>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
     if (e != cudaSuccess)
         return e;
-    return launch_pdl(k, dim3(pl.grid), dim3(pl.warps * 32), pl.smem, s, p);
+    if (!pl.cluster)
+        return launch_pdl(k, dim3(pl.grid), dim3(pl.warps * 32), pl.smem, s, p, maps);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(pl.grid);
+    cfg.blockDim = dim3(pl.warps * 32);
+    cfg.dynamicSmemBytes = pl.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = pl.splits;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, k, p, maps);
 }
 
-template <int LPR, int NS>
-static cudaError_t launch_b(const Q4KParams &p, const Q4KPlan &pl, int B, cudaStream_t s)
+template <int B, int NS, bool TMA>
+static cudaError_t launch_fxb(const Q4KParams &p, const FxMaps &maps, const Q4KPlan &pl, cudaStream_t s)
+{
+    auto k = p.soa ? q4k_gemv_fxb_kernel<B, NS, true, TMA> : q4k_gemv_fxb_kernel<B, NS, false, TMA>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
+    if (e != cudaSuccess)
+        return e;
+    return launch_pdl(k, dim3(pl.grid), dim3(pl.warps * 32), pl.smem, s, p, maps);
+}
+
+template <int NS, bool TMA>
+static cudaError_t launch_fx_b(const Q4KParams &p, const FxMaps &maps, const Q4KPlan &pl, int B, cudaStream_t s)
 {
     switch (B) {
-    case 1: return launch_one<LPR, 1, NS>(p, pl, s);
-    case 2: return launch_one<LPR, 2, NS>(p, pl, s);
-    case 3: return launch_one<LPR, 3, NS>(p, pl, s);
-    case 4: return launch_one<LPR, 4, NS>(p, pl, s);
-    case 5: return launch_one<LPR, 5, NS>(p, pl, s);
-    case 6: return launch_one<LPR, 6, NS>(p, pl, s);
-    case 7: return launch_one<LPR, 7, NS>(p, pl, s);
-    case 8: return launch_one<LPR, 8, NS>(p, pl, s);
+    case 1: return launch_fx<NS, TMA>(p, maps, pl, s);
+    case 2: return launch_fxb<2, NS, TMA>(p, maps, pl, s);
+    case 3: return launch_fxb<3, NS, TMA>(p, maps, pl, s);
+    case 4: return launch_fxb<4, NS, TMA>(p, maps, pl, s);
+    case 5: return launch_fxb<5, NS, TMA>(p, maps, pl, s);
+    case 6: return launch_fxb<6, NS, TMA>(p, maps, pl, s);
+    case 7: return launch_fxb<7, NS, TMA>(p, maps, pl, s);
+    case 8: return launch_fxb<8, NS, TMA>(p, maps, pl, s);
     default: return cudaErrorInvalidValue;
     }
 }
 
-template <int LPR, int NS>
-static cudaError_t launch_half(const Q4KParams &p, const Q4KPlan &pl, cudaStream_t s)
+Q4KPlan q4k_plan(long long N, int K, int B, int NS, int soa, int sm_count, int smem_optin)
 {
-    auto k = p.soa ? q4k_gemv_b1_kernel<LPR, NS, true> : q4k_gemv_b1_kernel<LPR, NS, false>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
-    if (e != cudaSuccess)
-        return e;
-    return launch_pdl(k, dim3(pl.grid), dim3(pl.warps * 32), pl.smem, s, p);
+    (void)soa;   // both layouts move 4-block chunks as one contiguous span per row
+    return plan_quarter_warp(N, K / kQ4KBlockElems, B, NS, sm_count, smem_optin);
 }
 
 cudaError_t q4k_gemv_launch(const Q4KParams &p, const Q4KPlan &pl, int B, int NS, cudaStream_t s)
 {
-    if (pl.fx)
-        return q4k_gemv_fx_launch(p, pl, B, NS, s);
-    if (pl.half) {
-        if (pl.lpr == 32)
-            return NS == 1 ? launch_half<32, 1>(p, pl, s) : launch_half<32, 2>(p, pl, s);
-        return NS == 1 ? launch_half<8, 1>(p, pl, s) : launch_half<8, 2>(p, pl, s);
+    FxMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    if (pl.tma) {
+        if (p.grp.n > 0) {
+            for (int m = 0; m < p.grp.n; ++m) {
+                const cudaError_t e = encode_weight_map(&maps.m[m], p.gw[m], p.grp.N[m], p.nb);
+                if (e != cudaSuccess)
+                    return e;
+            }
+        } else {
+            for (int st = 0; st < NS; ++st) {
+                const cudaError_t e = encode_weight_map(&maps.m[st], p.w[st], p.N, p.nb);
+                if (e != cudaSuccess)
+                    return e;
+            }
+        }
+        return NS == 1 ? launch_fx_b<1, true>(p, maps, pl, B, s) : launch_fx_b<2, true>(p, maps, pl, B, s);
     }
-    if (pl.lpr == 16)
-        return NS == 1 ? launch_b<16, 1>(p, pl, B, s) : launch_b<16, 2>(p, pl, B, s);
-    return NS == 1 ? launch_b<4, 1>(p, pl, B, s) : launch_b<4, 2>(p, pl, B, s);
+    return NS == 1 ? launch_fx_b<1, false>(p, maps, pl, B, s) : launch_fx_b<2, false>(p, maps, pl, B, s);
 }
 
 }  // namespace dq

@@ -334,9 +334,9 @@ def test_errors_launch_nothing_and_leave_the_stream_usable():
 
 @pytest.mark.parametrize("N,K", [(40000, 4096), (16000, 12288)])
 @pytest.mark.parametrize("layout", ["aos", "soa"])
-def test_q4k_gemv_long_matrices_full_block_lanes(N, K, layout):
-    # enough rows that batch 1 runs on full-block lanes (the LM-head kernel);
-    # the smaller shapes above run on half-block lanes
+def test_q4k_gemv_long_matrices(N, K, layout):
+    # enough rows that batch 1 runs without K splits, several tiles per warp
+    # (the LM-head plan); the smaller shapes above split K
     rng = np.random.default_rng(N + K)
     w = synth.q4k_matrix(rng, N, K)
     x = synth.activations(rng, 1, K)
