@@ -84,6 +84,12 @@ def activations(rng: np.random.Generator, B: int, K: int, scale: float = 1.0) ->
     return x
 
 
+def activations_f16(rng: np.random.Generator, M: int, K: int, scale: float = 1.0) -> np.ndarray:
+    """M x K binary16 activations (numpy float16): N(0,1) draws in fp32, times
+    `scale`, converted to the nearest binary16 value."""
+    return activations(rng, M, K, scale).astype(np.float16)
+
+
 # ---------------------------------------------------------------------------
 # Named workloads: the five decode shapes the library is measured on.
 # ---------------------------------------------------------------------------

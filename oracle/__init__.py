@@ -71,9 +71,17 @@ def _load():
             lib.oracle_argmax.argtypes = [p, i64]
             lib.oracle_split_qg.argtypes = [p, i64, i64, i64, p, p]
             lib.oracle_argmax.restype = i64
+            lib.oracle_float_to_fp16.argtypes = [ctypes.c_float]
+            lib.oracle_float_to_fp16.restype = ctypes.c_uint16
+            lib.oracle_float_to_fp16_array.argtypes = [p, i64, p]
+            lib.oracle_float_to_fp16_array.restype = None
+            lib.oracle_q4k_dequant_f16.argtypes = [p, ctypes.c_int, i64, i64, p]
+            lib.oracle_q4k_prefill_rows.argtypes = [p, ctypes.c_int, i64, i64, p, i64, p, i64,
+                                                    p, p]
             for name in ("oracle_q4k_repack_soa", "oracle_q8_0_dequant", "oracle_q4k_dequant",
                          "oracle_q4k_dequant_f32", "oracle_q8_0_dequant_f32",
-                         "oracle_q4k_gemv_rows", "oracle_q8_0_gemv_rows", "oracle_split_qg"):
+                         "oracle_q4k_gemv_rows", "oracle_q8_0_gemv_rows", "oracle_split_qg",
+                         "oracle_q4k_dequant_f16", "oracle_q4k_prefill_rows"):
                 getattr(lib, name).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -246,6 +254,50 @@ def split_qg(y, head_dim: int):
     g = np.empty((B, N // 2), np.float64)
     _check(_load().oracle_split_qg(_ptr(y2), B, N, head_dim, _ptr(q), _ptr(g)), "split_qg")
     return q, g
+
+
+# --- W4A16 prefill ------------------------------------------------------------
+
+def float_to_fp16(f) -> np.ndarray:
+    """fp32 values -> binary16 bit patterns (uint16), round to nearest even."""
+    f = np.ascontiguousarray(np.asarray(f, dtype=np.float32))
+    out = np.empty(f.shape, np.uint16)
+    _load().oracle_float_to_fp16_array(_ptr(f), f.size, _ptr(out))
+    return out
+
+
+def q4k_dequant_f16(w, N: int, K: int, layout: str = "aos") -> np.ndarray:
+    """N x K binary16 bit patterns of the weights rounded to fp32, then to fp16."""
+    w = _u8(w)
+    out = np.empty((N, K), np.uint16)
+    _check(_load().oracle_q4k_dequant_f16(_ptr(w), _layout_flag(layout), N, K, _ptr(out)),
+           "q4k_dequant_f16")
+    return out
+
+
+def q4k_prefill(w, N: int, K: int, x16, rows=None, layout: str = "aos"):
+    """W4A16 prefill: y, A (each M x nrows, float64) for x16 an M x K array of
+    binary16 bit patterns (uint16) or of float16 values; qualiaDB
+    qwen3_attention, prefill_weights (W4A16 M128 dispatcher)."""
+    w = _u8(w)
+    x16 = np.asarray(x16)
+    if x16.dtype == np.float16:
+        x16 = x16.view(np.uint16)
+    if x16.dtype != np.uint16:
+        raise TypeError("x16 must hold binary16 bit patterns (uint16) or float16 values")
+    x16 = np.ascontiguousarray(x16)
+    if x16.ndim == 1:
+        x16 = x16.reshape(1, -1)
+    if x16.shape[1] != K:
+        raise ValueError("x16 must have K columns")
+    rows = _rows_arg(rows, N)
+    M = x16.shape[0]
+    y = np.empty((M, rows.size), np.float64)
+    a = np.empty((M, rows.size), np.float64)
+    _check(_load().oracle_q4k_prefill_rows(_ptr(w), _layout_flag(layout), N, K, _ptr(x16), M,
+                                           _ptr(rows), rows.size, _ptr(y), _ptr(a)),
+           "q4k_prefill")
+    return y, a
 
 
 # --- tolerance rules ----------------------------------------------------------

@@ -375,3 +375,116 @@ int64_t oracle_argmax(const double *v, int64_t n)
             best = i;
     return best;
 }
+
+/* ------------------------------------------------------------------------ */
+/* W4A16 prefill: Y = X W^T with 16-bit operands (qualiaDB qwen3_attention: */
+/* prefill_weights, "W4A16 M128 dispatcher").  The pages name the operation */
+/* and its operand widths only; the reading taken here:                     */
+/*   - activations X (M x K) are IEEE binary16 values, given as bit         */
+/*     patterns;                                                            */
+/*   - each weight is the Q4_K weight rounded once to fp32 (as in           */
+/*     oracle_q4k_dequant_f32) and then to binary16, both round to nearest, */
+/*     ties to even;                                                        */
+/*   - Y (M x N) is the exact sum of those products (every product of two   */
+/*     binary16 values is exact in double; the double sum is the oracle).   */
+/* ------------------------------------------------------------------------ */
+
+/* fp32 -> IEEE binary16 bit pattern, round to nearest, ties to even.
+ * binary16 has an 11-bit significand; normal values are m * 2^(E-10) with
+ * 1024 <= m < 2048 and -14 <= E <= 15, subnormals m * 2^-24 with m < 1024.
+ * |f| >= 65520 (half-way between the largest finite value 65504 and 2^16)
+ * rounds to infinity.  NaN gives the quiet NaN 0x7E00 with f's sign. */
+uint16_t oracle_float_to_fp16(float f)
+{
+    double v = (double)f;
+    uint16_t sign = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (isnan(v))
+        return (uint16_t)(sign | 0x7E00);
+    if (a >= 65520.0)
+        return (uint16_t)(sign | 0x7C00);
+    if (a < ldexp(1.0, -14)) {
+        /* subnormal (or zero): m = a / 2^-24 rounded; m == 1024 is 2^-14 */
+        double m = nearbyint(ldexp(a, 24));
+        return (uint16_t)(sign | (uint16_t)m);
+    }
+    int ex;
+    frexp(a, &ex);              /* a = fr * 2^ex, 0.5 <= fr < 1 */
+    int E = ex - 1;             /* 2^E <= a < 2^(E+1) */
+    double m = nearbyint(ldexp(a, 10 - E));   /* in [1024, 2048] */
+    if (m == 2048.0) {
+        m = 1024.0;
+        E += 1;
+    }
+    /* E <= 15 here: a < 65520 rounds to at most 65504 = 2047 * 2^5 */
+    return (uint16_t)(sign | (uint16_t)((E + 15) << 10) | (uint16_t)(m - 1024.0));
+}
+
+void oracle_float_to_fp16_array(const float *f, int64_t n, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = oracle_float_to_fp16(f[i]);
+}
+
+/* Q4_K matrix -> binary16 weights (N x K bit patterns), as defined above. */
+int oracle_q4k_dequant_f16(const uint8_t *w, int soa, int64_t N, int64_t K, uint16_t *out)
+{
+    if (N < 0 || K < 0 || K % Q4K_BLOCK_ELEMS != 0)
+        return -1;
+    int64_t nb = K / Q4K_BLOCK_ELEMS;
+    uint8_t blk[Q4K_BLOCK_BYTES];
+    double tmp[Q4K_BLOCK_ELEMS];
+    for (int64_t n = 0; n < N; ++n) {
+        const uint8_t *row = w + n * nb * Q4K_BLOCK_BYTES;
+        for (int64_t kb = 0; kb < nb; ++kb) {
+            gather_q4k_block(row, nb, kb, soa, blk);
+            oracle_q4k_block(blk, tmp);
+            for (int i = 0; i < Q4K_BLOCK_ELEMS; ++i)
+                out[n * K + kb * Q4K_BLOCK_ELEMS + i] = oracle_float_to_fp16((float)tmp[i]);
+        }
+    }
+    return 0;
+}
+
+/* Prefill product on a list of weight rows.  x16 is M x K binary16 bit
+ * patterns (row-major); y and a are M x nrows (row-major):
+ *   y[m][r] = sum_k W16[rows[r]][k] * X16[m][k]      (double accumulation)
+ *   a[m][r] = sum_k |W16[rows[r]][k] * X16[m][k]|                           */
+int oracle_q4k_prefill_rows(const uint8_t *w, int soa, int64_t N, int64_t K,
+                            const uint16_t *x16, int64_t M, const int64_t *rows, int64_t nrows,
+                            double *y, double *a)
+{
+    if (N < 0 || K < 0 || K % Q4K_BLOCK_ELEMS != 0 || M < 1)
+        return -1;
+    int64_t nb = K / Q4K_BLOCK_ELEMS;
+    uint8_t blk[Q4K_BLOCK_BYTES];
+    double wv[Q4K_BLOCK_ELEMS];
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t n = rows[r];
+        if (n < 0 || n >= N)
+            return -2;
+        for (int64_t m = 0; m < M; ++m) {
+            y[m * nrows + r] = 0.0;
+            a[m * nrows + r] = 0.0;
+        }
+        const uint8_t *row = w + n * nb * Q4K_BLOCK_BYTES;
+        for (int64_t kb = 0; kb < nb; ++kb) {
+            gather_q4k_block(row, nb, kb, soa, blk);
+            oracle_q4k_block(blk, wv);
+            for (int i = 0; i < Q4K_BLOCK_ELEMS; ++i)
+                wv[i] = oracle_fp16_to_double(oracle_float_to_fp16((float)wv[i]));
+            for (int64_t m = 0; m < M; ++m) {
+                const uint16_t *xm = x16 + m * K + kb * Q4K_BLOCK_ELEMS;
+                double sy = 0.0, sa = 0.0;
+                for (int i = 0; i < Q4K_BLOCK_ELEMS; ++i) {
+                    double p = wv[i] * oracle_fp16_to_double(xm[i]);
+                    sy += p;
+                    sa += fabs(p);
+                }
+                y[m * nrows + r] += sy;
+                a[m * nrows + r] += sa;
+            }
+        }
+    }
+    return 0;
+}

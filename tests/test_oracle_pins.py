@@ -355,3 +355,101 @@ def test_split_qg_is_a_per_row_permutation_inverted_by_interleaving():
 def test_split_qg_rejects_rows_that_are_not_whole_heads():
     with pytest.raises(Exception):
         oracle.split_qg(np.zeros((1, 12)), 4)
+
+
+# --- W4A16 prefill ------------------------------------------------------------------
+
+def _fp16_midpoints():
+    """Every finite positive binary16 value, the midpoints between neighbours
+    (exact in fp32) and the fp32 values one ulp either side of each midpoint."""
+    pats = np.arange(0x7C00, dtype=np.uint16)
+    vals = pats.view(np.float16).astype(np.float32)
+    mids = ((vals[:-1].astype(np.float64) + vals[1:].astype(np.float64)) / 2).astype(np.float32)
+    assert np.all(mids.astype(np.float64) == (vals[:-1].astype(np.float64) + vals[1:]) / 2)
+    up = np.nextafter(mids, np.float32(np.inf))
+    down = np.nextafter(mids, np.float32(0))
+    return np.concatenate([vals, mids, up, down, np.float32([65504, 65519.996, 65520, 65536, 1e30])])
+
+
+def test_fp16_rounding_matches_numpy_on_values_midpoints_and_random_floats():
+    rng = np.random.default_rng(11)
+    rnd = (rng.standard_normal(400000) * np.exp2(rng.integers(-30, 18, 400000))).astype(np.float32)
+    f = np.concatenate([_fp16_midpoints(), rnd, np.float32([0.0, np.inf, np.nan])])
+    f = np.concatenate([f, -f])
+    got = oracle.float_to_fp16(f)
+    with np.errstate(over="ignore"):
+        ref = f.astype(np.float16).view(np.uint16)
+    nan = np.isnan(f)
+    assert np.array_equal(got[~nan], ref[~nan])
+    assert np.all((got[nan] & 0x7C00) == 0x7C00) and np.all((got[nan] & 0x3FF) != 0)
+
+
+def test_fp16_rounding_hand_worked_ties():
+    # 1 + 2^-11 is half-way between 1 and 1 + 2^-10: ties to the even significand (1.0);
+    # 1 + 3*2^-11 is half-way between 1 + 2^-10 and 1 + 2^-9: ties up to 1 + 2^-9.
+    one = 0x3C00
+    got = oracle.float_to_fp16(np.float32([1 + 2.0 ** -11, 1 + 3 * 2.0 ** -11, 2.0 ** -25,
+                                           3 * 2.0 ** -25, 65519.0, 65520.0]))
+    assert list(got) == [one, one + 2, 0x0000, 0x0002, 0x7BFF, 0x7C00]
+
+
+def test_q4k_dequant_f16_is_the_fp32_weight_rounded_to_binary16():
+    rng = np.random.default_rng(12)
+    N, K = 5, 768
+    w = synth.q4k_matrix(rng, N, K)
+    got = oracle.q4k_dequant_f16(w, N, K)
+    ref = oracle.q4k_dequant_f32(w, N, K).astype(np.float16).view(np.uint16)
+    assert np.array_equal(got, ref)
+    soa = oracle.q4k_repack_soa(w, N, K)
+    assert np.array_equal(oracle.q4k_dequant_f16(soa, N, K, layout="soa"), got)
+
+
+def test_q4k_prefill_hand_worked_weight_rounding():
+    # d = 1 + 2^-10 (0x3C01), scale 63, q 15, min 0: w = 945 * (1 + 2^-10) = 945.9228515625,
+    # exact in fp32; binary16 spacing in [512, 1024) is 0.5, so W16 = 946.  With x = 1 at
+    # that weight and 0 elsewhere the prefill result is 946 (the exact GEMV gives 945.92...).
+    blk = np.zeros(144, np.uint8)
+    blk[0:2] = [0x01, 0x3C]
+    blk[4] = 63                              # sub-block 0: scale 63, min 0
+    blk[16] = 0x0F                           # weight 0: q = 15
+    w = blk.reshape(1, 144)
+    x16 = np.zeros((1, 256), np.float16)
+    x16[0, 0] = 1.0
+    y, a = oracle.q4k_prefill(w, 1, 256, x16)
+    assert y[0, 0] == 946.0 and a[0, 0] == 946.0
+    yg, _ = oracle.q4k_gemv(w, 1, 256, x16.astype(np.float32))
+    assert yg[0, 0] == 945.9228515625
+
+
+@pytest.mark.parametrize("N,K,M", [(8, 256, 1), (3, 512, 5), (4, 768, 17)])
+def test_q4k_prefill_matches_dense_brute_force(N, K, M):
+    rng = np.random.default_rng(N * 100 + K + M)
+    w = synth.q4k_matrix(rng, N, K)
+    x16 = synth.activations_f16(rng, M, K)
+    w16 = oracle.q4k_dequant_f16(w, N, K).view(np.float16).astype(np.float64)
+    xd = x16.astype(np.float64)
+    y, a = oracle.q4k_prefill(w, N, K, x16)
+    assert y.shape == (M, N)
+    assert np.allclose(y, xd @ w16.T, rtol=1e-13, atol=1e-13)
+    assert np.allclose(a, np.abs(xd) @ np.abs(w16).T, rtol=1e-13, atol=1e-13)
+    rows = np.array([N - 1, 0])
+    ys, as_ = oracle.q4k_prefill(w, N, K, x16, rows=rows)
+    assert np.array_equal(ys, y[:, rows]) and np.array_equal(as_, a[:, rows])
+    soa = oracle.q4k_repack_soa(w, N, K)
+    assert np.array_equal(oracle.q4k_prefill(soa, N, K, x16, layout="soa")[0], y)
+
+
+def test_q4k_prefill_equals_the_gemv_when_weights_and_x_are_binary16_exact():
+    # d = 1, scale 1, min 0: every weight is its quant (exact in binary16); x is binary16, so
+    # the prefill and the fp32-input GEMV compute the same exact products.
+    N, K, M = 3, 512, 4
+    rng = np.random.default_rng(13)
+    nblk = N * K // 256
+    sc = np.array([1, 1, 1, 1, 0, 0, 0, 0, 1, 1, 1, 1], np.uint8)
+    w = synth.q4k_pack(np.ones(nblk, np.float16), np.zeros(nblk, np.float16),
+                       np.tile(sc, (nblk, 1)),
+                       rng.integers(0, 256, (nblk, 128), dtype=np.uint8)).reshape(N, -1)
+    x16 = synth.activations_f16(rng, M, K)
+    y, _ = oracle.q4k_prefill(w, N, K, x16)
+    yg, _ = oracle.q4k_gemv(w, N, K, x16.astype(np.float32))
+    assert np.array_equal(y, yg)
