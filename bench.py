@@ -273,7 +273,7 @@ def graph_table():
     torch.cuda.set_device(0)
     l2 = 126e6
 
-    def timed(name, fn, nbytes, copies, reps=20):
+    def timed(name, fn, nbytes, copies, reps=20, flops=0):
         s = torch.cuda.Stream()
         with torch.cuda.stream(s):
             for i in range(copies):
@@ -293,8 +293,11 @@ def graph_table():
         e1.record()
         torch.cuda.synchronize()
         us = e0.elapsed_time(e1) * 1e3 / (reps * copies)
-        print(json.dumps({"case": name, "us_per_call": round(us, 2), "GBps": round(nbytes / us / 1e3, 1),
-                          "bytes": nbytes, "copies": copies}), flush=True)
+        rec = {"case": name, "us_per_call": round(us, 2), "GBps": round(nbytes / us / 1e3, 1), "bytes": nbytes,
+               "copies": copies}
+        if flops:
+            rec["TFLOPs"] = round(flops / us / 1e6, 1)
+        print(json.dumps(rec), flush=True)
         del g
 
     cases = [("q4k_lmhead_248320x4096", 1, "gemv"), ("q4k_lmhead_248320x4096", 1, "argmax"),
@@ -375,6 +378,28 @@ def graph_table():
 
     nbytes = sum(m.numel() for m in mats[0]) + 4 * (KQ + H + F)
     timed("decode_step:qproj_split+swiglu+down", decode_step, nbytes, 2)
+    del mats
+    torch.cuda.empty_cache()
+
+    # W4A16 prefill on the tensor cores: M binary16 tokens through the down projection and
+    # through one gate/up matrix (bytes: weights + activations; flops: 2 M N K)
+    rng = np.random.default_rng(44)
+    for N, K in ((4096, 12288), (12288, 4096)):
+        wbytes = N * (K // 256) * 144
+        copies = max(1, int(np.ceil(1.3 * l2 / wbytes)))
+        pw = [torch.from_numpy(synth.q4k_matrix(rng, N, K)).cuda()]
+        for _ in range(1, copies):
+            pw.append(pw[0].clone())
+        for M in (16, 64, 128, 256, 512):
+            x16 = torch.from_numpy(synth.activations_f16(rng, M, K)).cuda()
+            yp = torch.empty((M, N), device="cuda")
+            scratch = torch.empty(max(1, dq.dq_workspace_bytes(dq.DQ_OP_Q4K_PREFILL, N, K, M)), dtype=torch.uint8,
+                                  device="cuda")
+            timed("prefill_%dx%d:M%d" % (N, K, M),
+                  lambda i: dq.q4k_prefill_gemm(pw[i], x16, N, K, y=yp, workspace=scratch),
+                  wbytes + 2 * M * K, copies, flops=2 * M * N * K)
+        del pw
+        torch.cuda.empty_cache()
 
 
 def main():

@@ -25,6 +25,8 @@ DQ_LAYOUT_SOA = 1
 DQ_OP_Q8_0_GEMV = 0
 DQ_OP_Q4K_GEMV = 1
 DQ_OP_Q4K_SWIGLU = 2
+DQ_OP_Q4K_PREFILL = 3
+MAX_PREFILL_M = 65536
 
 Q4K_BLOCK_ELEMS, Q4K_BLOCK_BYTES = 256, 144
 Q8_0_BLOCK_ELEMS, Q8_0_BLOCK_BYTES = 32, 34
@@ -32,7 +34,7 @@ Q8_0_BLOCK_ELEMS, Q8_0_BLOCK_BYTES = 32, 34
 EXPORTED = ("q8_0_gemv", "q4k_gemv", "q4k_swiglu_gemv", "q4k_repack_soa", "dq_workspace_bytes",
             "q8_0_dequant", "q4k_dequant", "dq_status_string", "dq_last_cuda_error",
             "dq_device_error", "q4k_gemv_noalloc", "dq_noalloc_scratch_bytes", "q4k_gemv_split_qg",
-            "q4k_gemv_group")
+            "q4k_gemv_group", "q4k_prefill_gemm")
 
 
 class DQError(RuntimeError):
@@ -74,6 +76,7 @@ def load_library(path: str = LIB_PATH):
             "q4k_gemv_noalloc": [p, i32, p, p, i64, i64, i32, p, p],
             "q4k_gemv_split_qg": [p, i32, p, p, p, i64, i64, i32, i64, p, sz, p],
             "q4k_gemv_group": [i32, p, p, p, i32, p, i64, p, sz, p],
+            "q4k_prefill_gemm": [p, i32, p, p, i64, i64, i64, p, sz, p],
         }
         for name, args in sigs.items():
             f = getattr(lib, name)
@@ -264,6 +267,28 @@ def q4k_gemv_split_qg(w, x, N: int, K: int, head_dim: int, layout="aos", q=None,
     if one_d:
         return q.view(half), g.view(half)
     return q.view(B, half), g.view(B, half)
+
+
+def q4k_prefill_gemm(w, x16, N: int, K: int, layout="aos", y=None, workspace=None, stream=None):
+    """W4A16 prefill: y (M, N) fp32 = x16 (M, K) binary16 times the binary16
+    rounding of the Q4_K matrix w (N x K), transposed, on the tensor cores."""
+    torch = _torch()
+    lib = load_library()
+    if x16.dim() != 2 or x16.shape[1] != K:
+        raise ValueError("x16 must be (M, K)")
+    M = x16.shape[0]
+    xp = _dev(x16, "x16", torch.float16)
+    wp = _weights(w, "w", N, K, Q4K_BLOCK_ELEMS, Q4K_BLOCK_BYTES)
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=x16.device)
+    yp = _dev(y, "y", torch.float32)
+    if y.numel() != M * N:
+        raise ValueError("y must hold M*N floats")
+    need = dq_workspace_bytes(DQ_OP_Q4K_PREFILL, N, K, M)
+    wsp, wsn, _keep = _workspace(workspace, need, x16.device)
+    _check("q4k_prefill_gemm", lib.q4k_prefill_gemm(wp, _layout(layout), xp, yp, N, K, M, wsp, wsn,
+                                                    _stream(stream)))
+    return y.view(M, N)
 
 
 MAX_GROUP = 4

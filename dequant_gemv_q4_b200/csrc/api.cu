@@ -84,6 +84,18 @@ dq_status check_q4k_shape(int64_t N, int64_t K, int B)
     return DQ_OK;
 }
 
+dq_status check_prefill_shape(int64_t N, int64_t K, int64_t M)
+{
+    if (N < 1 || N > 0x7FFFFFFFLL || K < 256 || K % 256 != 0 || K > DQ_MAX_K || M < 1 || M > DQ_MAX_PREFILL_M)
+        return DQ_ERR_SHAPE;
+    return DQ_OK;
+}
+
+size_t prefill_ws_bytes(const dq::PrefillPlan &pl, int64_t N, int64_t M)
+{
+    return pl.splits > 1 ? round_up(static_cast<size_t>(pl.splits) * M * N * sizeof(float), 256) : 0;
+}
+
 dq_status q4k_common(const void *w0, const void *w1, int layout, const float *x, float *y, int64_t N, int64_t K,
                      int B, int NS, int64_t *argmax_out, void *workspace, size_t ws_bytes, void *stream,
                      float *g_out = nullptr, int64_t qg_hd = 0, const dq::GroupOut *grp = nullptr,
@@ -221,6 +233,38 @@ dq_status q4k_gemv(const void *w, int layout, const float *x, float *y, int64_t 
     return q4k_common(w, nullptr, layout, x, y, N, K, B, 1, argmax_out, workspace, ws_bytes, stream);
 }
 
+dq_status q4k_prefill_gemm(const void *w, int layout, const uint16_t *x16, float *y, int64_t N, int64_t K, int64_t M,
+                           void *workspace, size_t ws_bytes, void *stream)
+{
+    if (!w || !x16 || !y)
+        return DQ_ERR_NULL;
+    if (layout != DQ_LAYOUT_AOS && layout != DQ_LAYOUT_SOA)
+        return DQ_ERR_LAYOUT;
+    dq_status st = check_prefill_shape(N, K, M);
+    if (st != DQ_OK)
+        return st;
+    if (!aligned(w, 16) || !aligned(x16, 16) || !aligned(y, 16))
+        return DQ_ERR_ALIGN;
+    DevInfo di;
+    st = dev_info(di);
+    if (st != DQ_OK)
+        return st;
+    if (!dq::tensor_map_encoder())
+        return cuda_fail(cudaErrorNotSupported);
+    const dq::PrefillPlan pl = dq::q4k_prefill_plan(N, static_cast<int>(K), M, di.sm_count, di.smem_optin);
+    if (!pl.ok)
+        return DQ_ERR_SHAPE;
+    const size_t need = prefill_ws_bytes(pl, N, M);
+    if (need > 0 && (!workspace || ws_bytes < need))
+        return DQ_ERR_WORKSPACE;
+    if (need > 0 && !aligned(workspace, 16))
+        return DQ_ERR_ALIGN;
+    const cudaError_t e = dq::q4k_prefill_launch(static_cast<const uint8_t *>(w), layout == DQ_LAYOUT_SOA, x16, y,
+                                                 static_cast<float *>(workspace), dq::device_error_flag(di.device), N,
+                                                 static_cast<int>(K), M, pl, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DQ_OK : cuda_fail(e);
+}
+
 dq_status q4k_gemv_split_qg(const void *w, int layout, const float *x, float *q, float *g, int64_t N, int64_t K,
                             int B, int64_t head_dim, void *workspace, size_t ws_bytes, void *stream)
 {
@@ -327,6 +371,15 @@ dq_status q4k_repack_soa(const void *w_aos, void *w_soa, int64_t N, int64_t K, v
 size_t dq_workspace_bytes(int op, int64_t N, int64_t K, int B, int with_argmax)
 {
     const size_t bad = static_cast<size_t>(-1);
+    if (op == DQ_OP_Q4K_PREFILL) {
+        if (with_argmax || check_prefill_shape(N, K, B) != DQ_OK)
+            return bad;
+        DevInfo di;
+        if (dev_info(di) != DQ_OK)
+            return bad;
+        const dq::PrefillPlan pl = dq::q4k_prefill_plan(N, static_cast<int>(K), B, di.sm_count, di.smem_optin);
+        return pl.ok ? prefill_ws_bytes(pl, N, B) : bad;
+    }
     if (op == DQ_OP_Q8_0_GEMV) {
         if (N < 1 || K < 32 || K % 32 != 0 || K > DQ_MAX_K || B < 1 || B > 8 || with_argmax)
             return bad;

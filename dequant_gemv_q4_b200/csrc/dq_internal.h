@@ -4,6 +4,8 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 namespace dq {
@@ -95,6 +97,27 @@ cudaError_t argmax_finalize_launch(const ArgmaxCand *cand, int ncand, long long 
 cudaError_t q4k_dequant_launch(const uint8_t *w, int soa, float *out, long long N, int K, cudaStream_t s);
 cudaError_t q8_0_dequant_launch(const uint8_t *w, float *out, long long N, int K, cudaStream_t s);
 cudaError_t q4k_repack_soa_launch(const uint8_t *aos, uint8_t *soa, long long N, int K, cudaStream_t s);
+
+// The driver's tensor-map encoder, looked up once (null when unavailable).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+
+// W4A16 prefill (tcgen05): Y = X W^T, X binary16, W Q4_K
+struct PrefillPlan {
+    bool ok;
+    int T;                 // tokens per tile (MMA N), multiple of 16, <= 256
+    int mtiles;            // token tiles
+    int ntiles;            // 128-row weight tiles
+    int splits;            // K splits (partials reduced by a second kernel when > 1)
+    int sb_per_split;      // super-blocks per split
+    int raw_depth;         // raw weight stages
+    int ab_depth;          // binary16 operand stages
+    int tmem_cols;         // tensor-memory columns allocated per CTA
+    int grid;
+    int smem;
+};
+PrefillPlan q4k_prefill_plan(long long N, int K, long long M, int sm_count, int smem_optin);
+cudaError_t q4k_prefill_launch(const uint8_t *w, int soa, const uint16_t *x16, float *y, float *part, int *err,
+                               long long N, int K, long long M, const PrefillPlan &pl, cudaStream_t s);
 
 // device error flag
 int *device_error_flag(int device);

@@ -854,7 +854,7 @@ static int pick_warps(long long tiles, int sm_count, int max_warps)
 }
 
 // The driver's tensor-map encoder, looked up once (null when unavailable).
-static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static std::once_flag once;

@@ -1,0 +1,589 @@
+// q4k_prefill.cu -- W4A16 prefill GEMM for sm_100a: Y (M x N, fp32) = X (M x K,
+// binary16) * W^T, with W an N x K Q4_K matrix, on the fifth-generation tensor
+// cores (tcgen05.mma, accumulators in tensor memory).
+//
+// The operation is the pages' batched-prefill projection with 4-bit weights and
+// 16-bit activations (qualiaDB qwen3_attention: prefill_weights, "W4A16 M128
+// dispatcher"); the pages give no more than its name and operand widths.  The
+// reading taken: each weight is the Q4_K weight rounded to fp32 (the same value
+// the dequantize entry point produces) and then to binary16, and the products
+// of those binary16 weights with the binary16 activations are summed.
+//
+// Work decomposition.  A CTA owns a tile of 128 weight rows (the MMA's M) by T
+// tokens (the MMA's N, a multiple of 16, at most 256) and a range of K.  Per
+// super-block the raw bytes of the 128 rows (18 KB) arrive by one TMA tile copy.
+// Eight dequantizing warps turn each quarter super-block (64 weights per row)
+// into a 128 x 64 binary16 tile in the tensor cores' K-major, 128-byte swizzled
+// shared-memory layout, while the activation tile of the same 64 columns
+// arrives by TMA in that same layout.  One thread issues four 128 x T x 16 MMAs
+// per stage into a T-column fp32 accumulator in tensor memory and, through
+// tcgen05.commit, releases the stage when they have read it.  After the last
+// stage the same eight warps read the accumulator back (tcgen05.ld) and store
+// Y, or the split's partial sums when K is split across CTAs.
+//
+//   warp 0      weight TMA producer (one lane)
+//   warp 1      tensor-memory allocation, MMA issue (one lane)
+//   warp 2      activation TMA producer (one lane)
+//   warp 3      idle
+//   warps 4-11  dequantization, then the epilogue
+//
+// Dequantization of one weight: the GEMV's exact fp32 weight formation
+// (q4k_decode.cuh: the quant read in place as a subnormal, one fma with the
+// scaled d*scale and dmin*min, giving the fp32-rounded weight times 2^-64), a
+// multiplication by 2^64 (exact), and cvt.rn to binary16.  So the tensor cores
+// see exactly the binary16 rounding of the weights the dequantize entry point
+// returns.
+//
+// All waits are bounded; a wait that runs out sets the device error flag and
+// the shared abort word, every role then stops issuing work, waits (bounded)
+// for its own copies and MMAs in flight, and the tensor memory is released.
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "dq_common.cuh"
+#include "dq_internal.h"
+#include "q4k_decode.cuh"
+
+namespace dq {
+
+constexpr int kPfRows = 128;                              // weight rows per tile (MMA M)
+constexpr int kPfK = 64;                                  // K per stage: one 128-byte row of binary16
+constexpr int kPfMaxT = 256;                              // tokens per tile (MMA N) at most
+constexpr int kPfRawBytes = kPfRows * kQ4KBlockBytes;     // one super-block of 128 rows
+constexpr int kPfATileBytes = kPfRows * kPfK * 2;         // 16 KB
+constexpr int kPfWarps = 12;
+constexpr int kPfDqWarp0 = 4;                             // first dequantizing warp
+constexpr int kPfDqThreads = (kPfWarps - kPfDqWarp0) * 32;
+constexpr int kPfMaxRaw = 3;
+constexpr int kPfMaxAB = 4;
+
+struct PrefillMaps {
+    CUtensorMap w;        // raw weight rows (AoS: 2-D bytes; SoA: 5-D gather of one block)
+    CUtensorMap w_tail;   // SoA only: the last, partial group of each row
+    CUtensorMap x;        // activations, binary16, 128-byte swizzle
+};
+
+// --- tcgen05 / TMA wrappers --------------------------------------------------
+
+// Shared-memory matrix descriptor of a K-major operand tile in the 128-byte
+// swizzled layout: rows of 128 bytes, 8-row groups 1024 bytes apart (stride
+// byte offset), the leading byte offset unused for this layout (set to 16).
+__device__ __forceinline__ uint64_t pf_desc_sw128(uint32_t saddr)
+{
+    return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (static_cast<uint64_t>(16 >> 4) << 16) |
+           (static_cast<uint64_t>(1024 >> 4) << 32) | (1ull << 46) /* descriptor version */ |
+           (2ull << 61) /* 128-byte swizzle */;
+}
+
+__device__ __forceinline__ void pf_mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrives once on `bar` when every MMA this thread issued so far has completed.
+__device__ __forceinline__ void pf_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void pf_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void pf_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void pf_tma_2d(uint32_t dst, const CUtensorMap *m, int x, int y, uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            dst),
+        "l"(m), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void pf_tma_5d(uint32_t dst, const CUtensorMap *m, int c0, int c1, int c2, int c3, int c4,
+                                          uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5, "
+        "%6}], [%7];" ::"r"(dst),
+        "l"(m), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(bar)
+        : "memory");
+}
+
+// Eight consecutive fp32 accumulator columns of this warp's 32 lanes.
+__device__ __forceinline__ void pf_tmem_ld8(uint32_t taddr, float (&v)[8])
+{
+    uint32_t r[8];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+        : "r"(taddr)
+        : "memory");
+    for (int i = 0; i < 8; ++i)
+        v[i] = __uint_as_float(r[i]);
+}
+
+// Bounded wait that also gives up at once when another role has aborted.
+__device__ __forceinline__ bool pf_wait(uint32_t bar, uint32_t parity, int *err, volatile int *abort)
+{
+    if (*abort)
+        return false;
+    if (mbar_wait_bounded(bar, parity, err))
+        return true;
+    *abort = 1;
+    return false;
+}
+
+// Two fp32 values -> one binary16 pair (round to nearest even), lo in bits 0..15.
+__device__ __forceinline__ uint32_t pf_pack_f16x2(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Binary16 weights of the 16 quant bytes of one row in `qv` (bytes 32c + 16h ..
+// 32c + 16h + 15 of the super-block): lo[0..1] are the 16 low-nibble weights
+// (k = 64c + 16h + 0..15) as two 8-weight chunks, hi[0..1] the 16 high-nibble
+// weights (k = 64c + 32 + 16h + 0..15).
+__device__ __forceinline__ void pf_dequant16(uint4 qv, const ChunkScales &cs, uint4 (&lo)[2], uint4 (&hi)[2])
+{
+    const float2 up = make_float2(0x1p64f, 0x1p64f);   // q4_word_weights forms w * 2^-64
+    const uint32_t words[4] = {qv.x, qv.y, qv.z, qv.w};
+    uint32_t plo[8], phi[8];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        float2 wv[4];   // {lo, hi} weights of bytes 4t .. 4t+3
+        q4_word_weights(words[t], cs, wv);
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+            wv[b] = __fmul2_rn(wv[b], up);
+        plo[2 * t] = pf_pack_f16x2(wv[0].x, wv[1].x);
+        plo[2 * t + 1] = pf_pack_f16x2(wv[2].x, wv[3].x);
+        phi[2 * t] = pf_pack_f16x2(wv[0].y, wv[1].y);
+        phi[2 * t + 1] = pf_pack_f16x2(wv[2].y, wv[3].y);
+    }
+    lo[0] = make_uint4(plo[0], plo[1], plo[2], plo[3]);
+    lo[1] = make_uint4(plo[4], plo[5], plo[6], plo[7]);
+    hi[0] = make_uint4(phi[0], phi[1], phi[2], phi[3]);
+    hi[1] = make_uint4(phi[4], phi[5], phi[6], phi[7]);
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v)
+{
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+struct PrefillParams {
+    float *out;        // Y (splits == 1) or the partial sums [splits][M][N]
+    int *err;          // device error flag
+    long long N;
+    long long M;
+    int nb;            // super-blocks per row (K / 256)
+    int T;             // tokens per tile (MMA N)
+    int mtiles;
+    int ntiles;
+    int sb_per_split;
+    int raw_depth;
+    int ab_depth;
+    int soa;
+    int soa_full;      // complete 4-block groups per row (SoA)
+    uint32_t idesc;    // MMA instruction descriptor
+    uint32_t tmem_cols;
+};
+
+__global__ void __launch_bounds__(kPfWarps * 32, 1)
+    q4k_prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ PrefillMaps maps)
+{
+    extern __shared__ __align__(1024) uint8_t smem[];
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_abort;
+    __shared__ __align__(8) uint64_t s_bars[2 * kPfMaxRaw + 3 * kPfMaxAB + 1];
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int AD = p.ab_depth;
+    const int RD = p.raw_depth;
+    const int T = p.T;
+    const uint32_t b_bytes = static_cast<uint32_t>(T) * 128;
+
+    const uint32_t a_s = (smem_u32(smem) + 1023u) & ~1023u;        // AD x 128 x 64 binary16 weights
+    const uint32_t b_s = a_s + AD * kPfATileBytes;                  // AD x T x 64 binary16 activations
+    const uint32_t raw_s = b_s + AD * b_bytes;                      // RD x 128 rows x 144 raw bytes
+    const uint32_t raw_full = smem_u32(s_bars);
+    const uint32_t raw_empty = raw_full + 8 * kPfMaxRaw;
+    const uint32_t a_full = raw_empty + 8 * kPfMaxRaw;
+    const uint32_t b_full = a_full + 8 * kPfMaxAB;
+    const uint32_t ab_empty = b_full + 8 * kPfMaxAB;
+    const uint32_t acc_full = ab_empty + 8 * kPfMaxAB;
+
+    // tile: consecutive CTAs share one weight tile (mt fastest), then row tiles, then splits
+    const int mt = static_cast<int>(blockIdx.x % p.mtiles);
+    const int rest = static_cast<int>(blockIdx.x / p.mtiles);
+    const int nt = rest % p.ntiles;
+    const int split = rest / p.ntiles;
+    const long long row0 = static_cast<long long>(nt) * kPfRows;
+    const long long m0 = static_cast<long long>(mt) * T;
+    const int kb0 = split * p.sb_per_split;
+    const int nsb = min(p.sb_per_split, p.nb - kb0);
+    const int nst = 4 * nsb;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < RD; ++i) {
+            mbar_init(raw_full + 8 * i, 1);
+            mbar_init(raw_empty + 8 * i, kPfDqThreads);
+        }
+        for (int i = 0; i < AD; ++i) {
+            mbar_init(a_full + 8 * i, kPfDqThreads);
+            mbar_init(b_full + 8 * i, 1);
+            mbar_init(ab_empty + 8 * i, 1);
+        }
+        mbar_init(acc_full, 1);
+        s_abort = 0;
+        mbar_fence_init();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
+                     "r"(p.tmem_cols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    pf_fence_before();
+    __syncthreads();
+    pf_fence_after();
+    const uint32_t tmem = s_tmem;
+    volatile int *abort = &s_abort;
+
+    pdl_wait();
+    pdl_launch_dependents();
+
+    if (warp == 0) {
+        // ---- weight producer: one TMA tile copy per super-block of the tile's rows
+        if (lane == 0) {
+            int issued = 0;
+            for (int i = 0; i < nsb; ++i) {
+                const int s = i % RD;
+                if (i >= RD && !pf_wait(raw_empty + 8 * s, ((i / RD) & 1) ^ 1, p.err, abort))
+                    break;
+                const uint32_t bar = raw_full + 8 * s;
+                const uint32_t dst = raw_s + s * kPfRawBytes;
+                const int kb = kb0 + i;
+                mbar_arrive_expect_tx(bar, kPfRawBytes);
+                if (!p.soa)
+                    pf_tma_2d(dst, &maps.w, kb * kQ4KBlockBytes, static_cast<int>(row0), bar);   // x: 144 kb bytes
+                else if (kb < 4 * p.soa_full)
+                    pf_tma_5d(dst, &maps.w, 0, kb & 3, 0, kb >> 2, static_cast<int>(row0), bar);
+                else
+                    pf_tma_5d(dst, &maps.w_tail, 0, kb - 4 * p.soa_full, 0, 0, static_cast<int>(row0), bar);
+                ++issued;
+            }
+            for (int i = issued > RD ? issued - RD : 0; i < issued; ++i)
+                mbar_wait_bounded(raw_full + 8 * (i % RD), (i / RD) & 1, p.err);
+        }
+    } else if (warp == 2) {
+        // ---- activation producer: one TMA tile copy (T x 64, swizzled) per stage
+        if (lane == 0) {
+            int issued = 0;
+            for (int j = 0; j < nst; ++j) {
+                const int s = j % AD;
+                if (j >= AD && !pf_wait(ab_empty + 8 * s, ((j / AD) & 1) ^ 1, p.err, abort))
+                    break;
+                const uint32_t bar = b_full + 8 * s;
+                mbar_arrive_expect_tx(bar, b_bytes);
+                pf_tma_2d(b_s + s * b_bytes, &maps.x, kb0 * kQ4KBlockElems + j * kPfK, static_cast<int>(m0), bar);
+                ++issued;
+            }
+            for (int j = issued > AD ? issued - AD : 0; j < issued; ++j)
+                mbar_wait_bounded(b_full + 8 * (j % AD), (j / AD) & 1, p.err);
+        }
+    } else if (warp == 1) {
+        // ---- MMA issue: four K = 16 steps per stage into the T-column accumulator
+        if (lane == 0) {
+            for (int j = 0; j < nst; ++j) {
+                const int s = j % AD;
+                const uint32_t ph = (j / AD) & 1;
+                if (!pf_wait(a_full + 8 * s, ph, p.err, abort) || !pf_wait(b_full + 8 * s, ph, p.err, abort))
+                    break;
+                pf_fence_after();
+                const uint32_t a0 = a_s + s * kPfATileBytes;
+                const uint32_t b0 = b_s + s * b_bytes;
+#pragma unroll
+                for (int kk = 0; kk < kPfK / 16; ++kk)
+                    pf_mma_f16(tmem, pf_desc_sw128(a0 + 32 * kk), pf_desc_sw128(b0 + 32 * kk), p.idesc,
+                               (j | kk) != 0);
+                pf_commit(ab_empty + 8 * s);
+            }
+            // arrives once every MMA issued above has completed
+            pf_commit(acc_full);
+        }
+    } else if (warp >= kPfDqWarp0) {
+        // ---- dequantization: thread (q, h, lane) forms row 32q + lane, quant bytes 16h .. 16h+15 of
+        // each 32-byte chunk, into the K-major 128-byte swizzled tile (16-byte unit u of row r at
+        // position u ^ (r % 8) of the row's 128 bytes; 8-row groups 1024 bytes apart)
+        const int q = warp & 3;
+        const int h = (warp - kPfDqWarp0) >> 2;
+        const int r = 32 * q + lane;
+        const uint32_t row_off = static_cast<uint32_t>((r >> 3) * 1024 + (r & 7) * 128);
+        const int sw = r & 7;
+        bool ok = true;
+        for (int i = 0; i < nsb && ok; ++i) {
+            const int rs = i % RD;
+            if (!pf_wait(raw_full + 8 * rs, (i / RD) & 1, p.err, abort))
+                break;
+            const uint32_t raw = raw_s + rs * kPfRawBytes + r * kQ4KBlockBytes;
+            const Hdr hd = decode_hdr(lds128(raw));
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int j = 4 * i + c;
+                const int s = j % AD;
+                if (j >= AD && !pf_wait(ab_empty + 8 * s, ((j / AD) & 1) ^ 1, p.err, abort)) {
+                    ok = false;
+                    break;
+                }
+                uint4 lo[2], hi[2];
+                pf_dequant16(lds128(raw + 16 + 32 * c + 16 * h), chunk_scales(hd, c), lo, hi);
+                const uint32_t at = a_s + s * kPfATileBytes + row_off;
+                sts128(at + (((2 * h) ^ sw) << 4), lo[0]);
+                sts128(at + (((2 * h + 1) ^ sw) << 4), lo[1]);
+                sts128(at + (((4 + 2 * h) ^ sw) << 4), hi[0]);
+                sts128(at + (((5 + 2 * h) ^ sw) << 4), hi[1]);
+                fence_proxy_async_smem();   // generic-proxy stores -> visible to the tensor cores
+                mbar_arrive(a_full + 8 * s);
+            }
+            if (!ok)
+                break;
+            mbar_arrive(raw_empty + 8 * rs);
+        }
+
+        // ---- epilogue: accumulator row r (lanes 32q .. 32q+31), columns [h T/2, (h+1) T/2)
+        const bool done = mbar_wait_bounded(acc_full, 0, p.err);
+        pf_fence_after();
+        // tcgen05.ld is warp-collective: the whole warp reads, or none of it
+        if (__all_sync(0xFFFFFFFFu, done && !*abort)) {
+            const long long n = row0 + r;
+            float *out = p.out + static_cast<long long>(split) * p.M * p.N;
+            const int half = T >> 1;
+            for (int c0 = h * half; c0 < (h + 1) * half; c0 += 8) {
+                float v[8];
+                pf_tmem_ld8(tmem + (static_cast<uint32_t>(32 * q) << 16) + c0, v);
+                if (n < p.N) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const long long m = m0 + c0 + e;
+                        if (m < p.M)
+                            out[m * p.N + n] = v[e];
+                    }
+                }
+            }
+        }
+    }
+
+    pf_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        pf_fence_after();
+        // every MMA has completed once acc_full's phase 0 has (bounded; normally it has long since)
+        mbar_wait_bounded(acc_full, 0, p.err);
+        __syncwarp();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(p.tmem_cols)
+                     : "memory");
+    }
+}
+
+// Sum of the K-split partial sums, in split order: y[i] = sum_s part[s][i].
+__global__ void __launch_bounds__(256) prefill_reduce_kernel(const float *part, int splits, long long count, float *y)
+{
+    pdl_wait();
+    pdl_launch_dependents();
+    const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+    const long long first = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if ((count & 3) == 0) {
+        const long long n4 = count >> 2;
+        const float4 *p4 = reinterpret_cast<const float4 *>(part);
+        for (long long i = first; i < n4; i += stride) {
+            const float4 a = __ldg(p4 + i);
+            float ax = a.x, ay = a.y, az = a.z, aw = a.w;
+            for (int s = 1; s < splits; ++s) {
+                const float4 b = __ldg(p4 + s * n4 + i);
+                ax += b.x;
+                ay += b.y;
+                az += b.z;
+                aw += b.w;
+            }
+            reinterpret_cast<float4 *>(y)[i] = make_float4(ax, ay, az, aw);
+        }
+    } else {
+        for (long long i = first; i < count; i += stride) {
+            float a = part[i];
+            for (int s = 1; s < splits; ++s)
+                a += part[s * count + i];
+            y[i] = a;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+// Tiles of 128 weight rows by T tokens (T a multiple of 16, at most 256, the
+// tokens split evenly over ceil(M / 256) tiles); K is split so that the tiles
+// fill the SMs once (one CTA per SM: the stages take most of shared memory);
+// as many stages as fit, up to 3 raw and 4 binary16 stages.
+PrefillPlan q4k_prefill_plan(long long N, int K, long long M, int sm_count, int smem_optin)
+{
+    PrefillPlan pl{};
+    if (N < 1 || M < 1 || K < kQ4KBlockElems || K % kQ4KBlockElems != 0 || tensor_map_encoder() == nullptr)
+        return pl;
+    const int nb = K / kQ4KBlockElems;
+    const long long mtiles = (M + kPfMaxT - 1) / kPfMaxT;
+    const long long per = (M + mtiles - 1) / mtiles;
+    const int T = static_cast<int>((per + 15) / 16 * 16);
+    const long long ntiles = (N + kPfRows - 1) / kPfRows;
+    const long long tiles = ntiles * mtiles;
+    int splits = 1;
+    if (tiles < sm_count) {
+        splits = static_cast<int>(sm_count / tiles);
+        if (splits > nb)
+            splits = nb;
+    }
+    const int sbps = (nb + splits - 1) / splits;
+    splits = (nb + sbps - 1) / sbps;
+    if (tiles * splits > 0x7FFFFFFFLL)
+        return pl;
+    const int ab = kPfATileBytes + T * 128;
+    const int budget = smem_optin - 1024 /*static shared memory*/ - 1024 /*alignment of the tiles*/;
+    int ad = kPfMaxAB, rd = kPfMaxRaw;
+    while (ad * ab + rd * kPfRawBytes > budget && ad > 2)
+        --ad;
+    while (ad * ab + rd * kPfRawBytes > budget && rd > 2)
+        --rd;
+    if (ad * ab + rd * kPfRawBytes > budget)
+        return pl;
+    int cols = 32;
+    while (cols < T)
+        cols *= 2;
+    pl.T = T;
+    pl.mtiles = static_cast<int>(mtiles);
+    pl.ntiles = static_cast<int>(ntiles);
+    pl.splits = splits;
+    pl.sb_per_split = sbps;
+    pl.raw_depth = rd;
+    pl.ab_depth = ad;
+    pl.tmem_cols = cols;
+    pl.grid = static_cast<int>(tiles * splits);
+    pl.smem = 1024 + ad * ab + rd * kPfRawBytes;
+    pl.ok = true;
+    return pl;
+}
+
+static cudaError_t encode(CUtensorMap *m, CUtensorMapDataType t, cuuint32_t rank, const void *base,
+                          const cuuint64_t *dims, const cuuint64_t *strides, const cuuint32_t *box,
+                          CUtensorMapSwizzle swz)
+{
+    const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    const CUresult r = tensor_map_encoder()(m, t, rank, const_cast<void *>(base), dims, strides, box, es,
+                                            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t q4k_prefill_launch(const uint8_t *w, int soa, const uint16_t *x16, float *y, float *part, int *err,
+                               long long N, int K, long long M, const PrefillPlan &pl, cudaStream_t s)
+{
+    const int nb = K / kQ4KBlockElems;
+    const cuuint64_t row = static_cast<cuuint64_t>(nb) * kQ4KBlockBytes;
+    PrefillMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    cudaError_t e = cudaSuccess;
+    int soa_full = 0;
+    if (!soa) {
+        // raw rows as bytes: box = one super-block (144 bytes) of 128 rows
+        const cuuint64_t dims[2] = {row, static_cast<cuuint64_t>(N)};
+        const cuuint64_t strides[1] = {row};
+        const cuuint32_t box[2] = {kQ4KBlockBytes, kPfRows};
+        e = encode(&maps.w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+    } else {
+        // SoA group of g blocks: 16-byte piece u (0: header, 1..8: quant slices) of block t at
+        // 64u... = 16 g u + 16 t.  Viewed as [row][group][u][t][16 bytes], a box of one t and all
+        // nine u gathers one block back into its 144-byte AoS order.
+        soa_full = nb / kQ4KSoaGroup;
+        const cuuint32_t box[5] = {16, 1, 9, 1, kPfRows};
+        if (soa_full > 0) {
+            const cuuint64_t dims[5] = {16, kQ4KSoaGroup, 9, static_cast<cuuint64_t>(soa_full),
+                                        static_cast<cuuint64_t>(N)};
+            const cuuint64_t strides[4] = {16, 16 * kQ4KSoaGroup, kQ4KSoaGroup * kQ4KBlockBytes, row};
+            e = encode(&maps.w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, w, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+        }
+        const int g = nb - soa_full * kQ4KSoaGroup;
+        if (e == cudaSuccess && g > 0) {
+            const cuuint64_t dims[5] = {16, static_cast<cuuint64_t>(g), 9, 1, static_cast<cuuint64_t>(N)};
+            const cuuint64_t strides[4] = {16, static_cast<cuuint64_t>(16 * g),
+                                           static_cast<cuuint64_t>(g * kQ4KBlockBytes), row};
+            e = encode(&maps.w_tail, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5,
+                       w + static_cast<size_t>(soa_full) * kQ4KSoaGroup * kQ4KBlockBytes, dims, strides, box,
+                       CU_TENSOR_MAP_SWIZZLE_NONE);
+        }
+    }
+    if (e != cudaSuccess)
+        return e;
+    {
+        // activations: box of 64 binary16 (128 bytes) x T tokens, 128-byte swizzle
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+        const cuuint32_t box[2] = {kPfK, static_cast<cuuint32_t>(pl.T)};
+        e = encode(&maps.x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x16, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (e != cudaSuccess)
+            return e;
+    }
+    PrefillParams p{};
+    p.out = pl.splits > 1 ? part : y;
+    p.err = err;
+    p.N = N;
+    p.M = M;
+    p.nb = nb;
+    p.T = pl.T;
+    p.mtiles = pl.mtiles;
+    p.ntiles = pl.ntiles;
+    p.sb_per_split = pl.sb_per_split;
+    p.raw_depth = pl.raw_depth;
+    p.ab_depth = pl.ab_depth;
+    p.soa = soa;
+    p.soa_full = soa_full;
+    // kind::f16 instruction descriptor: D fp32 (bits 4-5 = 1), A and B binary16 (bits 7-9, 10-12 = 0),
+    // both K-major (bits 15, 16 = 0), N >> 3 in bits 17-22, M >> 4 in bits 24-28
+    p.idesc = (1u << 4) | (static_cast<uint32_t>(pl.T >> 3) << 17) | (static_cast<uint32_t>(kPfRows >> 4) << 24);
+    p.tmem_cols = static_cast<uint32_t>(pl.tmem_cols);
+    e = cudaFuncSetAttribute(q4k_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
+    if (e != cudaSuccess)
+        return e;
+    e = launch_pdl(q4k_prefill_kernel, dim3(pl.grid), dim3(kPfWarps * 32), pl.smem, s, p, maps);
+    if (e != cudaSuccess || pl.splits == 1)
+        return e;
+    const long long count = M * N;
+    long long blocks = (count / 4 + 255) / 256;
+    if (blocks > 4LL * 148)
+        blocks = 4LL * 148;
+    if (blocks < 1)
+        blocks = 1;
+    return launch_pdl(prefill_reduce_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s,
+                      static_cast<const float *>(part), pl.splits, count, y);
+}
+
+}  // namespace dq

@@ -82,7 +82,8 @@ typedef enum dq_layout {
 typedef enum dq_op {
     DQ_OP_Q8_0_GEMV = 0,
     DQ_OP_Q4K_GEMV = 1,
-    DQ_OP_Q4K_SWIGLU = 2
+    DQ_OP_Q4K_SWIGLU = 2,
+    DQ_OP_Q4K_PREFILL = 3   /* q4k_prefill_gemm; the `B` argument is M */
 } dq_op;
 
 /* Largest K accepted by the GEMV entry points (fp32 activations of one split
@@ -163,6 +164,30 @@ dq_status q4k_gemv_group(int count, const void *const *w, const int64_t *N, floa
 dq_status q4k_swiglu_gemv(const void *w_gate, const void *w_up, int layout, const float *x,
                           float *out, int64_t N, int64_t K, int B, void *workspace,
                           size_t ws_bytes, void *stream);
+
+/*
+ * W4A16 prefill GEMM: 4-bit weights, 16-bit activations, M tokens at once
+ * (qualiaDB qwen3_attention, prefill_weights: "W4A16 M128 dispatcher"; the
+ * pages name the operation and its operand widths, nothing more).
+ *   y[m][n] = sum_k W16[n][k] * x16[m][k],  m < M, n < N,
+ * where W16[n][k] is the Q4_K weight rounded to fp32 (exactly the value
+ * q4k_dequant returns) and then to binary16 (round to nearest even), and x16
+ * holds binary16 values.  The products are summed in fp32 on the tensor cores
+ * (K split across CTAs when there are few tiles; the splits' partial sums are
+ * then added in a fixed order, so results are deterministic).
+ *   w          N x K Q4_K matrix in `layout`, 16-byte aligned.
+ *   x16        M x K binary16 bit patterns, row-major, 16-byte aligned.
+ *   y          M x N fp32, row-major, 16-byte aligned.
+ *   N >= 1;  K a positive multiple of 256, at most DQ_MAX_K;
+ *   M in [1, DQ_MAX_PREFILL_M].
+ *   workspace  at least dq_workspace_bytes(DQ_OP_Q4K_PREFILL, N, K, M, 0) bytes.
+ * Needs the driver's tensor-map encoder; without it the call returns
+ * DQ_ERR_CUDA (dq_last_cuda_error() = cudaErrorNotSupported) and enqueues
+ * nothing.
+ */
+#define DQ_MAX_PREFILL_M 65536
+dq_status q4k_prefill_gemm(const void *w, int layout, const uint16_t *x16, float *y, int64_t N, int64_t K,
+                           int64_t M, void *workspace, size_t ws_bytes, void *stream);
 
 /*
  * Offline repack of a Q4_K matrix from GGML block order (AoS) into this

@@ -145,3 +145,20 @@ def test_group_rejects_on_host(lib):
     assert f(2, W, N, (P * 2)(A16, P((1 << 20) + 2)), 0, A16, 256, None, 0, None) == DQ_ERR_ALIGN
     assert f(2, W, N, Y, 0, A16, 100, None, 0, None) == DQ_ERR_SHAPE
     assert f(2, W, N, Y, 7, A16, 256, None, 0, None) == DQ_ERR_LAYOUT
+
+
+def test_prefill_rejects_on_host(lib):
+    f = lib.q4k_prefill_gemm
+    f.argtypes = [P, ctypes.c_int, P, P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, P, ctypes.c_size_t, P]
+    assert f(None, 0, A16, A16, 128, 256, 16, None, 0, None) == DQ_ERR_NULL
+    assert f(A16, 0, None, A16, 128, 256, 16, None, 0, None) == DQ_ERR_NULL
+    assert f(A16, 2, A16, A16, 128, 256, 16, None, 0, None) == DQ_ERR_LAYOUT
+    assert f(A16, 0, A16, A16, 128, 100, 16, None, 0, None) == DQ_ERR_SHAPE    # K not a multiple of 256
+    assert f(A16, 0, A16, A16, 0, 256, 16, None, 0, None) == DQ_ERR_SHAPE      # N < 1
+    assert f(A16, 0, A16, A16, 128, 256, 0, None, 0, None) == DQ_ERR_SHAPE     # M < 1
+    assert f(A16, 0, A16, A16, 128, 256, 65537, None, 0, None) == DQ_ERR_SHAPE
+    assert f(A16, 0, A16, P((1 << 20) + 4), 128, 256, 16, None, 0, None) == DQ_ERR_ALIGN   # y needs 16 B
+    assert f(A16, 0, A8, A16, 128, 256, 16, None, 0, None) == DQ_ERR_ALIGN
+    bad = ctypes.c_size_t(-1).value
+    assert lib.dq_workspace_bytes(3, 128, 250, 16, 0) == bad
+    assert lib.dq_workspace_bytes(3, 128, 256, 16, 1) == bad                    # no argmax

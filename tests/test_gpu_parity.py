@@ -537,3 +537,70 @@ def test_q4k_gemv_group_matches_separate_oracle_gemvs(Ns, K, layout):
         y = host(ys[m])
         y_ref, a_ref = oracle.q4k_gemv(w, n, K, x)
         assert_within(y[None, :], y_ref, a_ref, "group matrix %d" % m)
+
+
+# --- W4A16 prefill on the tensor cores ---------------------------------------------------
+# y = x16 W16^T, W16 the binary16 rounding of the fp32 weights; bar: the GEMV rule against the
+# oracle's double sum over the same binary16 operands.
+
+@pytest.mark.parametrize("N,K,M,layout", [
+    (128, 256, 1, "aos"),      # one tile, one token (16-column MMA, 15 padding columns)
+    (200, 512, 5, "aos"),      # ragged rows (128 + 72)
+    (200, 512, 5, "soa"),
+    (300, 1024, 33, "aos"),    # ragged tokens (T = 48)
+    (256, 768, 130, "soa"),    # SoA rows of 3 blocks: the partial group only
+    (130, 1280, 64, "soa"),    # SoA rows of 5 blocks: a full group and a partial one
+    (384, 512, 700, "aos"),    # three token tiles of 240
+    (1000, 2048, 256, "aos"),  # eight row tiles, K split in two
+    (64, 4096, 17, "aos"),     # one tile, K split sixteen ways
+])
+def test_q4k_prefill_matches_oracle(N, K, M, layout):
+    rng = np.random.default_rng(N + K + M)
+    w = synth.q4k_matrix(rng, N, K)
+    x16 = synth.activations_f16(rng, M, K)
+    wl = w if layout == "aos" else oracle.q4k_repack_soa(w, N, K)
+    y = host(dq.q4k_prefill_gemm(dev(wl), dev(x16), N, K, layout=layout))
+    y_ref, a_ref = oracle_rows(lambda rows: oracle.q4k_prefill(w, N, K, x16, rows=rows), N, np.arange(N))
+    assert_within(y, y_ref, a_ref, "prefill %dx%d M=%d %s" % (N, K, M, layout))
+
+
+@pytest.mark.parametrize("N,K", [(4096, 12288), (12288, 4096)])
+def test_q4k_prefill_full_size_sampled_rows(N, K):
+    # the down projection and one gate/up matrix at M = 128 tokens, in the launch
+    # configuration bench.py times; the oracle computes 96 sampled rows
+    M = 128
+    rng = np.random.default_rng(N * 7 + K)
+    w = synth.q4k_matrix(rng, N, K)
+    x16 = synth.activations_f16(rng, M, K)
+    y = host(dq.q4k_prefill_gemm(dev(w), dev(x16), N, K))
+    rows = np.unique(np.concatenate([[0, N - 1], rng.integers(0, N, 94)]))
+    y_ref, a_ref = oracle_rows(lambda rows: oracle.q4k_prefill(w, N, K, x16, rows=rows), N, rows)
+    assert_within(y[:, rows], y_ref, a_ref, "prefill %dx%d sampled" % (N, K))
+
+
+def test_q4k_prefill_exact_integer_case_is_bit_exact():
+    # d = 1, scale 1, min 0: W16 = q in [0, 15]; x small integers: every partial sum is an
+    # integer below 2^24, so the fp32 tensor-core sum is exact and must equal the oracle
+    N, K, M = 256, 4096, 48
+    nb = K // 256
+    rng = np.random.default_rng(21)
+    sc = np.array([1, 1, 1, 1, 0, 0, 0, 0, 1, 1, 1, 1], np.uint8)
+    w = synth.q4k_pack(np.ones(N * nb, np.float16), np.zeros(N * nb, np.float16), np.tile(sc, (N * nb, 1)),
+                       rng.integers(0, 256, (N * nb, 128), dtype=np.uint8)).reshape(N, -1)
+    x16 = rng.integers(-3, 4, (M, K)).astype(np.float16)
+    y = host(dq.q4k_prefill_gemm(dev(w), dev(x16), N, K))
+    y_ref, _ = oracle.q4k_prefill(w, N, K, x16)
+    assert np.array_equal(y.astype(np.float64), y_ref)
+
+
+def test_q4k_prefill_is_deterministic_and_soa_equals_aos():
+    N, K, M = 520, 4096, 96      # few tiles: K is split and the partials are reduced
+    rng = np.random.default_rng(22)
+    w = synth.q4k_matrix(rng, N, K)
+    x16 = dev(synth.activations_f16(rng, M, K))
+    assert dq.dq_workspace_bytes(dq.DQ_OP_Q4K_PREFILL, N, K, M) > 0
+    y1 = host(dq.q4k_prefill_gemm(dev(w), x16, N, K))
+    y2 = host(dq.q4k_prefill_gemm(dev(w), x16, N, K))
+    y3 = host(dq.q4k_prefill_gemm(dev(oracle.q4k_repack_soa(w, N, K)), x16, N, K, layout="soa"))
+    assert np.array_equal(y1.view(np.uint32), y2.view(np.uint32))
+    assert np.array_equal(y1.view(np.uint32), y3.view(np.uint32))
