@@ -74,6 +74,8 @@ def parse():
     ap.add_argument("--table", action="store_true",
                     help="print one JSON line per workload: device time per call under CUDA-graph replay "
                          "(weights rotated through enough copies to exceed L2), then exit")
+    ap.add_argument("--only", default="",
+                    help="with --table: run only the cases whose name contains this text")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="approximate CPU budget of the oracle baseline")
     return ap.parse_args()
@@ -262,10 +264,11 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def graph_table():
+def graph_table(only=""):
     """Per-workload device time per call, each call captured in a CUDA graph and
     replayed back to back; every workload's weights rotate through enough copies
-    (more than 1.3 x the 126 MB L2) that each call streams them from HBM."""
+    (more than 1.3 x the 126 MB L2) that each call streams them from HBM.  `only`
+    keeps the cases whose name contains it."""
     import torch
     import dequant_gemv_q4_b200 as dq
     from dequant_gemv_q4_b200 import synth
@@ -305,7 +308,12 @@ def graph_table():
              ("q4k_down_4096x12288", 4, "gemv"), ("q4k_down_4096x12288", 8, "gemv"),
              ("q4k_swiglu_12288x4096", 1, "gemv"), ("q4k_gemv_4096x1024", 1, "gemv"),
              ("q4k_gemv_4096x1024", 1, "split_qg"), ("q8_0_gemv_1024x1024", 1, "gemv")]
+    def want(name):
+        return only in name
+
     for wname, B, mode in cases:
+        if not want("%s:B%d:%s" % (wname, B, mode)):
+            continue
         wl = synth.WORKLOADS[wname]
         inp = synth.make_inputs(wl, B=B)
         keys = ["w_gate", "w_up"] if wl.op == "swiglu" else ["w"]
@@ -333,8 +341,20 @@ def graph_table():
         del ws
         torch.cuda.empty_cache()
 
-    # Q, K and V projections of a hidden-4096 layer (8 KV heads of 128): one grouped
-    # launch, and three separate calls
+    if want("qkv_4096+1024+1024x4096"):
+        qkv_table(timed, l2)
+    if want("decode_step:qproj_split+swiglu+down"):
+        decode_step_table(timed)
+    prefill_table(timed, l2, want)
+
+
+def qkv_table(timed, l2):
+    """Q, K and V projections of a hidden-4096 layer (8 KV heads of 128): one
+    grouped launch, and three separate calls."""
+    import torch
+    import dequant_gemv_q4_b200 as dq
+    from dequant_gemv_q4_b200 import synth
+
     rng = np.random.default_rng(43)
     Hq, Ns = 4096, (4096, 1024, 1024)
     per_set = sum(n * (Hq // 256) * 144 for n in Ns)
@@ -356,8 +376,15 @@ def graph_table():
     del qkv
     torch.cuda.empty_cache()
 
-    # one decode step's GEMV sequence: q-projection with the Q/gate split (16 heads of
-    # 128), SwiGLU 2 x 12288 x 4096, and the down projection 4096 x 12288 of its output
+
+def decode_step_table(timed):
+    """One decode step's GEMV sequence: q-projection with the Q/gate split (16
+    heads of 128), SwiGLU 2 x 12288 x 4096, and the down projection 4096 x 12288
+    of its output."""
+    import torch
+    import dequant_gemv_q4_b200 as dq
+    from dequant_gemv_q4_b200 import synth
+
     rng = np.random.default_rng(41)
     H, F, NQ, KQ = 4096, 12288, 4096, 1024
     shapes = ((NQ, KQ), (F, H), (F, H), (H, F))
@@ -381,16 +408,28 @@ def graph_table():
     del mats
     torch.cuda.empty_cache()
 
-    # W4A16 prefill on the tensor cores: M binary16 tokens through the down projection and
-    # through one gate/up matrix (bytes: weights + activations; flops: 2 M N K)
+
+def prefill_table(timed, l2, want):
+    """W4A16 prefill on the tensor cores: M binary16 tokens through the down
+    projection and through one gate/up matrix (bytes: weights + activations;
+    flops: 2 M N K)."""
+    import torch
+    import dequant_gemv_q4_b200 as dq
+    from dequant_gemv_q4_b200 import synth
+
     rng = np.random.default_rng(44)
+    Ms = (16, 64, 128, 256, 512)
     for N, K in ((4096, 12288), (12288, 4096)):
+        if not any(want("prefill_%dx%d:M%d" % (N, K, M)) for M in Ms):
+            continue
         wbytes = N * (K // 256) * 144
         copies = max(1, int(np.ceil(1.3 * l2 / wbytes)))
         pw = [torch.from_numpy(synth.q4k_matrix(rng, N, K)).cuda()]
         for _ in range(1, copies):
             pw.append(pw[0].clone())
-        for M in (16, 64, 128, 256, 512):
+        for M in Ms:
+            if not want("prefill_%dx%d:M%d" % (N, K, M)):
+                continue
             x16 = torch.from_numpy(synth.activations_f16(rng, M, K)).cuda()
             yp = torch.empty((M, N), device="cuda")
             scratch = torch.empty(max(1, dq.dq_workspace_bytes(dq.DQ_OP_Q4K_PREFILL, N, K, M)), dtype=torch.uint8,
@@ -411,7 +450,7 @@ def main():
         run_reference(args, rank, world)
         return
     if args.table:
-        graph_table()
+        graph_table(args.only)
         return
 
     import torch

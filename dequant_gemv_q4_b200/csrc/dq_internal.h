@@ -104,13 +104,13 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 // W4A16 prefill (tcgen05): Y = X W^T, X binary16, W Q4_K
 struct PrefillPlan {
     bool ok;
-    int T;                 // tokens per tile (MMA N), multiple of 16, <= 256
-    int mtiles;            // token tiles
-    int ntiles;            // 128-row weight tiles
+    int th;                // accumulators of 128 tokens per CTA (1 or 2)
+    int mtiles;            // token tiles of 128 * th
+    int ntiles;            // 256-row weight tiles
     int splits;            // K splits (partials reduced by a second kernel when > 1)
     int sb_per_split;      // super-blocks per split
-    int raw_depth;         // raw weight stages
-    int ab_depth;          // binary16 operand stages
+    int raw_depth;         // raw weight ring (super-blocks)
+    int depth;             // operand ring (stages of 64 K)
     int tmem_cols;         // tensor-memory columns allocated per CTA
     int grid;
     int smem;

@@ -9,23 +9,29 @@
 // the dequantize entry point produces) and then to binary16, and the products
 // of those binary16 weights with the binary16 activations are summed.
 //
-// Work decomposition.  A CTA owns a tile of 128 weight rows (the MMA's M) by T
-// tokens (the MMA's N, a multiple of 16, at most 256) and a range of K.  Per
-// super-block the raw bytes of the 128 rows (18 KB) arrive by one TMA tile copy.
-// Eight dequantizing warps turn each quarter super-block (64 weights per row)
-// into a 128 x 64 binary16 tile in the tensor cores' K-major, 128-byte swizzled
-// shared-memory layout, while the activation tile of the same 64 columns
-// arrives by TMA in that same layout.  One thread issues four 128 x T x 16 MMAs
-// per stage into a T-column fp32 accumulator in tensor memory and, through
-// tcgen05.commit, releases the stage when they have read it.  After the last
-// stage the same eight warps read the accumulator back (tcgen05.ld) and store
-// Y, or the split's partial sums when K is split across CTAs.
+// Work decomposition.  A CTA owns a tile of 256 weight rows (the MMA's N) by
+// up to 256 tokens (two accumulators of 128 tokens, the MMA's M; tokens past M
+// are zeros from the TMA unit's out-of-bounds fill) and a range of K.  Putting
+// the tokens on M keeps every MMA a full 128 x 256 x 16 operation even for a
+// handful of tokens, so the issuing thread never limits the rate.  Per
+// super-block the raw bytes of the 256 rows (36 KB) arrive by one TMA tile copy.
+// Sixteen dequantizing warps turn each quarter super-block (64 weights per row)
+// into a 256 x 64 binary16 tile in the tensor cores' K-major, 128-byte swizzled
+// shared-memory layout, while the activation tile(s) of the same 64 columns
+// arrive by TMA in that same layout.  Every CTA starts its K range at a
+// different super-block (rotated by its tile index), so that the CTAs, which
+// all read the same activations, do not all ask L2 for the same tile at once.
+// One thread issues four (or eight) MMAs per stage into the fp32 accumulators
+// in tensor memory and, through tcgen05.commit, releases the stage when they
+// have read it.  After the last stage the same sixteen warps read the
+// accumulators back (tcgen05.ld) and store Y, or the split's partial sums when
+// K is split across CTAs.
 //
 //   warp 0      weight TMA producer (one lane)
 //   warp 1      tensor-memory allocation, MMA issue (one lane)
 //   warp 2      activation TMA producer (one lane)
 //   warp 3      idle
-//   warps 4-11  dequantization, then the epilogue
+//   warps 4-19  dequantization, then the epilogue
 //
 // Dequantization of one weight: the GEMV's exact fp32 weight formation
 // (q4k_decode.cuh: the quant read in place as a subnormal, one fma with the
@@ -50,16 +56,17 @@
 
 namespace dq {
 
-constexpr int kPfRows = 128;                              // weight rows per tile (MMA M)
+constexpr int kPfRows = 256;                              // weight rows per tile (MMA N)
+constexpr int kPfTok = 128;                               // tokens per accumulator (MMA M)
 constexpr int kPfK = 64;                                  // K per stage: one 128-byte row of binary16
-constexpr int kPfMaxT = 256;                              // tokens per tile (MMA N) at most
-constexpr int kPfRawBytes = kPfRows * kQ4KBlockBytes;     // one super-block of 128 rows
-constexpr int kPfATileBytes = kPfRows * kPfK * 2;         // 16 KB
-constexpr int kPfWarps = 12;
+constexpr int kPfRawBytes = kPfRows * kQ4KBlockBytes;     // one super-block of 256 rows: 36 KB
+constexpr int kPfWTileBytes = kPfRows * kPfK * 2;         // 32 KB
+constexpr int kPfXTileBytes = kPfTok * kPfK * 2;          // 16 KB
+constexpr int kPfWarps = 20;
 constexpr int kPfDqWarp0 = 4;                             // first dequantizing warp
-constexpr int kPfDqThreads = (kPfWarps - kPfDqWarp0) * 32;
-constexpr int kPfMaxRaw = 3;
-constexpr int kPfMaxAB = 4;
+constexpr int kPfDqWarps = kPfWarps - kPfDqWarp0;
+constexpr int kPfMaxRaw = 4;                              // raw weight ring, super-blocks
+constexpr int kPfMaxStages = 4;                           // operand ring, stages
 
 struct PrefillMaps {
     CUtensorMap w;        // raw weight rows (AoS: 2-D bytes; SoA: 5-D gather of one block)
@@ -138,15 +145,80 @@ __device__ __forceinline__ void pf_tmem_ld8(uint32_t taddr, float (&v)[8])
         v[i] = __uint_as_float(r[i]);
 }
 
-// Bounded wait that also gives up at once when another role has aborted.
+// One try of an mbarrier phase wait that suspends the thread in hardware until
+// the phase completes or kPfSleepNs pass, instead of returning at once: the
+// waiting warps then take no issue slots and no shared-memory bandwidth from the
+// single threads that issue the copies and the MMAs.
+constexpr uint32_t kPfSleepNs = 10000000u;
+
+__device__ __forceinline__ bool pf_try_wait_sleep(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(kPfSleepNs)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait (kWaitNanos of the global timer in all) that also gives up once
+// another role has aborted; a timeout sets the device error flag and the abort
+// word.
 __device__ __forceinline__ bool pf_wait(uint32_t bar, uint32_t parity, int *err, volatile int *abort)
 {
-    if (*abort)
-        return false;
-    if (mbar_wait_bounded(bar, parity, err))
+    if (pf_try_wait_sleep(bar, parity))
         return true;
-    *abort = 1;
+    const unsigned long long t0 = global_ns();
+    while (global_ns() - t0 <= kWaitNanos) {
+        if (abort && *abort)
+            return false;
+        if (pf_try_wait_sleep(bar, parity))
+            return true;
+    }
+    atomicExch(err, kDevErrWaitTimeout);
+    if (abort)
+        *abort = 1;
     return false;
+}
+
+// Position in a ring of `depth` slots: the slot and the parity of the pass over
+// the ring (the mbarrier phase a full-barrier wait expects; an empty-barrier
+// wait on a later pass expects the other one).
+struct Ring {
+    int slot;
+    uint32_t phase;
+    int depth;
+    __device__ __forceinline__ void next()
+    {
+        if (++slot == depth) {
+            slot = 0;
+            phase ^= 1u;
+        }
+    }
+    __device__ __forceinline__ void prev()
+    {
+        if (slot == 0) {
+            slot = depth;
+            phase ^= 1u;
+        }
+        --slot;
+    }
+};
+
+// pf_wait by lane 0 of a warp for the whole warp (one sleeping waiter instead of
+// 32); the outcome is the same for every lane, and __syncwarp orders the lanes'
+// later shared-memory accesses after lane 0's observation of the phase.
+__device__ __forceinline__ bool pf_wait_warp(uint32_t bar, uint32_t parity, int *err, volatile int *abort)
+{
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0)
+        ok = pf_wait(bar, parity, err, abort) ? 1 : 0;
+    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+    __syncwarp();
+    return ok != 0;
 }
 
 // Two fp32 values -> one binary16 pair (round to nearest even), lo in bits 0..15.
@@ -157,17 +229,16 @@ __device__ __forceinline__ uint32_t pf_pack_f16x2(float lo, float hi)
     return r;
 }
 
-// Binary16 weights of the 16 quant bytes of one row in `qv` (bytes 32c + 16h ..
-// 32c + 16h + 15 of the super-block): lo[0..1] are the 16 low-nibble weights
-// (k = 64c + 16h + 0..15) as two 8-weight chunks, hi[0..1] the 16 high-nibble
-// weights (k = 64c + 32 + 16h + 0..15).
-__device__ __forceinline__ void pf_dequant16(uint4 qv, const ChunkScales &cs, uint4 (&lo)[2], uint4 (&hi)[2])
+// Binary16 weights of the 8 quant bytes of one row in `qv` (bytes 32c + 8e ..
+// 32c + 8e + 7 of the super-block): lo holds the 8 low-nibble weights
+// (k = 64c + 8e + 0..7), hi the 8 high-nibble weights (k = 64c + 32 + 8e + 0..7).
+__device__ __forceinline__ void pf_dequant8(uint2 qv, const ChunkScales &cs, uint4 &lo, uint4 &hi)
 {
     const float2 up = make_float2(0x1p64f, 0x1p64f);   // q4_word_weights forms w * 2^-64
-    const uint32_t words[4] = {qv.x, qv.y, qv.z, qv.w};
-    uint32_t plo[8], phi[8];
+    const uint32_t words[2] = {qv.x, qv.y};
+    uint32_t plo[4], phi[4];
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
+    for (int t = 0; t < 2; ++t) {
         float2 wv[4];   // {lo, hi} weights of bytes 4t .. 4t+3
         q4_word_weights(words[t], cs, wv);
 #pragma unroll
@@ -178,10 +249,15 @@ __device__ __forceinline__ void pf_dequant16(uint4 qv, const ChunkScales &cs, ui
         phi[2 * t] = pf_pack_f16x2(wv[0].y, wv[1].y);
         phi[2 * t + 1] = pf_pack_f16x2(wv[2].y, wv[3].y);
     }
-    lo[0] = make_uint4(plo[0], plo[1], plo[2], plo[3]);
-    lo[1] = make_uint4(plo[4], plo[5], plo[6], plo[7]);
-    hi[0] = make_uint4(phi[0], phi[1], phi[2], phi[3]);
-    hi[1] = make_uint4(phi[4], phi[5], phi[6], phi[7]);
+    lo = make_uint4(plo[0], plo[1], plo[2], plo[3]);
+    hi = make_uint4(phi[0], phi[1], phi[2], phi[3]);
+}
+
+__device__ __forceinline__ uint2 lds64(uint32_t addr)
+{
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    return v;
 }
 
 __device__ __forceinline__ void sts128(uint32_t addr, uint4 v)
@@ -196,12 +272,12 @@ struct PrefillParams {
     long long N;
     long long M;
     int nb;            // super-blocks per row (K / 256)
-    int T;             // tokens per tile (MMA N)
-    int mtiles;
-    int ntiles;
+    int th;            // accumulators (token halves of 128) per CTA: 1 or 2
+    int mtiles;        // token tiles of 128 * th
+    int ntiles;        // weight-row tiles of 256
     int sb_per_split;
     int raw_depth;
-    int ab_depth;
+    int depth;         // operand ring stages
     int soa;
     int soa_full;      // complete 4-block groups per row (SoA)
     uint32_t idesc;    // MMA instruction descriptor
@@ -214,24 +290,24 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1)
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
-    __shared__ __align__(8) uint64_t s_bars[2 * kPfMaxRaw + 3 * kPfMaxAB + 1];
+    __shared__ __align__(8) uint64_t s_bars[2 * (kPfMaxRaw + kPfMaxStages) + 1];
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int AD = p.ab_depth;
+    const int SD = p.depth;
     const int RD = p.raw_depth;
-    const int T = p.T;
-    const uint32_t b_bytes = static_cast<uint32_t>(T) * 128;
+    const int TH = p.th;
+    const uint32_t x_bytes = static_cast<uint32_t>(TH) * kPfXTileBytes;
+    const uint32_t stage_bytes = kPfWTileBytes + x_bytes;
 
-    const uint32_t a_s = (smem_u32(smem) + 1023u) & ~1023u;        // AD x 128 x 64 binary16 weights
-    const uint32_t b_s = a_s + AD * kPfATileBytes;                  // AD x T x 64 binary16 activations
-    const uint32_t raw_s = b_s + AD * b_bytes;                      // RD x 128 rows x 144 raw bytes
+    // stage slot s: [binary16 weight tile, 32 KB][activation tile(s), 16 KB each]
+    const uint32_t st_s = (smem_u32(smem) + 1023u) & ~1023u;
+    const uint32_t raw_s = st_s + SD * stage_bytes;                 // RD x 256 rows x 144 raw bytes
     const uint32_t raw_full = smem_u32(s_bars);
     const uint32_t raw_empty = raw_full + 8 * kPfMaxRaw;
-    const uint32_t a_full = raw_empty + 8 * kPfMaxRaw;
-    const uint32_t b_full = a_full + 8 * kPfMaxAB;
-    const uint32_t ab_empty = b_full + 8 * kPfMaxAB;
-    const uint32_t acc_full = ab_empty + 8 * kPfMaxAB;
+    const uint32_t full = raw_empty + 8 * kPfMaxRaw;               // stage: weights formed + activations landed
+    const uint32_t empty = full + 8 * kPfMaxStages;                // stage: MMAs done reading it
+    const uint32_t acc_full = empty + 8 * kPfMaxStages;
 
     // tile: consecutive CTAs share one weight tile (mt fastest), then row tiles, then splits
     const int mt = static_cast<int>(blockIdx.x % p.mtiles);
@@ -239,20 +315,20 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1)
     const int nt = rest % p.ntiles;
     const int split = rest / p.ntiles;
     const long long row0 = static_cast<long long>(nt) * kPfRows;
-    const long long m0 = static_cast<long long>(mt) * T;
+    const long long m0 = static_cast<long long>(mt) * kPfTok * TH;
     const int kb0 = split * p.sb_per_split;
     const int nsb = min(p.sb_per_split, p.nb - kb0);
     const int nst = 4 * nsb;
+    const int rot = nt % nsb;   // first super-block of this CTA's K range, relative to kb0
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < RD; ++i) {
             mbar_init(raw_full + 8 * i, 1);
-            mbar_init(raw_empty + 8 * i, kPfDqThreads);
+            mbar_init(raw_empty + 8 * i, kPfDqWarps);
         }
-        for (int i = 0; i < AD; ++i) {
-            mbar_init(a_full + 8 * i, kPfDqThreads);
-            mbar_init(b_full + 8 * i, 1);
-            mbar_init(ab_empty + 8 * i, 1);
+        for (int i = 0; i < SD; ++i) {
+            mbar_init(full + 8 * i, kPfDqWarps + 1);   // one arrival per dequantizing warp + the activation copy
+            mbar_init(empty + 8 * i, 1);
         }
         mbar_init(acc_full, 1);
         s_abort = 0;
@@ -276,14 +352,15 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1)
     if (warp == 0) {
         // ---- weight producer: one TMA tile copy per super-block of the tile's rows
         if (lane == 0) {
+            Ring r{0, 0, RD};
+            int kbi = rot;    // super-block, relative to kb0
             int issued = 0;
-            for (int i = 0; i < nsb; ++i) {
-                const int s = i % RD;
-                if (i >= RD && !pf_wait(raw_empty + 8 * s, ((i / RD) & 1) ^ 1, p.err, abort))
+            for (; issued < nsb; ++issued) {
+                if (issued >= RD && !pf_wait(raw_empty + 8 * r.slot, r.phase ^ 1, p.err, abort))
                     break;
-                const uint32_t bar = raw_full + 8 * s;
-                const uint32_t dst = raw_s + s * kPfRawBytes;
-                const int kb = kb0 + i;
+                const uint32_t bar = raw_full + 8 * r.slot;
+                const uint32_t dst = raw_s + r.slot * kPfRawBytes;
+                const int kb = kb0 + kbi;
                 mbar_arrive_expect_tx(bar, kPfRawBytes);
                 if (!p.soa)
                     pf_tma_2d(dst, &maps.w, kb * kQ4KBlockBytes, static_cast<int>(row0), bar);   // x: 144 kb bytes
@@ -291,103 +368,143 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1)
                     pf_tma_5d(dst, &maps.w, 0, kb & 3, 0, kb >> 2, static_cast<int>(row0), bar);
                 else
                     pf_tma_5d(dst, &maps.w_tail, 0, kb - 4 * p.soa_full, 0, 0, static_cast<int>(row0), bar);
-                ++issued;
+                r.next();
+                if (++kbi == nsb)
+                    kbi = 0;
             }
-            for (int i = issued > RD ? issued - RD : 0; i < issued; ++i)
-                mbar_wait_bounded(raw_full + 8 * (i % RD), (i / RD) & 1, p.err);
+            // own copies still in flight complete before the CTA may exit
+            for (int u = 0; u < issued && u < RD; ++u) {
+                r.prev();
+                pf_wait(raw_full + 8 * r.slot, r.phase, p.err, nullptr);
+            }
         }
     } else if (warp == 2) {
-        // ---- activation producer: one TMA tile copy (T x 64, swizzled) per stage
+        // ---- activation producer: TH TMA tile copies (128 tokens x 64, swizzled) per stage, completing
+        // on the stage's full barrier together with the dequantizing warps' arrivals
         if (lane == 0) {
+            Ring r{0, 0, SD};
+            int kbi = rot, quarter = 0;
             int issued = 0;
-            for (int j = 0; j < nst; ++j) {
-                const int s = j % AD;
-                if (j >= AD && !pf_wait(ab_empty + 8 * s, ((j / AD) & 1) ^ 1, p.err, abort))
+            for (; issued < nst; ++issued) {
+                if (issued >= SD && !pf_wait(empty + 8 * r.slot, r.phase ^ 1, p.err, abort))
                     break;
-                const uint32_t bar = b_full + 8 * s;
-                mbar_arrive_expect_tx(bar, b_bytes);
-                pf_tma_2d(b_s + s * b_bytes, &maps.x, kb0 * kQ4KBlockElems + j * kPfK, static_cast<int>(m0), bar);
-                ++issued;
+                const uint32_t bar = full + 8 * r.slot;
+                const uint32_t dst = st_s + r.slot * stage_bytes + kPfWTileBytes;
+                const int k = (kb0 + kbi) * kQ4KBlockElems + quarter * kPfK;
+                mbar_arrive_expect_tx(bar, x_bytes);
+                for (int t = 0; t < TH; ++t)
+                    pf_tma_2d(dst + t * kPfXTileBytes, &maps.x, k, static_cast<int>(m0) + t * kPfTok, bar);
+                r.next();
+                if (++quarter == 4) {
+                    quarter = 0;
+                    if (++kbi == nsb)
+                        kbi = 0;
+                }
             }
-            for (int j = issued > AD ? issued - AD : 0; j < issued; ++j)
-                mbar_wait_bounded(b_full + 8 * (j % AD), (j / AD) & 1, p.err);
+            for (int u = 0; u < issued && u < SD; ++u) {
+                r.prev();
+                pf_wait(full + 8 * r.slot, r.phase, p.err, nullptr);
+            }
         }
     } else if (warp == 1) {
-        // ---- MMA issue: four K = 16 steps per stage into the T-column accumulator
+        // ---- MMA issue: per stage and accumulator, four K = 16 steps (128 tokens x 256 rows each).
+        // Descriptors advance by whole stages (and by 32 bytes per K step) in their 16-byte address field.
         if (lane == 0) {
+            Ring r{0, 0, SD};
+            const uint64_t w_desc0 = pf_desc_sw128(st_s);
+            const uint64_t x_desc0 = pf_desc_sw128(st_s + kPfWTileBytes);
+            const uint32_t idesc = p.idesc;
             for (int j = 0; j < nst; ++j) {
-                const int s = j % AD;
-                const uint32_t ph = (j / AD) & 1;
-                if (!pf_wait(a_full + 8 * s, ph, p.err, abort) || !pf_wait(b_full + 8 * s, ph, p.err, abort))
+                if (!pf_wait(full + 8 * r.slot, r.phase, p.err, abort))
                     break;
                 pf_fence_after();
-                const uint32_t a0 = a_s + s * kPfATileBytes;
-                const uint32_t b0 = b_s + s * b_bytes;
+                const uint64_t soff = static_cast<uint64_t>(r.slot * (stage_bytes >> 4));
+                for (int t = 0; t < TH; ++t) {
+                    const uint64_t xd = x_desc0 + soff + static_cast<uint64_t>(t * (kPfXTileBytes >> 4));
 #pragma unroll
-                for (int kk = 0; kk < kPfK / 16; ++kk)
-                    pf_mma_f16(tmem, pf_desc_sw128(a0 + 32 * kk), pf_desc_sw128(b0 + 32 * kk), p.idesc,
-                               (j | kk) != 0);
-                pf_commit(ab_empty + 8 * s);
+                    for (int kk = 0; kk < kPfK / 16; ++kk)
+                        pf_mma_f16(tmem + t * kPfRows, xd + 2 * kk, w_desc0 + soff + 2 * kk, idesc, (j | kk) != 0);
+                }
+                pf_commit(empty + 8 * r.slot);
+                r.next();
             }
             // arrives once every MMA issued above has completed
             pf_commit(acc_full);
         }
     } else if (warp >= kPfDqWarp0) {
-        // ---- dequantization: thread (q, h, lane) forms row 32q + lane, quant bytes 16h .. 16h+15 of
-        // each 32-byte chunk, into the K-major 128-byte swizzled tile (16-byte unit u of row r at
-        // position u ^ (r % 8) of the row's 128 bytes; 8-row groups 1024 bytes apart)
-        const int q = warp & 3;
-        const int h = (warp - kPfDqWarp0) >> 2;
-        const int r = 32 * q + lane;
+        // ---- dequantization: warp d = warp - 4 forms rows 32 (d % 8) + lane, quant bytes 16h .. 16h+15
+        // (h = d / 8) of each 32-byte chunk, into the K-major 128-byte swizzled weight tile (16-byte unit
+        // u of row r at position u ^ (r % 8) of the row's 128 bytes; 8-row groups 1024 bytes apart):
+        // low nibbles are units 2h, 2h+1, high nibbles units 4+2h, 5+2h
+        const int d = warp - kPfDqWarp0;
+        const int h = d >> 3;
+        const int r = 32 * (d & 7) + lane;
         const uint32_t row_off = static_cast<uint32_t>((r >> 3) * 1024 + (r & 7) * 128);
         const int sw = r & 7;
+        Ring rr{0, 0, RD}, rs{0, 0, SD};
+        int j = 0;   // stage
         bool ok = true;
         for (int i = 0; i < nsb && ok; ++i) {
-            const int rs = i % RD;
-            if (!pf_wait(raw_full + 8 * rs, (i / RD) & 1, p.err, abort))
+            if (!pf_wait_warp(raw_full + 8 * rr.slot, rr.phase, p.err, abort))
                 break;
-            const uint32_t raw = raw_s + rs * kPfRawBytes + r * kQ4KBlockBytes;
+            const uint32_t raw = raw_s + rr.slot * kPfRawBytes + r * kQ4KBlockBytes;
             const Hdr hd = decode_hdr(lds128(raw));
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                const int j = 4 * i + c;
-                const int s = j % AD;
-                if (j >= AD && !pf_wait(ab_empty + 8 * s, ((j / AD) & 1) ^ 1, p.err, abort)) {
+                if (j >= SD && !pf_wait_warp(empty + 8 * rs.slot, rs.phase ^ 1, p.err, abort)) {
                     ok = false;
                     break;
                 }
-                uint4 lo[2], hi[2];
-                pf_dequant16(lds128(raw + 16 + 32 * c + 16 * h), chunk_scales(hd, c), lo, hi);
-                const uint32_t at = a_s + s * kPfATileBytes + row_off;
-                sts128(at + (((2 * h) ^ sw) << 4), lo[0]);
-                sts128(at + (((2 * h + 1) ^ sw) << 4), lo[1]);
-                sts128(at + (((4 + 2 * h) ^ sw) << 4), hi[0]);
-                sts128(at + (((5 + 2 * h) ^ sw) << 4), hi[1]);
+                const ChunkScales cs = chunk_scales(hd, c);
+                const uint4 qv = lds128(raw + 16 + 32 * c + 16 * h);
+                uint4 lo0, hi0, lo1, hi1;
+                pf_dequant8(make_uint2(qv.x, qv.y), cs, lo0, hi0);
+                pf_dequant8(make_uint2(qv.z, qv.w), cs, lo1, hi1);
+                const uint32_t at = st_s + rs.slot * stage_bytes + row_off;
+                sts128(at + (((2 * h) ^ sw) << 4), lo0);
+                sts128(at + (((2 * h + 1) ^ sw) << 4), lo1);
+                sts128(at + (((4 + 2 * h) ^ sw) << 4), hi0);
+                sts128(at + (((5 + 2 * h) ^ sw) << 4), hi1);
                 fence_proxy_async_smem();   // generic-proxy stores -> visible to the tensor cores
-                mbar_arrive(a_full + 8 * s);
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(full + 8 * rs.slot);   // one arrival per warp
+                rs.next();
+                ++j;
             }
             if (!ok)
                 break;
-            mbar_arrive(raw_empty + 8 * rs);
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(raw_empty + 8 * rr.slot);
+            rr.next();
         }
 
-        // ---- epilogue: accumulator row r (lanes 32q .. 32q+31), columns [h T/2, (h+1) T/2)
-        const bool done = mbar_wait_bounded(acc_full, 0, p.err);
+        // ---- epilogue: warp (q = warp % 4, e = d / 4) reads accumulator lanes 32q .. 32q+31 (tokens)
+        // and columns 64e .. 64e+63 (weight rows) of each accumulator
+        const bool done = pf_wait_warp(acc_full, 0, p.err, nullptr);
         pf_fence_after();
         // tcgen05.ld is warp-collective: the whole warp reads, or none of it
         if (__all_sync(0xFFFFFFFFu, done && !*abort)) {
-            const long long n = row0 + r;
+            const int q = warp & 3;
+            const int e = d >> 2;
             float *out = p.out + static_cast<long long>(split) * p.M * p.N;
-            const int half = T >> 1;
-            for (int c0 = h * half; c0 < (h + 1) * half; c0 += 8) {
-                float v[8];
-                pf_tmem_ld8(tmem + (static_cast<uint32_t>(32 * q) << 16) + c0, v);
-                if (n < p.N) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const long long m = m0 + c0 + e;
-                        if (m < p.M)
-                            out[m * p.N + n] = v[e];
+            const bool vec = (p.N & 3) == 0;
+            for (int t = 0; t < TH; ++t) {
+                const long long m = m0 + t * kPfTok + 32 * q + lane;
+                for (int c0 = 64 * e; c0 < 64 * e + 64; c0 += 8) {
+                    float v[8];
+                    pf_tmem_ld8(tmem + (static_cast<uint32_t>(32 * q) << 16) + t * kPfRows + c0, v);
+                    const long long n = row0 + c0;
+                    if (m >= p.M || n >= p.N)
+                        continue;
+                    float *o = out + m * p.N + n;
+                    if (vec && n + 8 <= p.N) {
+                        reinterpret_cast<float4 *>(o)[0] = make_float4(v[0], v[1], v[2], v[3]);
+                        reinterpret_cast<float4 *>(o)[1] = make_float4(v[4], v[5], v[6], v[7]);
+                    } else {
+                        for (int u = 0; u < 8 && n + u < p.N; ++u)
+                            o[u] = v[u];
                     }
                 }
             }
@@ -399,7 +516,7 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1)
     if (warp == 1) {
         pf_fence_after();
         // every MMA has completed once acc_full's phase 0 has (bounded; normally it has long since)
-        mbar_wait_bounded(acc_full, 0, p.err);
+        pf_wait(acc_full, 0, p.err, nullptr);
         __syncwarp();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(p.tmem_cols)
                      : "memory");
@@ -442,53 +559,58 @@ __global__ void __launch_bounds__(256) prefill_reduce_kernel(const float *part, 
 // host side
 // ---------------------------------------------------------------------------
 
-// Tiles of 128 weight rows by T tokens (T a multiple of 16, at most 256, the
-// tokens split evenly over ceil(M / 256) tiles); K is split so that the tiles
-// fill the SMs once (one CTA per SM: the stages take most of shared memory);
-// as many stages as fit, up to 3 raw and 4 binary16 stages.
+// Tiles of 256 weight rows by 128 tokens (M <= 128) or 256 tokens (two
+// accumulators), one CTA per SM (the rings take most of shared memory).  K is
+// split into the number of parts that minimises (waves of CTAs) x (super-blocks
+// per CTA + a fixed cost of about six for the pipeline fill and the epilogue);
+// ties go to fewer parts.  Rings: as many operand stages as fit next to two raw
+// super-blocks, up to 4; the raw ring grows into what is left, up to 4.
 PrefillPlan q4k_prefill_plan(long long N, int K, long long M, int sm_count, int smem_optin)
 {
     PrefillPlan pl{};
-    if (N < 1 || M < 1 || K < kQ4KBlockElems || K % kQ4KBlockElems != 0 || tensor_map_encoder() == nullptr)
+    if (N < 1 || M < 1 || K < kQ4KBlockElems || K % kQ4KBlockElems != 0 || sm_count < 1 ||
+        tensor_map_encoder() == nullptr)
         return pl;
     const int nb = K / kQ4KBlockElems;
-    const long long mtiles = (M + kPfMaxT - 1) / kPfMaxT;
-    const long long per = (M + mtiles - 1) / mtiles;
-    const int T = static_cast<int>((per + 15) / 16 * 16);
+    const int th = M <= kPfTok ? 1 : 2;
+    const long long mtiles = (M + th * kPfTok - 1) / (th * kPfTok);
     const long long ntiles = (N + kPfRows - 1) / kPfRows;
     const long long tiles = ntiles * mtiles;
-    int splits = 1;
-    if (tiles < sm_count) {
-        splits = static_cast<int>(sm_count / tiles);
-        if (splits > nb)
-            splits = nb;
+    int splits = 1, sbps = nb;
+    long long best = -1;
+    for (int s = 1; s <= nb && s <= 64; ++s) {
+        const int per_split = (nb + s - 1) / s;
+        const int used = (nb + per_split - 1) / per_split;
+        const long long waves = (tiles * used + sm_count - 1) / sm_count;
+        const long long cost = waves * (per_split + 6);
+        if (best < 0 || cost < best) {
+            best = cost;
+            splits = used;
+            sbps = per_split;
+        }
     }
-    const int sbps = (nb + splits - 1) / splits;
-    splits = (nb + sbps - 1) / sbps;
     if (tiles * splits > 0x7FFFFFFFLL)
         return pl;
-    const int ab = kPfATileBytes + T * 128;
+    const int stage = kPfWTileBytes + th * kPfXTileBytes;
     const int budget = smem_optin - 1024 /*static shared memory*/ - 1024 /*alignment of the tiles*/;
-    int ad = kPfMaxAB, rd = kPfMaxRaw;
-    while (ad * ab + rd * kPfRawBytes > budget && ad > 2)
-        --ad;
-    while (ad * ab + rd * kPfRawBytes > budget && rd > 2)
-        --rd;
-    if (ad * ab + rd * kPfRawBytes > budget)
+    int depth = (budget - 2 * kPfRawBytes) / stage;
+    if (depth > kPfMaxStages)
+        depth = kPfMaxStages;
+    if (depth < 2)
         return pl;
-    int cols = 32;
-    while (cols < T)
-        cols *= 2;
-    pl.T = T;
+    int rd = (budget - depth * stage) / kPfRawBytes;
+    if (rd > kPfMaxRaw)
+        rd = kPfMaxRaw;
+    pl.th = th;
     pl.mtiles = static_cast<int>(mtiles);
     pl.ntiles = static_cast<int>(ntiles);
     pl.splits = splits;
     pl.sb_per_split = sbps;
     pl.raw_depth = rd;
-    pl.ab_depth = ad;
-    pl.tmem_cols = cols;
+    pl.depth = depth;
+    pl.tmem_cols = 256 * th;
     pl.grid = static_cast<int>(tiles * splits);
-    pl.smem = 1024 + ad * ab + rd * kPfRawBytes;
+    pl.smem = 1024 + depth * stage + rd * kPfRawBytes;
     pl.ok = true;
     return pl;
 }
@@ -514,7 +636,7 @@ cudaError_t q4k_prefill_launch(const uint8_t *w, int soa, const uint16_t *x16, f
     cudaError_t e = cudaSuccess;
     int soa_full = 0;
     if (!soa) {
-        // raw rows as bytes: box = one super-block (144 bytes) of 128 rows
+        // raw rows as bytes: box = one super-block (144 bytes) of 256 rows
         const cuuint64_t dims[2] = {row, static_cast<cuuint64_t>(N)};
         const cuuint64_t strides[1] = {row};
         const cuuint32_t box[2] = {kQ4KBlockBytes, kPfRows};
@@ -544,10 +666,10 @@ cudaError_t q4k_prefill_launch(const uint8_t *w, int soa, const uint16_t *x16, f
     if (e != cudaSuccess)
         return e;
     {
-        // activations: box of 64 binary16 (128 bytes) x T tokens, 128-byte swizzle
+        // activations: box of 64 binary16 (128 bytes) x 128 tokens, 128-byte swizzle
         const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
         const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-        const cuuint32_t box[2] = {kPfK, static_cast<cuuint32_t>(pl.T)};
+        const cuuint32_t box[2] = {kPfK, kPfTok};
         e = encode(&maps.x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x16, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
         if (e != cudaSuccess)
             return e;
@@ -558,17 +680,18 @@ cudaError_t q4k_prefill_launch(const uint8_t *w, int soa, const uint16_t *x16, f
     p.N = N;
     p.M = M;
     p.nb = nb;
-    p.T = pl.T;
+    p.th = pl.th;
     p.mtiles = pl.mtiles;
     p.ntiles = pl.ntiles;
     p.sb_per_split = pl.sb_per_split;
     p.raw_depth = pl.raw_depth;
-    p.ab_depth = pl.ab_depth;
+    p.depth = pl.depth;
     p.soa = soa;
     p.soa_full = soa_full;
     // kind::f16 instruction descriptor: D fp32 (bits 4-5 = 1), A and B binary16 (bits 7-9, 10-12 = 0),
-    // both K-major (bits 15, 16 = 0), N >> 3 in bits 17-22, M >> 4 in bits 24-28
-    p.idesc = (1u << 4) | (static_cast<uint32_t>(pl.T >> 3) << 17) | (static_cast<uint32_t>(kPfRows >> 4) << 24);
+    // both K-major (bits 15, 16 = 0), N >> 3 in bits 17-22, M >> 4 in bits 24-28; A = 128 tokens,
+    // B = 256 weight rows
+    p.idesc = (1u << 4) | (static_cast<uint32_t>(kPfRows >> 3) << 17) | (static_cast<uint32_t>(kPfTok >> 4) << 24);
     p.tmem_cols = static_cast<uint32_t>(pl.tmem_cols);
     e = cudaFuncSetAttribute(q4k_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
     if (e != cudaSuccess)
