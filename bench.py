@@ -49,8 +49,8 @@ FALLBACK_HBM_GBS = 6650.0
 
 # DRAM bytes (read + write) per launch of q4k_gemv_fx_kernel on this workload,
 # from one ncu capture, valid only for the kernel sources whose hash is recorded.
-NCU_TRAFFIC = {"sources_sha1": "67978a8cc32f7e81d47ff68172ede90989c9b562",
-               "bytes_per_launch": 572208128 + 4117248}   # profiles/q4k_gemv_fx_kernel_248320x4096_dram.md
+NCU_TRAFFIC = {"sources_sha1": "5473d0d9bdc0e977199b20f6531857538bba7134",
+               "bytes_per_launch": 572221184 + 4019200}   # profiles/q4k_gemv_fx_kernel_248320x4096_dram.md
 
 
 def kernel_sources_sha1() -> str:

@@ -290,6 +290,7 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1)
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
+    __shared__ int s_go[2];
     __shared__ __align__(8) uint64_t s_bars[2 * (kPfMaxRaw + kPfMaxStages) + 1];
 
     const int warp = threadIdx.x >> 5;
@@ -441,17 +442,33 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1)
         const int r = 32 * (d & 7) + lane;
         const uint32_t row_off = static_cast<uint32_t>((r >> 3) * 1024 + (r & 7) * 128);
         const int sw = r & 7;
+        const uint32_t o_lo0 = row_off + (((2 * h) ^ sw) << 4), o_lo1 = row_off + (((2 * h + 1) ^ sw) << 4);
+        const uint32_t o_hi0 = row_off + (((4 + 2 * h) ^ sw) << 4), o_hi1 = row_off + (((5 + 2 * h) ^ sw) << 4);
+        // One leader thread waits on the mbarriers for all sixteen warps and passes its outcome
+        // through s_go (two slots, alternating per barrier, so that a slot is rewritten only after
+        // every warp has read it); the warps meet at a named hardware barrier, where waiting takes
+        // no issue slots.
+        const bool leader = warp == kPfDqWarp0 && lane == 0;
+        int nb_sync = 0;
+        auto gate = [&](uint32_t bar, uint32_t parity) -> bool {
+            volatile int *go = s_go + (nb_sync & 1);
+            if (leader)
+                *go = pf_wait(bar, parity, p.err, abort) ? 1 : 0;
+            asm volatile("bar.sync 1, %0;" ::"n"(kPfDqWarps * 32) : "memory");
+            ++nb_sync;
+            return *go != 0;
+        };
         Ring rr{0, 0, RD}, rs{0, 0, SD};
         int j = 0;   // stage
         bool ok = true;
         for (int i = 0; i < nsb && ok; ++i) {
-            if (!pf_wait_warp(raw_full + 8 * rr.slot, rr.phase, p.err, abort))
+            if (!gate(raw_full + 8 * rr.slot, rr.phase))
                 break;
             const uint32_t raw = raw_s + rr.slot * kPfRawBytes + r * kQ4KBlockBytes;
             const Hdr hd = decode_hdr(lds128(raw));
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                if (j >= SD && !pf_wait_warp(empty + 8 * rs.slot, rs.phase ^ 1, p.err, abort)) {
+                if (j >= SD && !gate(empty + 8 * rs.slot, rs.phase ^ 1)) {
                     ok = false;
                     break;
                 }
@@ -460,11 +477,11 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1)
                 uint4 lo0, hi0, lo1, hi1;
                 pf_dequant8(make_uint2(qv.x, qv.y), cs, lo0, hi0);
                 pf_dequant8(make_uint2(qv.z, qv.w), cs, lo1, hi1);
-                const uint32_t at = st_s + rs.slot * stage_bytes + row_off;
-                sts128(at + (((2 * h) ^ sw) << 4), lo0);
-                sts128(at + (((2 * h + 1) ^ sw) << 4), lo1);
-                sts128(at + (((4 + 2 * h) ^ sw) << 4), hi0);
-                sts128(at + (((5 + 2 * h) ^ sw) << 4), hi1);
+                const uint32_t at = st_s + rs.slot * stage_bytes;
+                sts128(at + o_lo0, lo0);
+                sts128(at + o_lo1, lo1);
+                sts128(at + o_hi0, hi0);
+                sts128(at + o_hi1, hi1);
                 fence_proxy_async_smem();   // generic-proxy stores -> visible to the tensor cores
                 __syncwarp();
                 if (lane == 0)
