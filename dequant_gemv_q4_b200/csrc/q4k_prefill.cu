@@ -15,8 +15,8 @@
 // the tokens on M keeps every MMA a full 128 x 256 x 16 operation even for a
 // handful of tokens, so the issuing thread never limits the rate.  Per
 // super-block the raw bytes of the 256 rows (36 KB) arrive by one TMA tile copy.
-// Sixteen dequantizing warps turn each quarter super-block (64 weights per row)
-// into a 256 x 64 binary16 tile in the tensor cores' K-major, 128-byte swizzled
+// Sixteen dequantizing warps, in two groups that take alternate stages, turn
+// each quarter super-block (64 weights per row) into a 256 x 64 binary16 tile in the tensor cores' K-major, 128-byte swizzled
 // shared-memory layout, while the activation tile(s) of the same 64 columns
 // arrive by TMA in that same layout.  Every CTA starts its K range at a
 // different super-block (rotated by its tile index), so that the CTAs, which
@@ -290,7 +290,7 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1)
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
-    __shared__ int s_go[2];
+    __shared__ int s_go[4];
     __shared__ __align__(8) uint64_t s_bars[2 * (kPfMaxRaw + kPfMaxStages) + 1];
 
     const int warp = threadIdx.x >> 5;
@@ -328,7 +328,7 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1)
             mbar_init(raw_empty + 8 * i, kPfDqWarps);
         }
         for (int i = 0; i < SD; ++i) {
-            mbar_init(full + 8 * i, kPfDqWarps + 1);   // one arrival per dequantizing warp + the activation copy
+            mbar_init(full + 8 * i, kPfDqWarps / 2 + 1);   // one arrival per warp of a group + the activation copy
             mbar_init(empty + 8 * i, 1);
         }
         mbar_init(acc_full, 1);
@@ -433,33 +433,36 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1)
             pf_commit(acc_full);
         }
     } else if (warp >= kPfDqWarp0) {
-        // ---- dequantization: warp d = warp - 4 forms rows 32 (d % 8) + lane, quant bytes 16h .. 16h+15
-        // (h = d / 8) of each 32-byte chunk, into the K-major 128-byte swizzled weight tile (16-byte unit
-        // u of row r at position u ^ (r % 8) of the row's 128 bytes; 8-row groups 1024 bytes apart):
-        // low nibbles are units 2h, 2h+1, high nibbles units 4+2h, 5+2h
+        // ---- dequantization: the sixteen warps form two groups of eight that take alternate stages
+        // (group g the stages j with j % 2 == g, i.e. chunks g and g + 2 of each super-block), so
+        // two stages are formed at once.  Warp d = warp - 4 of group g = d / 8 forms row
+        // 32 (d % 8) + lane: all 32 quant bytes of the stage's chunk, written into the K-major
+        // 128-byte swizzled weight tile (16-byte unit u of row r at position u ^ (r % 8) of the
+        // row's 128 bytes; 8-row groups 1024 bytes apart): low nibbles are units 0-3, high
+        // nibbles units 4-7.
         const int d = warp - kPfDqWarp0;
-        const int h = d >> 3;
+        const int g = d >> 3;
         const int r = 32 * (d & 7) + lane;
         const uint32_t row_off = static_cast<uint32_t>((r >> 3) * 1024 + (r & 7) * 128);
         const int sw = r & 7;
-        const uint32_t o_lo0 = row_off + (((2 * h) ^ sw) << 4), o_lo1 = row_off + (((2 * h + 1) ^ sw) << 4);
-        const uint32_t o_hi0 = row_off + (((4 + 2 * h) ^ sw) << 4), o_hi1 = row_off + (((5 + 2 * h) ^ sw) << 4);
-        // One leader thread waits on the mbarriers for all sixteen warps and passes its outcome
-        // through s_go (two slots, alternating per barrier, so that a slot is rewritten only after
-        // every warp has read it); the warps meet at a named hardware barrier, where waiting takes
-        // no issue slots.
-        const bool leader = warp == kPfDqWarp0 && lane == 0;
+        // One leader thread per group waits on the mbarriers for the group's eight warps and passes
+        // its outcome through s_go (two slots per group, alternating per barrier, so that a slot is
+        // rewritten only after every warp of the group has read it); the warps meet at the group's
+        // named hardware barrier, where waiting takes no issue slots.
+        const bool leader = (d & 7) == 0 && lane == 0;
         int nb_sync = 0;
         auto gate = [&](uint32_t bar, uint32_t parity) -> bool {
-            volatile int *go = s_go + (nb_sync & 1);
+            volatile int *go = s_go + 2 * g + (nb_sync & 1);
             if (leader)
                 *go = pf_wait(bar, parity, p.err, abort) ? 1 : 0;
-            asm volatile("bar.sync 1, %0;" ::"n"(kPfDqWarps * 32) : "memory");
+            asm volatile("bar.sync %0, %1;" ::"r"(1 + g), "n"(kPfDqWarps * 16) : "memory");
             ++nb_sync;
             return *go != 0;
         };
         Ring rr{0, 0, RD}, rs{0, 0, SD};
-        int j = 0;   // stage
+        if (g == 1)
+            rs.next();   // the group's first stage is stage 1
+        int j = g;       // stage
         bool ok = true;
         for (int i = 0; i < nsb && ok; ++i) {
             if (!gate(raw_full + 8 * rr.slot, rr.phase))
@@ -467,27 +470,33 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1)
             const uint32_t raw = raw_s + rr.slot * kPfRawBytes + r * kQ4KBlockBytes;
             const Hdr hd = decode_hdr(lds128(raw));
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int cc = 0; cc < 2; ++cc) {
+                const int c = g + 2 * cc;
                 if (j >= SD && !gate(empty + 8 * rs.slot, rs.phase ^ 1)) {
                     ok = false;
                     break;
                 }
                 const ChunkScales cs = chunk_scales(hd, c);
-                const uint4 qv = lds128(raw + 16 + 32 * c + 16 * h);
-                uint4 lo0, hi0, lo1, hi1;
-                pf_dequant8(make_uint2(qv.x, qv.y), cs, lo0, hi0);
-                pf_dequant8(make_uint2(qv.z, qv.w), cs, lo1, hi1);
-                const uint32_t at = st_s + rs.slot * stage_bytes;
-                sts128(at + o_lo0, lo0);
-                sts128(at + o_lo1, lo1);
-                sts128(at + o_hi0, hi0);
-                sts128(at + o_hi1, hi1);
+                const uint4 qa = lds128(raw + 16 + 32 * c);
+                const uint4 qb = lds128(raw + 16 + 32 * c + 16);
+                uint4 lo[4], hi[4];
+                pf_dequant8(make_uint2(qa.x, qa.y), cs, lo[0], hi[0]);
+                pf_dequant8(make_uint2(qa.z, qa.w), cs, lo[1], hi[1]);
+                pf_dequant8(make_uint2(qb.x, qb.y), cs, lo[2], hi[2]);
+                pf_dequant8(make_uint2(qb.z, qb.w), cs, lo[3], hi[3]);
+                const uint32_t at = st_s + rs.slot * stage_bytes + row_off;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    sts128(at + ((u ^ sw) << 4), lo[u]);
+                    sts128(at + (((4 + u) ^ sw) << 4), hi[u]);
+                }
                 fence_proxy_async_smem();   // generic-proxy stores -> visible to the tensor cores
                 __syncwarp();
                 if (lane == 0)
-                    mbar_arrive(full + 8 * rs.slot);   // one arrival per warp
+                    mbar_arrive(full + 8 * rs.slot);   // one arrival per warp of the group
                 rs.next();
-                ++j;
+                rs.next();
+                j += 2;
             }
             if (!ok)
                 break;
