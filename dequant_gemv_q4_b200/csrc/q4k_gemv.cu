@@ -59,7 +59,9 @@
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <tuple>
 
 #include "dq_common.cuh"
 #include "dq_internal.h"
@@ -870,14 +872,50 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
     return fn;
 }
 
+// How many clusters of `size` CTAs of the batch-1 kernel (warps x 32 threads,
+// smem bytes of shared memory each) the device runs at once; 0 when the runtime
+// cannot tell.  Cached per shape.
+static int cluster_capacity(int size, int warps, int smem)
+{
+    static std::mutex mu;
+    static std::map<std::tuple<int, int, int>, int> cache;
+    const auto key = std::make_tuple(size, warps, smem);
+    std::lock_guard<std::mutex> lock(mu);
+    const auto it = cache.find(key);
+    if (it != cache.end())
+        return it->second;
+    auto k = q4k_gemv_fx_kernel<1, false, true>;
+    int n = 0;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(size);
+        cfg.blockDim = dim3(warps * 32);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = size;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&n, k, &cfg) != cudaSuccess)
+            n = 0;
+    }
+    cudaGetLastError();
+    cache[key] = n;
+    return n;
+}
+
 // Launch plan.  Slot copies by TMA when the driver's encoder is available.  K
 // is split until there are about eight tile tasks per SM (or each split is one
 // chunk), warps per CTA follow from the tasks per SM, and K is split further
 // if the activations would not fit beside a two-deep ring per warp; the ring
-// is as deep as shared memory allows, up to 4 slots.
+// is as deep as shared memory allows, up to 4 slots.  When the batch-1 splits
+// are added inside clusters, all clusters must be resident at once: the plan
+// then takes the fewest warps per CTA (the most CTAs, hence SMs) whose clusters
+// fit in one wave, and gives up the clusters if none does.
 static Q4KPlan plan_quarter_warp(long long N, int nb, int B, int NS, int sm_count, int smem_optin)
 {
-    Q4KPlan pl{};
     // DQGEMV_NO_TMA=1 selects the per-row bulk copies (same shared-memory
     // layout, bit-identical results), for comparing the two copy paths
     const char *no_tma = getenv("DQGEMV_NO_TMA");
@@ -892,8 +930,8 @@ static Q4KPlan plan_quarter_warp(long long N, int nb, int B, int NS, int sm_coun
     int splits_par = 1;
     while (tiles * splits_par < 8LL * sm_count && splits_par < nchunk)
         ++splits_par;
-    const int w0 = pick_warps(tiles * splits_par, sm_count, max_warps);
-    for (int warps = w0; warps >= 4 && !pl.ok; --warps) {
+    auto plan_for = [&](int warps, bool allow_cluster) {
+        Q4KPlan pl{};
         int splits = splits_par;
         int cps = (nchunk + splits - 1) / splits;
         while (cps * kFxBPC * stage + warps * 2 * kFxSlotBytes + misc > smem_optin && cps > 1) {
@@ -906,7 +944,7 @@ static Q4KPlan plan_quarter_warp(long long N, int nb, int B, int NS, int sm_coun
         if (depth > 4)
             depth = 4;
         if (depth < 2)
-            continue;
+            return pl;
         long long ctas = (tiles + warps - 1) / warps;
         const long long max_ctas = sm_count / splits > 0 ? sm_count / splits : 1;
         if (ctas > max_ctas)
@@ -922,12 +960,32 @@ static Q4KPlan plan_quarter_warp(long long N, int nb, int B, int NS, int sm_coun
         pl.grid = pl.ctas_per_split * splits;
         pl.smem = x_bytes + ((warps * depth * 8 + 127) & ~127) + 128 + warps * depth * kFxSlotBytes + 256;
         // batch-1 splits of at most one tile per warp are added inside a cluster
-        pl.cluster = B == 1 && splits > 1 && splits <= kFxMaxCluster &&
+        pl.cluster = allow_cluster && B == 1 && splits > 1 && splits <= kFxMaxCluster &&
                      tiles <= static_cast<long long>(pl.ctas_per_split) * warps &&
                      pl.smem + warps * kFxClusterPartBytes <= smem_optin;
         if (pl.cluster)
             pl.smem += warps * kFxClusterPartBytes;
         pl.ok = pl.smem <= smem_optin;
+        return pl;
+    };
+    auto first_fit = [&](bool allow_cluster) {
+        Q4KPlan pl{};
+        for (int warps = pick_warps(tiles * splits_par, sm_count, max_warps); warps >= 4 && !pl.ok; --warps)
+            pl = plan_for(warps, allow_cluster);
+        return pl;
+    };
+    Q4KPlan pl = first_fit(true);
+    if (pl.ok && pl.cluster) {
+        const int cap = cluster_capacity(pl.splits, pl.warps, pl.smem);
+        if (cap > 0) {
+            for (int warps = 4; warps <= max_warps; ++warps) {
+                const Q4KPlan c = plan_for(warps, true);
+                if (c.ok && c.cluster && c.ctas_per_split <= cluster_capacity(c.splits, c.warps, c.smem))
+                    return c;
+            }
+            if (pl.ctas_per_split > cap)
+                pl = first_fit(false);
+        }
     }
     return pl;
 }
