@@ -908,7 +908,8 @@ static int cluster_capacity(int size, int warps, int smem)
 
 // Launch plan.  Slot copies by TMA when the driver's encoder is available.  K
 // is split until there are about eight tile tasks per SM (or each split is one
-// chunk), warps per CTA follow from the tasks per SM, and K is split further
+// chunk), warps per CTA follow from the tasks per SM (batch 1) or from covering
+// the tiles with whole groups of four warps (batches 2-8), and K is split further
 // if the activations would not fit beside a two-deep ring per warp; the ring
 // is as deep as shared memory allows, up to 4 slots.  When the batch-1 splits
 // are added inside clusters, all clusters must be resident at once: the plan
@@ -968,9 +969,25 @@ static Q4KPlan plan_quarter_warp(long long N, int nb, int B, int NS, int sm_coun
         pl.ok = pl.smem <= smem_optin;
         return pl;
     };
+    // Warps per CTA to start from.  Batch 1: from the tile tasks per SM.  Batches 2-8 (one tile per
+    // warp and the same work per tile): the fewest warps, in multiples of four (one per scheduler),
+    // whose CTAs cover every tile on the SMs left to each split once the splits are whole numbers of
+    // chunks; a count that is not a multiple of four leaves one scheduler with an extra tile.
+    int w_start = pick_warps(tiles * splits_par, sm_count, max_warps);
+    if (B > 1) {
+        const int cps0 = (nchunk + splits_par - 1) / splits_par;
+        const int splits_eff = (nchunk + cps0 - 1) / cps0;
+        const long long per_split = sm_count / splits_eff > 0 ? sm_count / splits_eff : 1;
+        w_start = max_warps;
+        for (int w = 4; w <= max_warps; w += 4)
+            if ((tiles + w - 1) / w <= per_split) {
+                w_start = w;
+                break;
+            }
+    }
     auto first_fit = [&](bool allow_cluster) {
         Q4KPlan pl{};
-        for (int warps = pick_warps(tiles * splits_par, sm_count, max_warps); warps >= 4 && !pl.ok; --warps)
+        for (int warps = w_start; warps >= 4 && !pl.ok; --warps)
             pl = plan_for(warps, allow_cluster);
         return pl;
     };
