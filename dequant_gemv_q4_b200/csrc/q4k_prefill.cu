@@ -208,6 +208,31 @@ struct Ring {
     }
 };
 
+// Bounded wait for the single threads on the pipeline's critical path (the
+// producers, the MMA issuer and the group leaders): mbarrier.try_wait with the
+// system's own suspend limit, so that the thread resumes as soon as the phase
+// completes.  Otherwise as pf_wait.
+__device__ __forceinline__ bool pf_wait_fast(uint32_t bar, uint32_t parity, int *err, volatile int *abort)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const unsigned long long t0 = global_ns();
+    for (uint32_t i = 0;; ++i) {
+        if (mbar_try_wait(bar, parity))
+            return true;
+        if ((i & 15) == 15) {
+            if (abort && *abort)
+                return false;
+            if (global_ns() - t0 > kWaitNanos)
+                break;
+        }
+    }
+    atomicExch(err, kDevErrWaitTimeout);
+    if (abort)
+        *abort = 1;
+    return false;
+}
+
 // pf_wait by lane 0 of a warp for the whole warp (one sleeping waiter instead of
 // 32); the outcome is the same for every lane, and __syncwarp orders the lanes'
 // later shared-memory accesses after lane 0's observation of the phase.
@@ -357,7 +382,7 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1)
             int kbi = rot;    // super-block, relative to kb0
             int issued = 0;
             for (; issued < nsb; ++issued) {
-                if (issued >= RD && !pf_wait(raw_empty + 8 * r.slot, r.phase ^ 1, p.err, abort))
+                if (issued >= RD && !pf_wait_fast(raw_empty + 8 * r.slot, r.phase ^ 1, p.err, abort))
                     break;
                 const uint32_t bar = raw_full + 8 * r.slot;
                 const uint32_t dst = raw_s + r.slot * kPfRawBytes;
@@ -387,7 +412,7 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1)
             int kbi = rot, quarter = 0;
             int issued = 0;
             for (; issued < nst; ++issued) {
-                if (issued >= SD && !pf_wait(empty + 8 * r.slot, r.phase ^ 1, p.err, abort))
+                if (issued >= SD && !pf_wait_fast(empty + 8 * r.slot, r.phase ^ 1, p.err, abort))
                     break;
                 const uint32_t bar = full + 8 * r.slot;
                 const uint32_t dst = st_s + r.slot * stage_bytes + kPfWTileBytes;
@@ -416,7 +441,7 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1)
             const uint64_t x_desc0 = pf_desc_sw128(st_s + kPfWTileBytes);
             const uint32_t idesc = p.idesc;
             for (int j = 0; j < nst; ++j) {
-                if (!pf_wait(full + 8 * r.slot, r.phase, p.err, abort))
+                if (!pf_wait_fast(full + 8 * r.slot, r.phase, p.err, abort))
                     break;
                 pf_fence_after();
                 const uint64_t soff = static_cast<uint64_t>(r.slot * (stage_bytes >> 4));
@@ -454,7 +479,7 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1)
         auto gate = [&](uint32_t bar, uint32_t parity) -> bool {
             volatile int *go = s_go + 2 * g + (nb_sync & 1);
             if (leader)
-                *go = pf_wait(bar, parity, p.err, abort) ? 1 : 0;
+                *go = pf_wait_fast(bar, parity, p.err, abort) ? 1 : 0;
             asm volatile("bar.sync %0, %1;" ::"r"(1 + g), "n"(kPfDqWarps * 16) : "memory");
             ++nb_sync;
             return *go != 0;
