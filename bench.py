@@ -49,8 +49,8 @@ FALLBACK_HBM_GBS = 6650.0
 
 # DRAM bytes (read + write) per launch of q4k_gemv_fx_kernel on this workload,
 # from one ncu capture, valid only for the kernel sources whose hash is recorded.
-NCU_TRAFFIC = {"sources_sha1": "1a37c6872009d47e7d6c97a67263bfa6448cbdde",
-               "bytes_per_launch": 572207872 + 4249856}   # profiles/q4k_gemv_fx_kernel_248320x4096_dram.md
+NCU_TRAFFIC = {"sources_sha1": "97e73226d35cc0a24934390a6c594a86437ad853",
+               "bytes_per_launch": 572207616 + 4335872}   # profiles/q4k_gemv_fx_kernel_248320x4096_dram.md
 
 
 def kernel_sources_sha1() -> str:

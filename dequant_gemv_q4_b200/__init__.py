@@ -34,7 +34,7 @@ Q8_0_BLOCK_ELEMS, Q8_0_BLOCK_BYTES = 32, 34
 EXPORTED = ("q8_0_gemv", "q4k_gemv", "q4k_swiglu_gemv", "q4k_repack_soa", "dq_workspace_bytes",
             "q8_0_dequant", "q4k_dequant", "dq_status_string", "dq_last_cuda_error",
             "dq_device_error", "q4k_gemv_noalloc", "dq_noalloc_scratch_bytes", "q4k_gemv_split_qg",
-            "q4k_gemv_group", "q4k_prefill_gemm")
+            "q4k_gemv_group", "q4k_prefill_gemm", "q4k_gemv_residual")
 
 
 class DQError(RuntimeError):
@@ -77,6 +77,7 @@ def load_library(path: str = LIB_PATH):
             "q4k_gemv_split_qg": [p, i32, p, p, p, i64, i64, i32, i64, p, sz, p],
             "q4k_gemv_group": [i32, p, p, p, i32, p, i64, p, sz, p],
             "q4k_prefill_gemm": [p, i32, p, p, i64, i64, i64, p, sz, p],
+            "q4k_gemv_residual": [p, i32, p, p, p, i64, i64, i32, p, p, sz, p],
         }
         for name, args in sigs.items():
             f = getattr(lib, name)
@@ -204,6 +205,37 @@ def q4k_gemv(w, x, N: int, K: int, layout="aos", y=None, argmax: bool = False, w
     wsp, wsn, _keep = _workspace(workspace, need, x.device)
     _check("q4k_gemv", lib.q4k_gemv(wp, _layout(layout), ctypes.c_void_p(x2.data_ptr()), yp, N, K, B,
                                     ip, wsp, wsn, _stream(stream)))
+    out = y.view(N) if one_d else y.view(B, N)
+    return (out, idx) if argmax else out
+
+
+def q4k_gemv_residual(w, x, residual, N: int, K: int, layout="aos", y=None, argmax: bool = False,
+                      workspace=None, stream=None):
+    """y = W x + residual (the FFN block's down projection with its residual add);
+    residual has y's shape and may be y itself.  Returns as q4k_gemv."""
+    torch = _torch()
+    lib = load_library()
+    one_d = x.dim() == 1
+    x2 = _x2d(x, K)
+    B = x2.shape[0]
+    wp = _weights(w, "w", N, K, Q4K_BLOCK_ELEMS, Q4K_BLOCK_BYTES)
+    rp = _dev(residual, "residual", torch.float32)
+    if residual.numel() != B * N:
+        raise ValueError("residual must hold B*N floats")
+    if y is None:
+        y = torch.empty((B, N), dtype=torch.float32, device=x.device)
+    yp = _dev(y, "y", torch.float32)
+    if y.numel() != B * N:
+        raise ValueError("y must hold B*N floats")
+    idx = None
+    ip = ctypes.c_void_p(0)
+    if argmax:
+        idx = torch.empty(1, dtype=torch.int64, device=x.device)
+        ip = ctypes.c_void_p(idx.data_ptr())
+    need = dq_workspace_bytes(DQ_OP_Q4K_GEMV, N, K, B, argmax)
+    wsp, wsn, _keep = _workspace(workspace, need, x.device)
+    _check("q4k_gemv_residual", lib.q4k_gemv_residual(wp, _layout(layout), ctypes.c_void_p(x2.data_ptr()), rp, yp,
+                                                      N, K, B, ip, wsp, wsn, _stream(stream)))
     out = y.view(N) if one_d else y.view(B, N)
     return (out, idx) if argmax else out
 

@@ -99,7 +99,7 @@ size_t prefill_ws_bytes(const dq::PrefillPlan &pl, int64_t N, int64_t M)
 dq_status q4k_common(const void *w0, const void *w1, int layout, const float *x, float *y, int64_t N, int64_t K,
                      int B, int NS, int64_t *argmax_out, void *workspace, size_t ws_bytes, void *stream,
                      float *g_out = nullptr, int64_t qg_hd = 0, const dq::GroupOut *grp = nullptr,
-                     const void *const *gw = nullptr)
+                     const void *const *gw = nullptr, const float *res = nullptr)
 {
     if (!w0 || (NS == 2 && !w1) || !x || !y)
         return DQ_ERR_NULL;
@@ -134,6 +134,7 @@ dq_status q4k_common(const void *w0, const void *w1, int layout, const float *x,
     p.x = x;
     p.y = y;
     p.g = g_out;
+    p.res = res;
     p.qg_hd = static_cast<int>(qg_hd);
     if (grp) {
         p.grp = *grp;
@@ -159,7 +160,8 @@ dq_status q4k_common(const void *w0, const void *w1, int layout, const float *x,
     if (e != cudaSuccess)
         return cuda_fail(e);
     if (pl.splits > 1 && !pl.cluster) {
-        e = dq::splitk_reduce_launch(p.part, pl.splits, NS, B, N, y, p.g, p.qg_hd, p.grp, p.cand, dq::reduce_grid(N, B),
+        e = dq::splitk_reduce_launch(p.part, pl.splits, NS, B, N, y, p.g, p.qg_hd, p.grp, p.res, p.cand,
+                                     dq::reduce_grid(N, B),
                                      s);
         if (e != cudaSuccess)
             return cuda_fail(e);
@@ -231,6 +233,17 @@ dq_status q4k_gemv(const void *w, int layout, const float *x, float *y, int64_t 
                    int64_t *argmax_out, void *workspace, size_t ws_bytes, void *stream)
 {
     return q4k_common(w, nullptr, layout, x, y, N, K, B, 1, argmax_out, workspace, ws_bytes, stream);
+}
+
+dq_status q4k_gemv_residual(const void *w, int layout, const float *x, const float *residual, float *y, int64_t N,
+                            int64_t K, int B, int64_t *argmax_out, void *workspace, size_t ws_bytes, void *stream)
+{
+    if (!residual)
+        return DQ_ERR_NULL;
+    if (!aligned(residual, 4))
+        return DQ_ERR_ALIGN;
+    return q4k_common(w, nullptr, layout, x, y, N, K, B, 1, argmax_out, workspace, ws_bytes, stream, nullptr, 0,
+                      nullptr, nullptr, residual);
 }
 
 dq_status q4k_prefill_gemm(const void *w, int layout, const uint16_t *x16, float *y, int64_t N, int64_t K, int64_t M,

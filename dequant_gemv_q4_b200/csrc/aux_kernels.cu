@@ -189,8 +189,9 @@ int reduce_grid(long long N, int B)
 
 __global__ void __launch_bounds__(kReduceThreads) splitk_reduce_kernel(const float *__restrict__ part, int splits,
                                                                        int NS, int B, long long N,
-                                                                       float *__restrict__ y, float *__restrict__ g_out,
-                                                                       int qg_hd, const GroupOut grp, ArgmaxCand *cand)
+                                                                       float *y, float *__restrict__ g_out,
+                                                                       int qg_hd, const GroupOut grp,
+                                                                       const float *res, ArgmaxCand *cand)
 {
     pdl_wait();
     pdl_launch_dependents();
@@ -207,7 +208,7 @@ __global__ void __launch_bounds__(kReduceThreads) splitk_reduce_kernel(const flo
             if (NS == 2)
                 u += part[((static_cast<long long>(s) * NS + 1) * B + b) * N + n];
         }
-        const float out = (NS == 2) ? g / (1.0f + expf(-g)) * u : g;
+        const float out = (NS == 2) ? g / (1.0f + expf(-g)) * u : (res ? g + res[i] : g);
         if (grp.n > 0) {
             // padded row n of a grouped GEMV: the matrix holding it, and its row there
             int m = 0;
@@ -255,10 +256,11 @@ __global__ void __launch_bounds__(kReduceThreads) splitk_reduce_kernel(const flo
 }
 
 cudaError_t splitk_reduce_launch(const float *part, int splits, int NS, int B, long long N, float *y, float *g,
-                                 int qg_hd, const GroupOut &grp, ArgmaxCand *cand, int grid, cudaStream_t s)
+                                 int qg_hd, const GroupOut &grp, const float *res, ArgmaxCand *cand, int grid,
+                                 cudaStream_t s)
 {
     return launch_pdl(splitk_reduce_kernel, dim3(grid), dim3(kReduceThreads), 0, s, part, splits, NS, B, N, y, g,
-                      qg_hd, grp, cand);
+                      qg_hd, grp, res, cand);
 }
 
 // One CTA folds all candidates into the final index.

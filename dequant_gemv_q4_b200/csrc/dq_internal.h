@@ -30,6 +30,7 @@ struct Q4KParams {
     const float *x;        // B x K
     float *y;              // B x N final output (splits == 1); Q when qg_hd > 0
     float *g;              // G output of the fused Q/gate split (qg_hd > 0), else null
+    const float *res;      // B x N residual added to the plain output (may alias y), or null
     int qg_hd;             // head dim of the fused Q/gate split, 0 for a plain output
     float *part;           // [splits][NS][B][N] partial sums (splits > 1)
     ArgmaxCand *cand;      // per-CTA argmax candidates (argmax, splits == 1)
@@ -90,7 +91,8 @@ cudaError_t q8_0_gemv_launch(const Q8Params &p, const Q8Plan &pl, int B, cudaStr
 // split-K reduction (+ SwiGLU epilogue, + argmax candidates), argmax finalisation
 int reduce_grid(long long N, int B);
 cudaError_t splitk_reduce_launch(const float *part, int splits, int NS, int B, long long N, float *y, float *g,
-                                 int qg_hd, const GroupOut &grp, ArgmaxCand *cand, int grid, cudaStream_t s);
+                                 int qg_hd, const GroupOut &grp, const float *res, ArgmaxCand *cand, int grid,
+                                 cudaStream_t s);
 cudaError_t argmax_finalize_launch(const ArgmaxCand *cand, int ncand, long long *out, cudaStream_t s);
 
 // debug dequant, repack

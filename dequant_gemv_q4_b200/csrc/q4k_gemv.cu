@@ -514,6 +514,8 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
                 out = gv / (1.0f + expf(-gv)) * static_cast<float>(t);
             } else {
                 out = static_cast<float>(t);
+                if (p.res)
+                    out += p.res[n];
             }
             *gemv_out_addr(p.y, p.g, p.qg_hd, p.N, 0, n) = out;
             if (p.argmax && cand_better(out, n, best_v, best_i)) {
@@ -560,6 +562,8 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
                     out = gv / (1.0f + expf(-gv)) * static_cast<float>(u);
                 } else {
                     out = static_cast<float>(g);
+                    if (p.res)
+                        out += p.res[n];
                 }
                 *gemv_out_addr(p.y, p.g, p.qg_hd, p.N, 0, n) = out;
                 if (p.argmax && cand_better(out, n, best_v, best_i)) {
@@ -821,6 +825,8 @@ __global__ void __launch_bounds__(kFxbMaxWarps(B) * 32, 1)
                     out = gv / (1.0f + expf(-gv)) * (v[k] * 0x1p64f);
                 } else {
                     out = v[k] * 0x1p64f;
+                    if (p.res)
+                        out += p.res[static_cast<long long>(b) * p.N + n];
                 }
                 *gemv_out_addr(p.y, p.g, p.qg_hd, p.N, b, n) = out;
             }

@@ -117,6 +117,18 @@ dq_status q4k_gemv(const void *w, int layout, const float *x, float *y, int64_t 
                    int B, int64_t *argmax_out, void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * Q4_K GEMV with a fused residual add, the down projection of a decoder
+ * layer's FFN block (qualiaDB cuda_lane: try_q4k_soa_ffn_block_residual):
+ *   y[b][n] = sum_k W[n][k] * x[b][k] + residual[b][n].
+ *   residual  B x N fp32, 4-byte aligned; it may be y itself (y += W x).
+ *   Other arguments, the workspace and argmax (over the sums) as for q4k_gemv.
+ * The product is formed exactly as q4k_gemv forms it, rounded to fp32, and the
+ * residual is then added in fp32.
+ */
+dq_status q4k_gemv_residual(const void *w, int layout, const float *x, const float *residual, float *y, int64_t N,
+                            int64_t K, int B, int64_t *argmax_out, void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * Q4_K GEMV of a q-projection-with-gate matrix with the Q/gate de-interleave
  * fused into the store (Doppler 0.1.8, split_qg.wgsl: "attentionOutputGate"
  * models interleave, per head, head_dim Q rows and head_dim gate rows):

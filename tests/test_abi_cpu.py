@@ -162,3 +162,13 @@ def test_prefill_rejects_on_host(lib):
     bad = ctypes.c_size_t(-1).value
     assert lib.dq_workspace_bytes(3, 128, 250, 16, 0) == bad
     assert lib.dq_workspace_bytes(3, 128, 256, 16, 1) == bad                    # no argmax
+
+
+def test_residual_gemv_rejects_on_host(lib):
+    f = lib.q4k_gemv_residual
+    f.argtypes = [P, ctypes.c_int, P, P, P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, P, P, ctypes.c_size_t, P]
+    assert f(A16, 0, A16, None, A16, 64, 256, 1, None, None, 0, None) == DQ_ERR_NULL
+    assert f(A16, 0, A16, P((1 << 20) + 2), A16, 64, 256, 1, None, None, 0, None) == DQ_ERR_ALIGN
+    # the GEMV's own checks still apply
+    assert f(A16, 0, A16, A16, A16, 64, 100, 1, None, None, 0, None) == DQ_ERR_SHAPE
+    assert f(A16, 0, A16, A16, A16, 64, 256, 9, None, None, 0, None) == DQ_ERR_SHAPE

@@ -604,3 +604,30 @@ def test_q4k_prefill_is_deterministic_and_soa_equals_aos():
     y3 = host(dq.q4k_prefill_gemm(dev(oracle.q4k_repack_soa(w, N, K)), x16, N, K, layout="soa"))
     assert np.array_equal(y1.view(np.uint32), y2.view(np.uint32))
     assert np.array_equal(y1.view(np.uint32), y3.view(np.uint32))
+
+
+# --- fused residual add (FFN block down projection) ----------------------------------------
+
+@pytest.mark.parametrize("N,K,B,inplace", [
+    (4096, 12288, 1, False),   # the down projection, K split in clusters
+    (4096, 12288, 1, True),    # y += W x
+    (1000, 4096, 3, False),    # batch 3
+    (300, 65536, 1, True),     # long K: split-K reduction kernel
+    (77, 1024, 2, True),
+])
+def test_q4k_gemv_residual_is_the_gemv_plus_the_residual(N, K, B, inplace):
+    rng = np.random.default_rng(N + K + B)
+    w = synth.q4k_matrix(rng, N, K)
+    x = synth.activations(rng, B, K)
+    r = synth.activations(rng, B, N, scale=4.0)
+    rd = dev(r)
+    y = dq.q4k_gemv_residual(dev(w), dev(x), rd, N, K, y=rd if inplace else None)
+    got = host(y).reshape(B, N).astype(np.float64)
+    plain = host(dq.q4k_gemv(dev(w), dev(x), N, K)).reshape(B, N)
+    y_ref, a_ref = oracle_rows(lambda rows: oracle.q4k_gemv(w, N, K, x, rows=rows), N, np.arange(N))
+    want = y_ref + r.astype(np.float64)
+    # the GEMV rule, plus one fp32 rounding of the sum
+    tol = oracle.gemv_tolerance(a_ref) + np.abs(want) * 2.0 ** -23
+    assert np.all(np.abs(got - want) <= tol)
+    # and exactly the fp32 sum of q4k_gemv's own output and the residual
+    assert np.array_equal(got.astype(np.float32), (plain + r).astype(np.float32))
