@@ -26,6 +26,7 @@ DQ_OP_Q8_0_GEMV = 0
 DQ_OP_Q4K_GEMV = 1
 DQ_OP_Q4K_SWIGLU = 2
 DQ_OP_Q4K_PREFILL = 3
+DQ_OP_Q4K_FFN = 4
 MAX_PREFILL_M = 65536
 
 Q4K_BLOCK_ELEMS, Q4K_BLOCK_BYTES = 256, 144
@@ -34,7 +35,7 @@ Q8_0_BLOCK_ELEMS, Q8_0_BLOCK_BYTES = 32, 34
 EXPORTED = ("q8_0_gemv", "q4k_gemv", "q4k_swiglu_gemv", "q4k_repack_soa", "dq_workspace_bytes",
             "q8_0_dequant", "q4k_dequant", "dq_status_string", "dq_last_cuda_error",
             "dq_device_error", "q4k_gemv_noalloc", "dq_noalloc_scratch_bytes", "q4k_gemv_split_qg",
-            "q4k_gemv_group", "q4k_prefill_gemm", "q4k_gemv_residual")
+            "q4k_gemv_group", "q4k_prefill_gemm", "q4k_gemv_residual", "q4k_ffn_block")
 
 
 class DQError(RuntimeError):
@@ -78,6 +79,7 @@ def load_library(path: str = LIB_PATH):
             "q4k_gemv_group": [i32, p, p, p, i32, p, i64, p, sz, p],
             "q4k_prefill_gemm": [p, i32, p, p, i64, i64, i64, p, sz, p],
             "q4k_gemv_residual": [p, i32, p, p, p, i64, i64, i32, p, p, sz, p],
+            "q4k_ffn_block": [p, p, p, i32, p, p, p, i64, i64, i32, p, sz, p],
         }
         for name, args in sigs.items():
             f = getattr(lib, name)
@@ -238,6 +240,35 @@ def q4k_gemv_residual(w, x, residual, N: int, K: int, layout="aos", y=None, argm
                                                       N, K, B, ip, wsp, wsn, _stream(stream)))
     out = y.view(N) if one_d else y.view(B, N)
     return (out, idx) if argmax else out
+
+
+def q4k_ffn_block(w_gate, w_up, w_down, x, H: int, F: int, residual=None, layout="aos", y=None,
+                  workspace=None, stream=None):
+    """A decoder layer's FFN block: y = W_down (silu(W_gate x) * (W_up x)) [+ residual].
+    x: (H,) or (B, H) fp32; W_gate, W_up: F x H; W_down: H x F.  residual may be x or y."""
+    torch = _torch()
+    lib = load_library()
+    one_d = x.dim() == 1
+    x2 = _x2d(x, H)
+    B = x2.shape[0]
+    gp = _weights(w_gate, "w_gate", F, H, Q4K_BLOCK_ELEMS, Q4K_BLOCK_BYTES)
+    up = _weights(w_up, "w_up", F, H, Q4K_BLOCK_ELEMS, Q4K_BLOCK_BYTES)
+    dp = _weights(w_down, "w_down", H, F, Q4K_BLOCK_ELEMS, Q4K_BLOCK_BYTES)
+    rp = ctypes.c_void_p(0)
+    if residual is not None:
+        rp = _dev(residual, "residual", torch.float32)
+        if residual.numel() != B * H:
+            raise ValueError("residual must hold B*H floats")
+    if y is None:
+        y = torch.empty((B, H), dtype=torch.float32, device=x.device)
+    yp = _dev(y, "y", torch.float32)
+    if y.numel() != B * H:
+        raise ValueError("y must hold B*H floats")
+    need = dq_workspace_bytes(DQ_OP_Q4K_FFN, H, F, B)
+    wsp, wsn, _keep = _workspace(workspace, need, x.device)
+    _check("q4k_ffn_block", lib.q4k_ffn_block(gp, up, dp, _layout(layout), ctypes.c_void_p(x2.data_ptr()), rp, yp,
+                                              H, F, B, wsp, wsn, _stream(stream)))
+    return y.view(H) if one_d else y.view(B, H)
 
 
 def q4k_gemv_noalloc(w, x, N: int, K: int, layout="aos", y=None, argmax: bool = False, stream=None):

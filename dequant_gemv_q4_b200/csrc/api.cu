@@ -84,6 +84,40 @@ dq_status check_q4k_shape(int64_t N, int64_t K, int B)
     return DQ_OK;
 }
 
+// Scratch of one Q4_K GEMV (NS = 1) or SwiGLU pair (NS = 2) on the current
+// device, for either layout; (size_t)-1 if the shape has no plan.
+size_t q4k_gemv_ws_bytes(int64_t N, int64_t K, int B, int NS, bool argmax)
+{
+    const size_t bad = static_cast<size_t>(-1);
+    if (check_q4k_shape(N, K, B) != DQ_OK)
+        return bad;
+    DevInfo di;
+    if (dev_info(di) != DQ_OK)
+        return bad;
+    size_t need = 0;
+    for (int soa = 0; soa < 2; ++soa) {
+        const dq::Q4KPlan pl = dq::q4k_plan(N, static_cast<int>(K), B, NS, soa, di.sm_count, di.smem_optin);
+        if (!pl.ok)
+            return bad;
+        const size_t t = q4k_ws(pl, N, B, NS, argmax).total();
+        if (t > need)
+            need = t;
+    }
+    return need;
+}
+
+// FFN block scratch: the SwiGLU output h (B x F) and then the larger of the two
+// GEMVs' own scratch.
+size_t ffn_ws_bytes(int64_t H, int64_t F, int B)
+{
+    const size_t bad = static_cast<size_t>(-1);
+    const size_t a = q4k_gemv_ws_bytes(F, H, B, 2, false);
+    const size_t b = q4k_gemv_ws_bytes(H, F, B, 1, false);
+    if (a == bad || b == bad)
+        return bad;
+    return round_up(static_cast<size_t>(B) * F * sizeof(float), 256) + (a > b ? a : b);
+}
+
 dq_status check_prefill_shape(int64_t N, int64_t K, int64_t M)
 {
     if (N < 1 || N > 0x7FFFFFFFLL || K < 256 || K % 256 != 0 || K > DQ_MAX_K || M < 1 || M > DQ_MAX_PREFILL_M)
@@ -235,6 +269,43 @@ dq_status q4k_gemv(const void *w, int layout, const float *x, float *y, int64_t 
     return q4k_common(w, nullptr, layout, x, y, N, K, B, 1, argmax_out, workspace, ws_bytes, stream);
 }
 
+dq_status q4k_ffn_block(const void *w_gate, const void *w_up, const void *w_down, int layout, const float *x,
+                        const float *residual, float *y, int64_t H, int64_t F, int B, void *workspace, size_t ws_bytes,
+                        void *stream)
+{
+    if (!w_gate || !w_up || !w_down || !x || !y)
+        return DQ_ERR_NULL;
+    if (layout != DQ_LAYOUT_AOS && layout != DQ_LAYOUT_SOA)
+        return DQ_ERR_LAYOUT;
+    dq_status st = check_q4k_shape(F, H, B);
+    if (st != DQ_OK)
+        return st;
+    if ((st = check_q4k_shape(H, F, B)) != DQ_OK)
+        return st;
+    if (!aligned(w_gate, 16) || !aligned(w_up, 16) || !aligned(w_down, 16) || !aligned(x, 16) || !aligned(y, 4) ||
+        (residual && !aligned(residual, 4)))
+        return DQ_ERR_ALIGN;
+    // everything either GEMV could reject is checked here, before the first launch
+    const size_t need = ffn_ws_bytes(H, F, B);
+    if (need == static_cast<size_t>(-1))
+        return DQ_ERR_SHAPE;
+    if (!workspace || ws_bytes < need)
+        return DQ_ERR_WORKSPACE;
+    if (!aligned(workspace, 16))
+        return DQ_ERR_ALIGN;
+    const size_t hbytes = round_up(static_cast<size_t>(B) * F * sizeof(float), 256);
+    float *h = static_cast<float *>(workspace);
+    void *rest = static_cast<uint8_t *>(workspace) + hbytes;
+    const size_t rest_bytes = ws_bytes - hbytes;
+    st = q4k_common(w_gate, w_up, layout, x, h, F, H, B, 2, nullptr, rest, rest_bytes, stream);
+    if (st != DQ_OK)
+        return st;
+    if (residual)
+        return q4k_common(w_down, nullptr, layout, h, y, H, F, B, 1, nullptr, rest, rest_bytes, stream, nullptr, 0,
+                          nullptr, nullptr, residual);
+    return q4k_common(w_down, nullptr, layout, h, y, H, F, B, 1, nullptr, rest, rest_bytes, stream);
+}
+
 dq_status q4k_gemv_residual(const void *w, int layout, const float *x, const float *residual, float *y, int64_t N,
                             int64_t K, int B, int64_t *argmax_out, void *workspace, size_t ws_bytes, void *stream)
 {
@@ -384,6 +455,8 @@ dq_status q4k_repack_soa(const void *w_aos, void *w_soa, int64_t N, int64_t K, v
 size_t dq_workspace_bytes(int op, int64_t N, int64_t K, int B, int with_argmax)
 {
     const size_t bad = static_cast<size_t>(-1);
+    if (op == DQ_OP_Q4K_FFN)
+        return with_argmax ? bad : ffn_ws_bytes(N, K, B);
     if (op == DQ_OP_Q4K_PREFILL) {
         if (with_argmax || check_prefill_shape(N, K, B) != DQ_OK)
             return bad;
@@ -400,26 +473,12 @@ size_t dq_workspace_bytes(int op, int64_t N, int64_t K, int B, int with_argmax)
     }
     if (op != DQ_OP_Q4K_GEMV && op != DQ_OP_Q4K_SWIGLU)
         return bad;
-    if (check_q4k_shape(N, K, B) != DQ_OK)
-        return bad;
     const int NS = (op == DQ_OP_Q4K_SWIGLU) ? 2 : 1;
     if (with_argmax && (B != 1 || NS != 1))
         return bad;
-    DevInfo di;
-    if (dev_info(di) != DQ_OK)
-        return bad;
     // the plan does not depend on the layout except through the chunk width,
     // so take the larger of the two requirements
-    size_t need = 0;
-    for (int soa = 0; soa < 2; ++soa) {
-        const dq::Q4KPlan pl = dq::q4k_plan(N, static_cast<int>(K), B, NS, soa, di.sm_count, di.smem_optin);
-        if (!pl.ok)
-            return bad;
-        const size_t t = q4k_ws(pl, N, B, NS, with_argmax != 0).total();
-        if (t > need)
-            need = t;
-    }
-    return need;
+    return q4k_gemv_ws_bytes(N, K, B, NS, with_argmax != 0);
 }
 
 dq_status q8_0_dequant(const void *w, float *out, int64_t N, int64_t K, void *stream)

@@ -83,7 +83,8 @@ typedef enum dq_op {
     DQ_OP_Q8_0_GEMV = 0,
     DQ_OP_Q4K_GEMV = 1,
     DQ_OP_Q4K_SWIGLU = 2,
-    DQ_OP_Q4K_PREFILL = 3   /* q4k_prefill_gemm; the `B` argument is M */
+    DQ_OP_Q4K_PREFILL = 3,  /* q4k_prefill_gemm; the `B` argument is M */
+    DQ_OP_Q4K_FFN = 4       /* q4k_ffn_block; the `N`, `K` arguments are H, F */
 } dq_op;
 
 /* Largest K accepted by the GEMV entry points (fp32 activations of one split
@@ -127,6 +128,27 @@ dq_status q4k_gemv(const void *w, int layout, const float *x, float *y, int64_t 
  */
 dq_status q4k_gemv_residual(const void *w, int layout, const float *x, const float *residual, float *y, int64_t N,
                             int64_t K, int B, int64_t *argmax_out, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * A decoder layer's FFN block in one call (qualiaDB cuda_lane:
+ * try_q4k_soa_ffn_block, try_q4k_soa_ffn_block_residual):
+ *   h = silu(W_gate x) * (W_up x)        (B x F; q4k_swiglu_gemv)
+ *   y = W_down h [+ residual]            (B x H; q4k_gemv / q4k_gemv_residual)
+ * as two launches on `stream`, the second chained to the first by programmatic
+ * dependent launch; h lives in the workspace.
+ *   w_gate, w_up  F x H Q4_K matrices;  w_down  H x F;  all in `layout`,
+ *                 16-byte aligned.
+ *   x             B x H fp32, 16-byte aligned.   y  B x H fp32, 4-byte aligned.
+ *   residual      NULL, or B x H fp32, 4-byte aligned; it may be x or y
+ *                 (y = x + FFN(x) in place is allowed).
+ *   H, F          positive multiples of 256.     B  1..8.
+ *   workspace     at least dq_workspace_bytes(DQ_OP_Q4K_FFN, H, F, B, 0) bytes.
+ * Every argument is checked before the first launch.  The results are exactly
+ * those of the two separate calls.
+ */
+dq_status q4k_ffn_block(const void *w_gate, const void *w_up, const void *w_down, int layout, const float *x,
+                        const float *residual, float *y, int64_t H, int64_t F, int B, void *workspace, size_t ws_bytes,
+                        void *stream);
 
 /*
  * Q4_K GEMV of a q-projection-with-gate matrix with the Q/gate de-interleave

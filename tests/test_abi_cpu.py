@@ -172,3 +172,17 @@ def test_residual_gemv_rejects_on_host(lib):
     # the GEMV's own checks still apply
     assert f(A16, 0, A16, A16, A16, 64, 100, 1, None, None, 0, None) == DQ_ERR_SHAPE
     assert f(A16, 0, A16, A16, A16, 64, 256, 9, None, None, 0, None) == DQ_ERR_SHAPE
+
+
+def test_ffn_block_rejects_on_host(lib):
+    f = lib.q4k_ffn_block
+    f.argtypes = [P, P, P, ctypes.c_int, P, P, P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, P,
+                  ctypes.c_size_t, P]
+    assert f(A16, None, A16, 0, A16, None, A16, 256, 512, 1, A16, 1 << 20, None) == DQ_ERR_NULL
+    assert f(A16, A16, A16, 3, A16, None, A16, 256, 512, 1, A16, 1 << 20, None) == DQ_ERR_LAYOUT
+    assert f(A16, A16, A16, 0, A16, None, A16, 256, 500, 1, A16, 1 << 20, None) == DQ_ERR_SHAPE
+    assert f(A16, A16, A16, 0, A16, None, A16, 256, 512, 9, A16, 1 << 20, None) == DQ_ERR_SHAPE
+    assert f(A16, A16, A8, 0, A16, None, A16, 256, 512, 1, A16, 1 << 20, None) == DQ_ERR_ALIGN
+    assert f(A16, A16, A16, 0, A16, P((1 << 20) + 2), A16, 256, 512, 1, A16, 1 << 20, None) == DQ_ERR_ALIGN
+    bad = ctypes.c_size_t(-1).value
+    assert lib.dq_workspace_bytes(4, 256, 512, 1, 1) == bad        # no argmax

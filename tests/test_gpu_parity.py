@@ -631,3 +631,36 @@ def test_q4k_gemv_residual_is_the_gemv_plus_the_residual(N, K, B, inplace):
     assert np.all(np.abs(got - want) <= tol)
     # and exactly the fp32 sum of q4k_gemv's own output and the residual
     assert np.array_equal(got.astype(np.float32), (plain + r).astype(np.float32))
+
+
+@pytest.mark.parametrize("H,F,B,mode", [
+    (4096, 12288, 1, "residual_x"),   # the decode shape, y = x + FFN(x)
+    (4096, 12288, 1, "inplace"),      # x = x + FFN(x) in place
+    (1024, 4096, 3, "none"),          # batch 3, no residual
+    (512, 1536, 2, "residual_x"),
+])
+def test_q4k_ffn_block_matches_the_separate_calls_and_the_oracle(H, F, B, mode):
+    rng = np.random.default_rng(H + F + B)
+    wg, wu = synth.q4k_matrix(rng, F, H), synth.q4k_matrix(rng, F, H)
+    wd = synth.q4k_matrix(rng, H, F)
+    x = synth.activations(rng, B, H)
+    dwg, dwu, dwd, dx = dev(wg), dev(wu), dev(wd), dev(x)
+    # the separate calls
+    h = dq.q4k_swiglu_gemv(dwg, dwu, dx, F, H)
+    sep = host(dq.q4k_gemv_residual(dwd, h, dx, H, F) if mode != "none" else dq.q4k_gemv(dwd, h, H, F))
+    hv = host(h).reshape(B, F)
+    if mode == "inplace":
+        xin = dev(x)
+        y = dq.q4k_ffn_block(dwg, dwu, dwd, xin, H, F, residual=xin, y=xin)
+    else:
+        y = dq.q4k_ffn_block(dwg, dwu, dwd, dx, H, F, residual=dx if mode == "residual_x" else None)
+    got = host(y).reshape(B, H)
+    assert np.array_equal(got.view(np.uint32), sep.reshape(B, H).view(np.uint32))
+    # the oracle: SwiGLU within its bound, then the down projection of the GPU's own h
+    g_ref, a_g = oracle_rows(lambda rows: oracle.q4k_gemv(wg, F, H, x, rows=rows), F, np.arange(F))
+    u_ref, a_u = oracle_rows(lambda rows: oracle.q4k_gemv(wu, F, H, x, rows=rows), F, np.arange(F))
+    assert np.all(np.abs(hv - oracle.swiglu(g_ref, u_ref)) <= oracle.swiglu_tolerance(g_ref, u_ref, a_g, a_u))
+    y_ref, a_ref = oracle_rows(lambda rows: oracle.q4k_gemv(wd, H, F, hv, rows=rows), H, np.arange(H))
+    want = y_ref + (x.astype(np.float64) if mode != "none" else 0.0)
+    tol = oracle.gemv_tolerance(a_ref) + np.abs(want) * 2.0 ** -23
+    assert np.all(np.abs(got - want) <= tol)
