@@ -345,12 +345,12 @@ def graph_table(only=""):
         qkv_table(timed, l2)
     if want("decode_step:qproj_split+swiglu+down"):
         decode_step_table(timed)
-    if want("ffn_block_4096x12288"):
-        ffn_table(timed)
+    if want("ffn_block_4096x12288:one_call") or want("ffn_block_4096x12288:separate"):
+        ffn_table(timed, want)
     prefill_table(timed, l2, want)
 
 
-def ffn_table(timed):
+def ffn_table(timed, want):
     """A decoder layer's FFN block, x = x + W_down(silu(W_gate x) * (W_up x)) with H =
     4096 and F = 12288: the one-call entry point and the two separate calls."""
     import torch
@@ -366,15 +366,17 @@ def ffn_table(timed):
     hid = torch.empty((1, F), device="cuda")
     scratch = torch.empty(1 << 26, dtype=torch.uint8, device="cuda")
     nbytes = sum(m.numel() for m in mats[0]) + 4 * (2 * H + F)
-    timed("ffn_block_4096x12288:one_call",
-          lambda i: dq.q4k_ffn_block(mats[i][0], mats[i][1], mats[i][2], x, H, F, residual=x, y=y,
-                                     workspace=scratch), nbytes, 2)
+    if want("ffn_block_4096x12288:one_call"):
+        timed("ffn_block_4096x12288:one_call",
+              lambda i: dq.q4k_ffn_block(mats[i][0], mats[i][1], mats[i][2], x, H, F, residual=x, y=y,
+                                         workspace=scratch), nbytes, 2)
 
     def separate(i):
         dq.q4k_swiglu_gemv(mats[i][0], mats[i][1], x, F, H, out=hid, workspace=scratch)
         dq.q4k_gemv_residual(mats[i][2], hid, x, H, F, y=y, workspace=scratch)
 
-    timed("ffn_block_4096x12288:separate", separate, nbytes, 2)
+    if want("ffn_block_4096x12288:separate"):
+        timed("ffn_block_4096x12288:separate", separate, nbytes, 2)
     del mats
     torch.cuda.empty_cache()
 
