@@ -278,13 +278,6 @@ __device__ __forceinline__ void pf_dequant8(uint2 qv, const ChunkScales &cs, uin
     hi = make_uint4(phi[0], phi[1], phi[2], phi[3]);
 }
 
-__device__ __forceinline__ uint2 lds64(uint32_t addr)
-{
-    uint2 v;
-    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
-    return v;
-}
-
 __device__ __forceinline__ void sts128(uint32_t addr, uint4 v)
 {
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
