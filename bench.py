@@ -582,24 +582,36 @@ def main():
 
     # ---- end to end: host x in, host logits + argmax out ----
     # Every step copies its x host->device (pinned), runs the same C-ABI call
-    # and copies its logits (+ argmax) device->host (pinned).  The copy-back of
-    # step i runs on a second stream while step i+1 computes, into one of two
-    # output buffers; the timed region ends when the last copy-back is done.
+    # and copies its logits (+ argmax) device->host (pinned).  Both copies run
+    # on their own streams, into one of two buffers each: the copy-in of step
+    # i+1 overlaps step i, the copy-back of step i overlaps step i+1, and the
+    # timed region ends when the last copy-back is done.
     x_host = torch.from_numpy(inp["x"]).pin_memory()
     y_host = [torch.empty((B, wl.N), dtype=torch.float32).pin_memory() for _ in range(2)]
     i_host = [torch.empty(1, dtype=torch.int64).pin_memory() for _ in range(2)]
-    x_dev = torch.empty_like(x)
+    x_dev = [torch.empty_like(x), torch.empty_like(x)]
     y_dev = [y, torch.empty_like(y)]
     copy_stream = torch.cuda.Stream(dev)
-    done = [torch.cuda.Event(), torch.cuda.Event()]    # step using buffer j has computed
-    freed = [torch.cuda.Event(), torch.cuda.Event()]   # buffer j has been copied back
+    h2d_stream = torch.cuda.Stream(dev)
+    done = [torch.cuda.Event(), torch.cuda.Event()]     # step using buffer j has computed
+    freed = [torch.cuda.Event(), torch.cuda.Event()]    # output buffer j has been copied back
+    x_ready = [torch.cuda.Event(), torch.cuda.Event()]  # input buffer j holds its step's x
 
-    def e2e_step(i):
+    def e2e_copy_in(i):
+        j = i & 1
+        h2d_stream.wait_event(done[j])   # the step that last read buffer j has finished
+        with torch.cuda.stream(h2d_stream):
+            x_dev[j].copy_(x_host, non_blocking=True)
+        x_ready[j].record(h2d_stream)
+
+    def e2e_step(i, last):
         j = i & 1
         stream.wait_event(freed[j])
-        x_dev.copy_(x_host, non_blocking=True)
-        idx = step(x_dev, y_dev[j])
+        stream.wait_event(x_ready[j])
+        idx = step(x_dev[j], y_dev[j])
         done[j].record(stream)
+        if i + 1 < last:
+            e2e_copy_in(i + 1)
         copy_stream.wait_event(done[j])
         with torch.cuda.stream(copy_stream):
             y_host[j].copy_(y_dev[j], non_blocking=True)
@@ -610,14 +622,18 @@ def main():
 
     for j in range(2):
         freed[j].record(copy_stream)
+        done[j].record(stream)
+    e2e_copy_in(0)
     for i in range(3):
-        e2e_step(i)
+        e2e_step(i, 3)
     torch.cuda.synchronize(dev)
     barrier()
     h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     h0.record(stream)
+    h2d_stream.wait_stream(stream)   # the first copy-in starts inside the timed region
+    e2e_copy_in(0)
     for i in range(args.steps):
-        e2e_step(i)
+        e2e_step(i, args.steps)
     for j in range(2):
         stream.wait_event(freed[j])
     h1.record(stream)
@@ -652,8 +668,9 @@ def main():
                      else "fallback"},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms,
-                "note": "weights resident; per step x in (pinned H2D) and logits+argmax out (pinned D2H, "
-                        "overlapping the next step on a copy stream, double-buffered)"},
+                "note": "weights resident; per step x in (pinned H2D on its own stream, overlapping the "
+                        "previous step) and logits+argmax out (pinned D2H on a copy stream, overlapping the next "
+                        "step); both double-buffered"},
         "gpu_launches": launches_per_step * args.steps,
         "gpu_launches_note": "device-timed loop; the roofline loop adds 3 x steps GEMV launches and the e2e loop "
                              "launches_per_step x steps more",
