@@ -11,11 +11,16 @@ combine in fp64, reduction, logits + argmax.  The matrix is larger than the
 Metric: effective HBM GB/s = (weight bytes + activation bytes) / time.
   value  - device time of K steps (CUDA events, inputs resident in HBM), max over ranks
   e2e    - the same metric through the same C-ABI call, with each step's x copied
-           host->device from pinned memory and its logits + argmax copied back
-           (weights stay resident, as a decode loop keeps them)
+           host->device from pinned memory and its logits + argmax copied back, both
+           copies on their own streams into double buffers so that they overlap the
+           neighbouring steps (weights stay resident, as a decode loop keeps them)
   roofline - dominant kernel (q4k_gemv_fx_kernel) timed alone with CUDA events on its
            stream, against the measured HBM copy bandwidth in MEASURED_PEAKS.json
   cpu_baseline - the CPU oracle timed on this host (rank 0, N = 1)
+
+--table prints per-workload device times under CUDA-graph replay instead: the
+decode shapes, grouped QKV, a decode step, the FFN block and the W4A16 prefill
+(--only selects cases by name).
 
 --impl reference times the CPU oracle itself (there is no other implementation
 of this path to install): each step is a bounded row sample of the workload.
