@@ -16,7 +16,12 @@ Metric: effective HBM GB/s = (weight bytes + activation bytes) / time.
            neighbouring steps (weights stay resident, as a decode loop keeps them)
   roofline - dominant kernel (q4k_gemv_fx_kernel) timed alone with CUDA events on its
            stream, against the measured HBM copy bandwidth in MEASURED_PEAKS.json
-  cpu_baseline - the CPU oracle timed on this host (rank 0, N = 1)
+           (and, as frac_of_nominal_8tbs, against the nominal 8 TB/s)
+  secondary - the same roofline record for the down projection at batch 1
+           (4096 x 12288) and the fused SwiGLU (2 x 12288 x 4096), timed under
+           CUDA-graph replay over weight copies that exceed L2 (N = 1 only)
+  cpu_baseline / cpu_baseline_all_cores - the CPU oracle timed on this host (rank 0,
+           N = 1): one thread, and one thread per core over disjoint rows
 
 --table prints per-workload device times under CUDA-graph replay instead: the
 decode shapes, grouped QKV, a decode step, the FFN block and the W4A16 prefill
@@ -52,10 +57,12 @@ UNIT = "GB/s"
 WORKLOAD = "q4k_lmhead_248320x4096"
 FALLBACK_HBM_GBS = 6650.0
 
-# DRAM bytes (read + write) per launch of q4k_gemv_fx_kernel on this workload,
-# from one ncu capture, valid only for the kernel sources whose hash is recorded.
+NOMINAL_HBM_GBS = 8000.0   # B200 HBM3e, nominal
+
+# DRAM bytes (read + write) per launch of q4k_gemv_fx_kernel, from one ncu
+# capture per workload, valid only for the kernel sources whose hash is recorded.
 NCU_TRAFFIC = {"sources_sha1": "97e73226d35cc0a24934390a6c594a86437ad853",
-               "bytes_per_launch": 572207616 + 4335872}   # profiles/q4k_gemv_fx_kernel_248320x4096_dram.md
+               "bytes_per_launch": {"q4k_lmhead_248320x4096": 572207616 + 4335872}}
 
 
 def kernel_sources_sha1() -> str:
@@ -76,6 +83,8 @@ def parse():
     ap.add_argument("--rows", type=int, default=0,
                     help="override N (a smaller case of the same kernel, e.g. for ncu captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the roofline records of the down projection and the SwiGLU")
     ap.add_argument("--table", action="store_true",
                     help="print one JSON line per workload: device time per call under CUDA-graph replay "
                          "(weights rotated through enough copies to exceed L2), then exit")
@@ -192,6 +201,60 @@ class ClockSampler:
                 "reasons": names, "samples": len(self.samples)}
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline_all_cores(wl, inp, budget_s):
+    """Time the CPU oracle (as it stands) over rows split across every host core:
+    one thread per core, each running the oracle on its own consecutive rows (the
+    oracle's C loop releases the interpreter, so the threads run in parallel)."""
+    import concurrent.futures
+    import oracle
+    from dequant_gemv_q4_b200 import synth
+    cores = host_cores()
+    weights_per_row = wl.K * (2 if wl.op == "swiglu" else 1)
+    rows = int(max(64 * cores, min(wl.N, budget_s * cores * 9.0e7 / weights_per_row)))
+    parts = [p for p in np.array_split(np.arange(rows, dtype=np.int64), cores) if p.size]
+
+    def run(sel):
+        if wl.op == "swiglu":
+            g, _ = oracle.q4k_gemv(inp["w_gate"], wl.N, wl.K, inp["x"], rows=sel)
+            u, _ = oracle.q4k_gemv(inp["w_up"], wl.N, wl.K, inp["x"], rows=sel)
+            return oracle.swiglu(g, u)
+        if wl.fmt == "q4k":
+            return oracle.q4k_gemv(inp["w"], wl.N, wl.K, inp["x"], rows=sel)[0]
+        return oracle.q8_0_gemv(inp["w"], wl.N, wl.K, inp["x"], rows=sel)[0]
+
+    t = time.perf_counter()
+    with concurrent.futures.ThreadPoolExecutor(cores) as ex:
+        ys = list(ex.map(run, parts))
+    if wl.op == "gemv_argmax":
+        oracle.argmax(np.concatenate([y[0] for y in ys]))
+    dt = time.perf_counter() - t
+    per_block = synth.Q4K_BLOCK_BYTES if wl.fmt == "q4k" else synth.Q8_0_BLOCK_BYTES
+    elems = synth.Q4K_BLOCK_ELEMS if wl.fmt == "q4k" else synth.Q8_0_BLOCK_ELEMS
+    nbytes = (2 if wl.op == "swiglu" else 1) * rows * (wl.K // elems) * per_block + 4 * wl.K
+    return {"value": nbytes / dt / 1e9, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "cpu_model": cpu_model(), "nproc": os.cpu_count(),
+            "sample": "%d of %d rows (%.3g weights), %d threads (one per core), %.1f s" % (
+                rows, wl.N, rows * weights_per_row, cores, dt)}
+
+
 def cpu_baseline(wl, inp, budget_s):
     """Time the CPU oracle (single thread, as it stands) on a bounded row sample."""
     import oracle
@@ -216,6 +279,7 @@ def cpu_baseline(wl, inp, budget_s):
     elems = synth.Q4K_BLOCK_ELEMS if wl.fmt == "q4k" else synth.Q8_0_BLOCK_ELEMS
     nbytes = (2 if wl.op == "swiglu" else 1) * rows * (wl.K // elems) * per_block + 4 * wl.K
     return {"value": nbytes / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "cpu_model": cpu_model(), "nproc": os.cpu_count(),
             "sample": "%d of %d rows (%.3g weights), single thread, %.1f s" % (rows, wl.N, rows * weights_per_row, dt)}
 
 
@@ -269,6 +333,35 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def graph_us_per_call(fn, copies, reps=20):
+    """Device time per call of fn(0) .. fn(copies - 1), captured once in a CUDA graph
+    and replayed `reps` times back to back (3 untimed replays first); CUDA events on
+    the replay stream."""
+    import torch
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        for i in range(copies):
+            fn(i)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for i in range(copies):
+            fn(i)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        e0.record(s)
+        for _ in range(reps):
+            g.replay()
+        e1.record(s)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / (reps * copies)
+    del g
+    return us
+
+
 def graph_table(only=""):
     """Per-workload device time per call, each call captured in a CUDA graph and
     replayed back to back; every workload's weights rotate through enough copies
@@ -282,31 +375,12 @@ def graph_table(only=""):
     l2 = 126e6
 
     def timed(name, fn, nbytes, copies, reps=20, flops=0):
-        s = torch.cuda.Stream()
-        with torch.cuda.stream(s):
-            for i in range(copies):
-                fn(i)
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=s):
-            for i in range(copies):
-                fn(i)
-        for _ in range(3):
-            g.replay()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(reps):
-            g.replay()
-        e1.record()
-        torch.cuda.synchronize()
-        us = e0.elapsed_time(e1) * 1e3 / (reps * copies)
+        us = graph_us_per_call(fn, copies, reps)
         rec = {"case": name, "us_per_call": round(us, 2), "GBps": round(nbytes / us / 1e3, 1), "bytes": nbytes,
                "copies": copies}
         if flops:
             rec["TFLOPs"] = round(flops / us / 1e6, 1)
         print(json.dumps(rec), flush=True)
-        del g
 
     cases = [("q4k_lmhead_248320x4096", 1, "gemv"), ("q4k_lmhead_248320x4096", 1, "argmax"),
              ("q4k_down_4096x12288", 1, "gemv"), ("q4k_down_4096x12288", 2, "gemv"),
@@ -477,6 +551,52 @@ def prefill_table(timed, l2, want):
                   wbytes + 2 * M * K, copies, flops=2 * M * N * K)
         del pw
         torch.cuda.empty_cache()
+
+
+def secondary_rooflines(peak, peak_kind, reps=50):
+    """Roofline records of the other HBM-bound decode shapes, on the same device:
+    the down projection at batch 1 (4096 x 12288, gated like the LM head) and the
+    fused SwiGLU (2 x 12288 x 4096).  Each launch's weights rotate through enough
+    copies to exceed L2 (> 1.3 x 126 MB), the calls are replayed from a CUDA graph,
+    and achieved = algorithmic bytes per call / device time per call."""
+    import torch
+    import dequant_gemv_q4_b200 as dq
+    from dequant_gemv_q4_b200 import synth
+    out = []
+    for wname in ("q4k_down_4096x12288", "q4k_swiglu_12288x4096"):
+        wl = synth.WORKLOADS[wname]
+        inp = synth.make_inputs(wl, B=1)
+        keys = ["w_gate", "w_up"] if wl.op == "swiglu" else ["w"]
+        wbytes = sum(inp[k].nbytes for k in keys)
+        copies = max(1, int(np.ceil(1.3 * 126e6 / wbytes)))
+        ws = [[torch.from_numpy(inp[k]).cuda() for k in keys]]
+        for _ in range(1, copies):
+            ws.append([t.clone() for t in ws[0]])
+        x = torch.from_numpy(inp["x"]).cuda()
+        y = torch.empty((1, wl.N), device="cuda")
+        scratch = torch.empty(1 << 24, dtype=torch.uint8, device="cuda")
+        if wl.op == "swiglu":
+            fn = lambda i: dq.q4k_swiglu_gemv(ws[i][0], ws[i][1], x, wl.N, wl.K, out=y, workspace=scratch)
+            split = dq.dq_workspace_bytes(dq.DQ_OP_Q4K_SWIGLU, wl.N, wl.K, 1) > 0
+        else:
+            fn = lambda i: dq.q4k_gemv(ws[i][0], x, wl.N, wl.K, y=y, workspace=scratch)
+            split = dq.dq_workspace_bytes(dq.DQ_OP_Q4K_GEMV, wl.N, wl.K, 1) > 0
+        us = graph_us_per_call(fn, copies, reps)
+        nbytes = algorithmic_bytes(wl, 1)
+        achieved = nbytes / (us * 1e-6) / 1e9
+        traffic = NCU_TRAFFIC["bytes_per_launch"].get(wname) \
+            if NCU_TRAFFIC["sources_sha1"] == kernel_sources_sha1() else None
+        out.append({"workload": wname, "B": 1, "us_per_call": us,
+                    "launches_per_call": 2 if split else 1,
+                    "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": UNIT,
+                                 "frac": achieved / peak, "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
+                                 "traffic": traffic, "kernel": "q4k_gemv_fx_kernel",
+                                 "peak_kind": peak_kind,
+                                 "timing": "CUDA-graph replay of %d calls over %d weight copies, %d replays" % (
+                                     copies, copies, reps)}})
+        del ws
+        torch.cuda.empty_cache()
+    return out
 
 
 def main():
@@ -652,8 +772,15 @@ def main():
     peak, peak_kind = measured_peak()
     achieved = nbytes / (kms * 1e-3) / 1e9
     traffic = None
-    if NCU_TRAFFIC["sources_sha1"] == kernel_sources_sha1() and wl.name == WORKLOAD:
-        traffic = NCU_TRAFFIC["bytes_per_launch"]
+    if NCU_TRAFFIC["sources_sha1"] == kernel_sources_sha1():
+        traffic = NCU_TRAFFIC["bytes_per_launch"].get(wl.name)
+    peak_label = peak_kind + " (MEASURED_PEAKS.json hbm_gbs, burst)" if peak_kind == "measured" else "fallback"
+    secondary = []
+    if not args.no_secondary and world == 1 and wl.name == WORKLOAD:
+        with ClockSampler(local_rank) as sec_clocks:
+            secondary = secondary_rooflines(peak, peak_label)
+        for rec in secondary:
+            rec["clocks"] = sec_clocks.summary()
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -667,10 +794,12 @@ def main():
                    else "weights fit in L2: NOT flushed (value is L2-assisted)",
                    "parallelism": "replicas x%d (independent problems, no collective)" % world},
         "pct_of_peak_hbm": 100.0 * value / world / peak,
+        "pct_of_nominal_8tbs": 100.0 * value / world / NOMINAL_HBM_GBS,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
+                     "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
                      "traffic": traffic, "kernel": "q4k_gemv_fx_kernel", "kernel_ms": kms,
-                     "peak_kind": peak_kind + " (MEASURED_PEAKS.json hbm_gbs, burst)" if peak_kind == "measured"
-                     else "fallback"},
+                     "peak_kind": peak_label},
+        "secondary": secondary,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms,
                 "note": "weights resident; per step x in (pinned H2D on its own stream, overlapping the "
@@ -683,6 +812,7 @@ def main():
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, inp, args.cpu_seconds)
+        line["cpu_baseline_all_cores"] = cpu_baseline_all_cores(wl, inp, args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist_on:

@@ -35,7 +35,7 @@ Q8_0_BLOCK_ELEMS, Q8_0_BLOCK_BYTES = 32, 34
 EXPORTED = ("q8_0_gemv", "q4k_gemv", "q4k_swiglu_gemv", "q4k_repack_soa", "dq_workspace_bytes",
             "q8_0_dequant", "q4k_dequant", "dq_status_string", "dq_last_cuda_error",
             "dq_device_error", "q4k_gemv_noalloc", "dq_noalloc_scratch_bytes", "q4k_gemv_split_qg",
-            "q4k_gemv_group", "q4k_prefill_gemm", "q4k_gemv_residual", "q4k_ffn_block")
+            "q4k_gemv_group", "q4k_prefill_gemm", "q4k_gemv_residual", "q4k_ffn_block", "dq_test_lost_copy")
 
 
 class DQError(RuntimeError):
@@ -80,6 +80,7 @@ def load_library(path: str = LIB_PATH):
             "q4k_prefill_gemm": [p, i32, p, p, i64, i64, i64, p, sz, p],
             "q4k_gemv_residual": [p, i32, p, p, p, i64, i64, i32, p, p, sz, p],
             "q4k_ffn_block": [p, p, p, i32, p, p, p, i64, i64, i32, p, sz, p],
+            "dq_test_lost_copy": [p, p, p, i64, i64, ctypes.c_uint64, p, sz, p],
         }
         for name, args in sigs.items():
             f = getattr(lib, name)

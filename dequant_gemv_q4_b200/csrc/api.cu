@@ -68,8 +68,10 @@ Q4KWorkspace q4k_ws(const dq::Q4KPlan &pl, long long N, int B, int NS, bool argm
 {
     Q4KWorkspace ws{};
     const bool reduce_kernel = pl.splits > 1 && !pl.cluster;
+    // batch 1 adds two planes of per-row bounds (error, sum of |y|) to the sums
+    const size_t planes = (B == 1) ? 3 : 1;
     if (reduce_kernel)
-        ws.part_bytes = round_up(static_cast<size_t>(pl.splits) * NS * B * N * sizeof(float), 256);
+        ws.part_bytes = round_up(planes * pl.splits * NS * B * N * sizeof(float), 256);
     if (argmax) {
         ws.ncand = reduce_kernel ? dq::reduce_grid(N, B) : pl.grid;
         ws.cand_bytes = round_up(static_cast<size_t>(ws.ncand) * sizeof(dq::ArgmaxCand), 256);
@@ -133,7 +135,8 @@ size_t prefill_ws_bytes(const dq::PrefillPlan &pl, int64_t N, int64_t M)
 dq_status q4k_common(const void *w0, const void *w1, int layout, const float *x, float *y, int64_t N, int64_t K,
                      int B, int NS, int64_t *argmax_out, void *workspace, size_t ws_bytes, void *stream,
                      float *g_out = nullptr, int64_t qg_hd = 0, const dq::GroupOut *grp = nullptr,
-                     const void *const *gw = nullptr, const float *res = nullptr)
+                     const void *const *gw = nullptr, const float *res = nullptr,
+                     unsigned long long wait_ns = dq::kWaitNanos, int lost_copy = 0)
 {
     if (!w0 || (NS == 2 && !w1) || !x || !y)
         return DQ_ERR_NULL;
@@ -189,14 +192,24 @@ dq_status q4k_common(const void *w0, const void *w1, int layout, const float *x,
     p.argmax = argmax_out != nullptr;
     p.tiles = pl.tiles;
     p.cluster = pl.cluster ? 1 : 0;
+    p.wait_ns = wait_ns;
+    p.lost_copy = lost_copy;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = dq::q4k_gemv_launch(p, pl, B, NS, s);
     if (e != cudaSuccess)
         return cuda_fail(e);
     if (pl.splits > 1 && !pl.cluster) {
-        e = dq::splitk_reduce_launch(p.part, pl.splits, NS, B, N, y, p.g, p.qg_hd, p.grp, p.res, p.cand,
-                                     dq::reduce_grid(N, B),
-                                     s);
+        dq::ExactArgs ex{};
+        ex.w[0] = p.w[0];
+        ex.w[1] = p.w[1];
+        for (int m = 0; m < dq::kMaxGroup; ++m)
+            ex.gw[m] = p.gw[m];
+        ex.x = x;
+        ex.nb = p.nb;
+        ex.soa = p.soa;
+        ex.bounds = B == 1;
+        e = dq::splitk_reduce_launch(p.part, pl.splits, NS, B, N, y, p.g, p.qg_hd, p.grp, p.res, p.cand, ex,
+                                     dq::reduce_grid(N, B), s);
         if (e != cudaSuccess)
             return cuda_fail(e);
     }
@@ -222,21 +235,25 @@ namespace {
 
 std::mutex g_noalloc_mutex;
 void *g_noalloc_ptr[64] = {};
+CUcontext g_noalloc_ctx[64] = {};
 
 // Device address of g_noalloc_scratch on the current device.  The symbol's
-// host-side name is only a stand-in, so the address is looked up once per
-// device (with that device current) and cached.
+// host-side name is only a stand-in, so the address is looked up with the
+// device current, once per device and context (a device reset makes a new
+// context, and the next call looks the address up again), and cached.
 dq_status noalloc_scratch(int device, void **ptr)
 {
     if (device < 0 || device >= 64)
         return DQ_ERR_ARG;
+    const CUcontext cur = dq::current_context();
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_ptr[device]) {
+    if (!g_noalloc_ptr[device] || g_noalloc_ctx[device] != cur) {
         void *p = nullptr;
         cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess)
             return cuda_fail(e);
         g_noalloc_ptr[device] = p;
+        g_noalloc_ctx[device] = cur;
     }
     *ptr = g_noalloc_ptr[device];
     return DQ_OK;
@@ -261,6 +278,15 @@ dq_status q4k_gemv_noalloc(const void *w, int layout, const float *x, float *y, 
 }
 
 size_t dq_noalloc_scratch_bytes(void) { return DQ_NOALLOC_SCRATCH_BYTES; }
+
+dq_status dq_test_lost_copy(const void *w, const float *x, float *y, int64_t N, int64_t K, uint64_t wait_ns,
+                            void *workspace, size_t ws_bytes, void *stream)
+{
+    if (wait_ns < 1000 || wait_ns > dq::kWaitNanos)
+        return DQ_ERR_ARG;
+    return q4k_common(w, nullptr, DQ_LAYOUT_AOS, x, y, N, K, 1, 1, nullptr, workspace, ws_bytes, stream, nullptr, 0,
+                      nullptr, nullptr, nullptr, static_cast<unsigned long long>(wait_ns), 1);
+}
 
 
 dq_status q4k_gemv(const void *w, int layout, const float *x, float *y, int64_t N, int64_t K, int B,

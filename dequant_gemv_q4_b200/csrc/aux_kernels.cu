@@ -3,27 +3,55 @@
 // finalisation, plus the per-device error flag.
 #include <cuda_fp16.h>
 #include <cstdint>
+#include <mutex>
 
 #include "dq_common.cuh"
 #include "dq_internal.h"
 #include "q4k_decode.cuh"
 #include "q8_decode.cuh"
+#include "q4k_exact.cuh"
 
 namespace dq {
 
 // Set by kernels whose bounded waits gave up (see dq_device_error in dqgemv.h).
 __device__ int g_dq_error_flag;
 
+CUcontext current_context()
+{
+    static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+        else
+            cudaGetLastError();
+    });
+    CUcontext c = nullptr;
+    if (fn && fn(&c) != CUDA_SUCCESS)
+        c = nullptr;
+    return c;
+}
+
+// Device address of the error flag on `device` (the current device), looked up
+// once per context.
 int *device_error_flag(int device)
 {
+    static std::mutex mu;
+    static CUcontext ctx[64] = {};
     static int *addr[64] = {};
     if (device < 0 || device >= 64)
         return nullptr;
-    if (!addr[device]) {
+    const CUcontext cur = current_context();
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[device] || ctx[device] != cur) {
         void *a = nullptr;
         if (cudaGetSymbolAddress(&a, g_dq_error_flag) != cudaSuccess)
             return nullptr;
         addr[device] = static_cast<int *>(a);
+        ctx[device] = cur;
     }
     return addr[device];
 }
@@ -174,7 +202,8 @@ cudaError_t q4k_repack_soa_launch(const uint8_t *aos, uint8_t *soa, long long N,
 }
 
 // ---------------------------------------------------------------------------
-// Split-K reduction: out = sum over splits in split order; SwiGLU epilogue when
+// Split-K reduction: out = sum over splits in split order (in fp64), with the
+// batch-1 bound check and exact recomputation of a failing row; SwiGLU epilogue when
 // NS == 2; per-CTA argmax candidates when cand != nullptr (B == 1).
 // ---------------------------------------------------------------------------
 constexpr int kReduceThreads = 256;
@@ -191,36 +220,76 @@ __global__ void __launch_bounds__(kReduceThreads) splitk_reduce_kernel(const flo
                                                                        int NS, int B, long long N,
                                                                        float *y, float *__restrict__ g_out,
                                                                        int qg_hd, const GroupOut grp,
-                                                                       const float *res, ArgmaxCand *cand)
+                                                                       const float *res, ArgmaxCand *cand,
+                                                                       const ExactArgs ex)
 {
     pdl_wait();
     pdl_launch_dependents();
     float best_v = -INFINITY;
     long long best_i = 0x7fffffffffffffffLL;
+    const int lane = threadIdx.x & 31;
     const long long total = N * B;
-    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
-         i += static_cast<long long>(gridDim.x) * blockDim.x) {
-        const long long n = i % N;
-        const int b = static_cast<int>(i / N);
-        float g = 0.f, u = 0.f;
-        for (int s = 0; s < splits; ++s) {
-            g += part[((static_cast<long long>(s) * NS + 0) * B + b) * N + n];
-            if (NS == 2)
-                u += part[((static_cast<long long>(s) * NS + 1) * B + b) * N + n];
+    const long long P = static_cast<long long>(splits) * NS * B * N;   // one plane of partials
+    const long long row_bytes = static_cast<long long>(ex.nb) * kQ4KBlockBytes;
+    // whole warps step together (the exact recomputation of a row is warp-wide)
+    for (long long base = blockIdx.x * static_cast<long long>(blockDim.x) + (threadIdx.x & ~31); base < total;
+         base += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long i = base + lane;
+        const bool in = i < total;
+        const long long n = in ? i % N : 0;
+        const int b = in ? static_cast<int>(i / N) : 0;
+        // the fp32 partials are added in fp64 (in split order), so the sum adds
+        // no rounding beyond the partials' own and the final one; batch-1 bounds
+        // are added rounded outwards
+        double gd = 0.0, ud = 0.0;
+        float ge = 0.f, gs = 0.f, ue = 0.f, us = 0.f;
+        if (in) {
+            for (int s = 0; s < splits; ++s) {
+                const long long ig = ((static_cast<long long>(s) * NS + 0) * B + b) * N + n;
+                gd += part[ig];
+                if (ex.bounds) {
+                    ge = __fadd_ru(ge, part[P + ig]);
+                    gs = __fadd_rd(gs, part[2 * P + ig]);
+                }
+                if (NS == 2) {
+                    const long long iu = ig + static_cast<long long>(B) * N;
+                    ud += part[iu];
+                    if (ex.bounds) {
+                        ue = __fadd_ru(ue, part[P + iu]);
+                        us = __fadd_rd(us, part[2 * P + iu]);
+                    }
+                }
+            }
         }
-        const float out = (NS == 2) ? g / (1.0f + expf(-g)) * u : (res ? g + res[i] : g);
+        // padded row n of a grouped GEMV: the matrix holding it, and its row there
+        int m = 0;
+        long long row = n;
+        bool valid = in;
+        float *ym = nullptr;
         if (grp.n > 0) {
-            // padded row n of a grouped GEMV: the matrix holding it, and its row there
-            int m = 0;
 #pragma unroll
             for (int k = 1; k < kMaxGroup; ++k)
                 if (k < grp.n && n >= grp.base[k])
                     m = k;
-            const long long base = m == 0 ? grp.base[0] : m == 1 ? grp.base[1] : m == 2 ? grp.base[2] : grp.base[3];
+            const long long gbase = m == 0 ? grp.base[0] : m == 1 ? grp.base[1] : m == 2 ? grp.base[2] : grp.base[3];
             const long long rows = m == 0 ? grp.N[0] : m == 1 ? grp.N[1] : m == 2 ? grp.N[2] : grp.N[3];
-            float *ym = m == 0 ? grp.y[0] : m == 1 ? grp.y[1] : m == 2 ? grp.y[2] : grp.y[3];
-            if (n - base < rows)
-                ym[n - base] = out;
+            ym = m == 0 ? grp.y[0] : m == 1 ? grp.y[1] : m == 2 ? grp.y[2] : grp.y[3];
+            row = n - gbase;
+            valid = in && row < rows;
+        }
+        if (ex.bounds) {
+            const uint8_t *w0 = grp.n > 0 ? (m == 0 ? ex.gw[0] : m == 1 ? ex.gw[1] : m == 2 ? ex.gw[2] : ex.gw[3])
+                                          : ex.w[0];
+            gd = fx_fix_rows(gd, ge, gs, valid, w0 + row * row_bytes, ex.nb, ex.soa, ex.x);
+            if (NS == 2)
+                ud = fx_fix_rows(ud, ue, us, valid, ex.w[1] + row * row_bytes, ex.nb, ex.soa, ex.x);
+        }
+        if (!valid)
+            continue;
+        const float g = static_cast<float>(gd), u = static_cast<float>(ud);
+        const float out = (NS == 2) ? g / (1.0f + expf(-g)) * u : (res ? g + res[i] : g);
+        if (grp.n > 0) {
+            ym[row] = out;
             continue;
         }
         *gemv_out_addr(y, g_out, qg_hd, N, b, n) = out;
@@ -256,11 +325,11 @@ __global__ void __launch_bounds__(kReduceThreads) splitk_reduce_kernel(const flo
 }
 
 cudaError_t splitk_reduce_launch(const float *part, int splits, int NS, int B, long long N, float *y, float *g,
-                                 int qg_hd, const GroupOut &grp, const float *res, ArgmaxCand *cand, int grid,
-                                 cudaStream_t s)
+                                 int qg_hd, const GroupOut &grp, const float *res, ArgmaxCand *cand,
+                                 const ExactArgs &ex, int grid, cudaStream_t s)
 {
     return launch_pdl(splitk_reduce_kernel, dim3(grid), dim3(kReduceThreads), 0, s, part, splits, NS, B, N, y, g,
-                      qg_hd, grp, res, cand);
+                      qg_hd, grp, res, cand, ex);
 }
 
 // One CTA folds all candidates into the final index.

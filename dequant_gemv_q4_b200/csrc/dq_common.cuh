@@ -112,9 +112,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
-// Bounded wait for phase `parity` of barrier `bar`.  Returns false (after
-// setting the device error flag) if the phase did not complete in time.
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, int *err)
+// Bounded wait for phase `parity` of barrier `bar`: at most limit_ns of the
+// global timer (and kWaitLimit polls).  Returns false (after setting the
+// device error flag, when err is given) if the phase did not complete in time.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, int *err,
+                                                  unsigned long long limit_ns = kWaitNanos)
 {
     if (mbar_try_wait(bar, parity))
         return true;
@@ -122,7 +124,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     for (uint32_t i = 0; i < kWaitLimit; ++i) {
         if (mbar_try_wait(bar, parity))
             return true;
-        if ((i & 63) == 63 && global_ns() - t0 > kWaitNanos)
+        if ((i & 63) == 63 && global_ns() - t0 > limit_ns)
             break;
     }
     if (err)

@@ -48,6 +48,8 @@ struct Q4KParams {
     int cluster;           // fx kernel: split partials are added inside each cluster of `splits` CTAs
     GroupOut grp;          // grouped GEMV (fx kernel, batch 1): N is then the padded total
     const uint8_t *gw[kMaxGroup];   // weights of the grouped matrices
+    unsigned long long wait_ns;     // limit of every bounded wait (kWaitNanos unless a test lowers it)
+    int lost_copy;         // test hook: warp 0 of CTA 0 arms its first slot but issues no copy
 };
 
 struct Q4KPlan {
@@ -88,11 +90,21 @@ struct Q8Plan {
 Q8Plan q8_plan(long long N, int K, int B, int sm_count, int smem_optin);
 cudaError_t q8_0_gemv_launch(const Q8Params &p, const Q8Plan &pl, int B, cudaStream_t s);
 
-// split-K reduction (+ SwiGLU epilogue, + argmax candidates), argmax finalisation
+// split-K reduction (+ SwiGLU epilogue, + argmax candidates), argmax finalisation.
+// Batch-1 partials carry error-bound planes; a row whose bound fails is
+// recomputed exactly from these:
+struct ExactArgs {
+    const uint8_t *w[2];           // the matrix (gate and up for SwiGLU)
+    const uint8_t *gw[kMaxGroup];  // grouped matrices
+    const float *x;
+    int nb;                        // K / 256
+    int soa;
+    int bounds;                    // 1: partials are [sums][bounds][|y| sums] planes (batch 1)
+};
 int reduce_grid(long long N, int B);
 cudaError_t splitk_reduce_launch(const float *part, int splits, int NS, int B, long long N, float *y, float *g,
-                                 int qg_hd, const GroupOut &grp, const float *res, ArgmaxCand *cand, int grid,
-                                 cudaStream_t s);
+                                 int qg_hd, const GroupOut &grp, const float *res, ArgmaxCand *cand,
+                                 const ExactArgs &ex, int grid, cudaStream_t s);
 cudaError_t argmax_finalize_launch(const ArgmaxCand *cand, int ncand, long long *out, cudaStream_t s);
 
 // debug dequant, repack
@@ -123,5 +135,10 @@ cudaError_t q4k_prefill_launch(const uint8_t *w, int soa, const uint16_t *x16, f
 
 // device error flag
 int *device_error_flag(int device);
+
+// The calling thread's current driver context (null if none or unknown): the
+// key under which device addresses of this library's __device__ arrays are
+// cached, so that a new context (after a device reset) looks them up again.
+CUcontext current_context();
 
 }  // namespace dq

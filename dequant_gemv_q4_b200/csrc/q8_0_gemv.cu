@@ -64,12 +64,15 @@ __global__ void __launch_bounds__(kQ8Threads) q8_0_gemv_kernel(const Q8Params p)
 
     for (long long ti = blockIdx.x; ti < ntiles; ti += gridDim.x) {
         const long long row0 = ti * kQ8Rows;
-        float2 acc[kQ8RowsPerWarp][B];
+        // each chunk's products are summed in fp32 (16 per accumulator) and then
+        // added into fp64, so the rounding error stays that of 16 + 7 additions
+        // whatever K is
+        double dacc[kQ8RowsPerWarp][B];
 #pragma unroll
         for (int rr = 0; rr < kQ8RowsPerWarp; ++rr)
 #pragma unroll
             for (int b = 0; b < B; ++b)
-                acc[rr][b] = make_float2(0.f, 0.f);
+                dacc[rr][b] = 0.0;
 
         for (int ch = 0; ch < nchunk; ++ch) {
             const int kb0 = ch * kQ8ChunkBlocks;
@@ -98,6 +101,12 @@ __global__ void __launch_bounds__(kQ8Threads) q8_0_gemv_kernel(const Q8Params p)
             }
             __syncthreads();
 
+            float2 acc[kQ8RowsPerWarp][B];
+#pragma unroll
+            for (int rr = 0; rr < kQ8RowsPerWarp; ++rr)
+#pragma unroll
+                for (int b = 0; b < B; ++b)
+                    acc[rr][b] = make_float2(0.f, 0.f);
             if (lane < nblk) {
                 const int kb = kb0 + lane;
                 uint32_t q[kQ8RowsPerWarp][8];
@@ -138,6 +147,11 @@ __global__ void __launch_bounds__(kQ8Threads) q8_0_gemv_kernel(const Q8Params p)
                     }
                 }
             }
+#pragma unroll
+            for (int rr = 0; rr < kQ8RowsPerWarp; ++rr)
+#pragma unroll
+                for (int b = 0; b < B; ++b)
+                    dacc[rr][b] += static_cast<double>(acc[rr][b].x) + static_cast<double>(acc[rr][b].y);
         }
 
         // reduce the 32 lanes' partial sums of each (row, batch)
@@ -146,7 +160,7 @@ __global__ void __launch_bounds__(kQ8Threads) q8_0_gemv_kernel(const Q8Params p)
         for (int rr = 0; rr < kQ8RowsPerWarp; ++rr)
 #pragma unroll
             for (int b = 0; b < B; ++b)
-                v[rr * B + b] = acc[rr][b].x + acc[rr][b].y;
+                v[rr * B + b] = static_cast<float>(dacc[rr][b]);
 #pragma unroll
         for (int j = MV; j < MP; ++j)
             v[j] = 0.f;

@@ -22,18 +22,23 @@
  *
  * Numerics.  Results satisfy
  *     |y - y_exact| <= 1e-4 * sum_k |W[n][k] * x[k]| + 1e-6
- * (y_exact: the exact sum over the exact dequantized weights) for finite
- * inputs, up to fp32 overflow of the result.
+ * (y_exact: the exact sum over the exact dequantized weights) for every finite
+ * input, up to fp32 overflow of the result.
  *   - Q8_0 and Q4_K with B >= 2: every weight is formed exactly as the fp32
  *     value nearest to its dequantized value (the bits the *_dequant entry
- *     points return) and the products are accumulated in fp32.
+ *     points return) and the products are accumulated in fp32, at most 1024
+ *     products per accumulator (Q4_K: K is split so; Q8_0: each 1024-wide
+ *     chunk of K is summed in fp32 and the chunks in fp64), then in fp64.
  *   - Q4_K with B == 1 (q4k_gemv, q4k_swiglu_gemv, q4k_gemv_split_qg,
- *     q4k_gemv_group): each activation is rounded
- *     to a 30-bit fixed point shared by its super-block of 256 activations;
- *     the dot products over the exact quants, scales and mins are then exact
- *     (integers, fp64), rounded once to fp32.  The error is at most
- *     sum over super-blocks of 2^(e - 30) * sum |W[n][k]| over the block, where
- *     2^e <= (largest |x| of the block) < 2^(e+1).  An infinity or NaN in x
+ *     q4k_gemv_group, q4k_gemv_residual, q4k_ffn_block): each activation is
+ *     rounded to a 30-bit fixed point shared by its super-block of 256
+ *     activations, and the dot products over the exact quants, scales and mins
+ *     are then exact (integers, fp64).  Beside every output the kernel keeps an
+ *     upper bound on the error that rounding caused and a lower bound on
+ *     sum_k |W[n][k] x[k]|; an output whose bound does not prove the inequality
+ *     above (possible only when a super-block mixes activations of very
+ *     different sizes and its large ones meet near-zero weights) is recomputed
+ *     with exact weights in fp64 before it is stored.  An infinity or NaN in x
  *     makes every result that reads it NaN.
  *   - Environment: DQGEMV_NO_TMA=1 makes the batch-1 kernel fill its shared
  *     memory with per-row bulk copies instead of TMA tile copies (bitwise
@@ -266,6 +271,8 @@ dq_status q4k_dequant(const void *w, int layout, float *out, int64_t N, int64_t 
  *   DQ_ERR_WORKSPACE and launches nothing.
  *   The first call on each device looks up the array's device address (with
  *   that device current); make that first call before any stream capture.
+ *   The address is cached per device and driver context: after a device
+ *   reset (a new context) the next call looks it up again.
  *   It never calls cudaMalloc, cudaFree or any allocating routine.
  *   Every call shares the one array and nothing in it needs to start at zero;
  *   calls that may overlap on the GPU (other streams, other host threads)
@@ -276,6 +283,21 @@ dq_status q4k_gemv_noalloc(const void *w, int layout, const float *x, float *y, 
 
 /* Size in bytes of the fixed scratch array q4k_gemv_noalloc uses. */
 size_t dq_noalloc_scratch_bytes(void);
+
+/*
+ * Test of the bounded waits (no counterpart on the pages; this library's
+ * failure detection, see dq_device_error).  A batch-1 q4k_gemv call (AoS
+ * layout, no argmax) in which warp 0 of the first CTA arms the mbarrier of its
+ * first slot but issues no copy into it, so that its wait runs out; every
+ * bounded wait of the launch gives up after wait_ns nanoseconds instead of the
+ * usual 2 s.  The kernel then sets the device error flag, waits (bounded) for
+ * its other copies in flight and returns; the rows of that slot's tile are not
+ * written correctly, the others are.  No fault, trap or hang is involved.
+ *   wait_ns    1,000 .. 2,000,000,000.   Other arguments as for q4k_gemv.
+ * Returns DQ_ERR_ARG for a wait_ns outside that range; otherwise as q4k_gemv.
+ */
+dq_status dq_test_lost_copy(const void *w, const float *x, float *y, int64_t N, int64_t K, uint64_t wait_ns,
+                            void *workspace, size_t ws_bytes, void *stream);
 
 /* Static string naming a status code. */
 const char *dq_status_string(int status);

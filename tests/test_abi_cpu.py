@@ -186,3 +186,11 @@ def test_ffn_block_rejects_on_host(lib):
     assert f(A16, A16, A16, 0, A16, P((1 << 20) + 2), A16, 256, 512, 1, A16, 1 << 20, None) == DQ_ERR_ALIGN
     bad = ctypes.c_size_t(-1).value
     assert lib.dq_workspace_bytes(4, 256, 512, 1, 1) == bad        # no argmax
+
+
+def test_lost_copy_test_entry_rejects_on_host(lib):
+    # wait limits outside 1 us .. 2 s are refused before anything else is looked at
+    assert lib.dq_test_lost_copy(None, None, None, 64, 1024, 10, None, 0, None) == 7
+    assert lib.dq_test_lost_copy(None, None, None, 64, 1024, 3_000_000_000, None, 0, None) == 7
+    # then the q4k_gemv checks: null pointers
+    assert lib.dq_test_lost_copy(None, None, None, 64, 1024, 1_000_000, None, 0, None) == 1

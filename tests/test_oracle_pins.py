@@ -143,6 +143,11 @@ def test_q8_0_handworked_block(spec):
     assert np.array_equal(oracle.q8_0_block(blk), want)
     mat = np.concatenate([blk, blk]).reshape(1, 68)
     assert np.array_equal(oracle.q8_0_dequant(mat, 1, 64)[0], np.concatenate([want, want]))
+    # the fp32 dequant (the bit-exact reference of the GPU's debug dequant): every
+    # hand-worked weight here is exact in fp32, so it must come back unchanged
+    f32 = oracle.q8_0_dequant_f32(mat, 1, 64)[0]
+    assert f32.dtype == np.float32
+    assert np.array_equal(f32, np.concatenate([want, want]).astype(np.float32))
 
 
 def test_nibble_order_rejects_the_low_nibbles_first_reading():
@@ -453,3 +458,21 @@ def test_q4k_prefill_equals_the_gemv_when_weights_and_x_are_binary16_exact():
     y, _ = oracle.q4k_prefill(w, N, K, x16)
     yg, _ = oracle.q4k_gemv(w, N, K, x16.astype(np.float32))
     assert np.array_equal(y, yg)
+
+
+def test_q8_0_fp32_dequant_is_exact_for_every_scale_and_quant():
+    # d has 11 significant bits and q 8, so d*q (<= 19 bits, exponent within
+    # fp32's range) is exact in fp32: the fp32 dequant must equal the exact one
+    # for every fp16 scale pattern (finite) against the extreme quants
+    d_bits = np.arange(0, 0x7C00, dtype=np.uint16)           # every finite non-negative fp16
+    d_bits = np.concatenate([d_bits, d_bits | 0x8000])
+    q = np.array([-128, -127, -1, 0, 1, 127], np.int8)
+    blocks = np.zeros((d_bits.size, 34), np.uint8)
+    blocks[:, 0:2] = d_bits.view(np.uint8).reshape(-1, 2)
+    blocks[:, 2:] = np.resize(q.view(np.uint8), 32)
+    N = d_bits.size
+    exact = oracle.q8_0_dequant(blocks, N, 32)
+    f32 = oracle.q8_0_dequant_f32(blocks, N, 32)
+    assert np.array_equal(f32.astype(np.float64), exact)
+    d = d_bits.view(np.float16).astype(np.float64)
+    assert np.array_equal(exact, d[:, None] * np.resize(q.astype(np.float64), 32)[None, :])
