@@ -35,13 +35,15 @@ __device__ __forceinline__ BlockOffsets row_block_offsets(int kb, int nb, bool s
 }
 
 // sum_k W[k] x[k] over one row (wrow: its nb super-blocks) with exact weights,
-// in fp64.  Called by all 32 lanes of a warp (super-blocks are spread over the
-// lanes); every lane returns the same sum, added in a fixed order.
+// in fp64.  Called by all 32 lanes of a warp: the row's 16-byte quant slices
+// (32 weights each) are spread over the lanes; every lane returns the same sum,
+// added in a fixed order.
 static __device__ __noinline__ double q4k_exact_row(const uint8_t *wrow, int nb, int soa, const float *x)
 {
     const int lane = threadIdx.x & 31;
     double acc = 0.0;
-    for (int kb = lane; kb < nb; kb += 32) {
+    for (int u = lane; u < nb * 8; u += 32) {
+        const int kb = u >> 3, s = u & 7;
         const BlockOffsets bo = row_block_offsets(kb, nb, soa != 0);
         const uint4 h = __ldg(reinterpret_cast<const uint4 *>(wrow + bo.hdr));
         const double d = static_cast<double>(__half2float(__ushort_as_half(static_cast<unsigned short>(h.x & 0xFFFFu))));
@@ -49,25 +51,30 @@ static __device__ __noinline__ double q4k_exact_row(const uint8_t *wrow, int nb,
         // get_scale_min_k4 fields, four per word (one per byte)
         const uint32_t scw[2] = {h.y & 0x3F3F3F3Fu, (h.w & 0x0F0F0F0Fu) | ((h.y >> 2) & 0x30303030u)};
         const uint32_t mnw[2] = {h.z & 0x3F3F3F3Fu, ((h.w >> 4) & 0x0F0F0F0Fu) | ((h.z >> 2) & 0x30303030u)};
-        const float *xb = x + static_cast<long long>(kb) * kQ4KBlockElems;
-        for (int s = 0; s < 8; ++s) {
-            // slice s holds bytes 16(s%2) .. 16(s%2)+15 of chunk c = s/2: low nibbles are
-            // weights 64c + r of sub-block 2c, high nibbles 64c + 32 + r of sub-block 2c+1
-            const uint4 qv = __ldg(reinterpret_cast<const uint4 *>(wrow + bo.qs0 + s * bo.qs_step));
-            const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
-            const int c = s >> 1;
-            const int jl = 2 * c, jh = 2 * c + 1;
-            const double al = d * static_cast<double>((scw[jl >> 2] >> (8 * (jl & 3))) & 0xFFu);
-            const double bl = dm * static_cast<double>((mnw[jl >> 2] >> (8 * (jl & 3))) & 0xFFu);
-            const double ah = d * static_cast<double>((scw[jh >> 2] >> (8 * (jh & 3))) & 0xFFu);
-            const double bh = dm * static_cast<double>((mnw[jh >> 2] >> (8 * (jh & 3))) & 0xFFu);
-            const float *xl = xb + 64 * c + 16 * (s & 1);
-            for (int t = 0; t < 16; ++t) {
-                const uint32_t byte = (qw[t >> 2] >> (8 * (t & 3))) & 0xFFu;
+        // slice s holds bytes 16(s%2) .. 16(s%2)+15 of chunk c = s/2: low nibbles are
+        // weights 64c + r of sub-block 2c, high nibbles 64c + 32 + r of sub-block 2c+1
+        const uint4 qv = __ldg(reinterpret_cast<const uint4 *>(wrow + bo.qs0 + s * bo.qs_step));
+        const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+        const int c = s >> 1;
+        const int jl = 2 * c, jh = 2 * c + 1;
+        const double al = d * static_cast<double>((scw[jl >> 2] >> (8 * (jl & 3))) & 0xFFu);
+        const double bl = dm * static_cast<double>((mnw[jl >> 2] >> (8 * (jl & 3))) & 0xFFu);
+        const double ah = d * static_cast<double>((scw[jh >> 2] >> (8 * (jh & 3))) & 0xFFu);
+        const double bh = dm * static_cast<double>((mnw[jh >> 2] >> (8 * (jh & 3))) & 0xFFu);
+        const float *xl = x + static_cast<long long>(kb) * kQ4KBlockElems + 64 * c + 16 * (s & 1);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            const float4 xa = __ldg(reinterpret_cast<const float4 *>(xl + 4 * v));
+            const float4 xb = __ldg(reinterpret_cast<const float4 *>(xl + 32 + 4 * v));
+            const float xlo[4] = {xa.x, xa.y, xa.z, xa.w};
+            const float xhi[4] = {xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const uint32_t byte = (qw[v] >> (8 * t)) & 0xFFu;
                 const double wl = al * static_cast<double>(byte & 15u) - bl;   // exact
                 const double wh = ah * static_cast<double>(byte >> 4) - bh;     // exact
-                acc = fma(wl, static_cast<double>(__ldg(xl + t)), acc);
-                acc = fma(wh, static_cast<double>(__ldg(xl + 32 + t)), acc);
+                acc = fma(wl, static_cast<double>(xlo[t]), acc);
+                acc = fma(wh, static_cast<double>(xhi[t]), acc);
             }
         }
     }
