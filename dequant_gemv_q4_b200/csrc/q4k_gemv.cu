@@ -109,6 +109,8 @@ constexpr int kFxRowPitch = kFxChunkBytes + 16;           // 592
 constexpr int kFxSlotBytes = kFxTileRows * kFxRowPitch;
 static_assert(kFxSlotBytes % 128 == 0, "slots must keep the ring 128-byte aligned");
 constexpr int kFxMaxWarps = 12;
+// Ring slots a warp fills before it stages its activations (the rest after).
+constexpr int kFxPreIssue = 1;
 int q4k_fx_tile_rows() { return kFxTileRows; }
 // In-cluster split reduction: per warp and stream, the 16 row partials (fp64)
 // and their bounds (two floats).
@@ -579,13 +581,20 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
     pdl_launch_dependents();
     FxXPre pre;
     fx_stage_load(p.x, kb_begin, nbs, warp, nwarps, lane, pre);
-    for (int s = 0; s < p.depth && issued < total; ++s, ++issued) {
+    // only the first slots before staging: the activation loads are not to
+    // wait behind every SM's full ring of weight requests
+    for (int s = 0; s < min(p.depth, kFxPreIssue) && issued < total; ++s, ++issued) {
         const bool lost = p.lost_copy && s == 0 && warp == 0 && blockIdx.x == 0;
         fx_issue_slot<TMA>(p, maps, pc, s, c_begin, my_ring_s, my_bars_s, lane, lost);
         pc.advance(nch, NS, row_step);
     }
 
     fx_stage(p.x, kb_begin, nbs, limbs, aux, warp, nwarps, lane, pre, p.nb >= kFxMin3LimbBlocks);
+    for (int s = static_cast<int>(issued); s < p.depth && issued < total; ++s, ++issued) {
+        const bool lost = p.lost_copy && s == 0 && warp == 0 && blockIdx.x == 0;
+        fx_issue_slot<TMA>(p, maps, pc, s, c_begin, my_ring_s, my_bars_s, lane, lost);
+        pc.advance(nch, NS, row_step);
+    }
     __syncthreads();
 
     float best_v = -INFINITY;
@@ -733,17 +742,35 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
             double g = 0.0, u = 0.0;
             float ge = 0.f, gs = 0.f, ue = 0.f, us = 0.f;
             const int lr = lane & (kFxTileRows - 1);
-            for (int r = 0; r < p.splits; ++r) {
-                const double *rp = cl.map_shared_rank(cpart, r);
-                const float2 *rb = cl.map_shared_rank(cbnd, r);
-                g += rp[(warp * 2 + 0) * kFxTileRows + lr];
-                u += rp[(warp * 2 + 1) * kFxTileRows + lr];
-                const float2 bg = rb[(warp * 2 + 0) * kFxTileRows + lr];
-                const float2 bu = rb[(warp * 2 + 1) * kFxTileRows + lr];
-                ge = __fadd_ru(ge, bg.x);
-                gs = __fadd_rd(gs, bg.y);
-                ue = __fadd_ru(ue, bu.x);
-                us = __fadd_rd(us, bu.y);
+            // all remote loads first (each is a round trip to another SM), then
+            // the sums in rank order
+            double pg[kFxMaxCluster], pu[kFxMaxCluster];
+            float2 bg[kFxMaxCluster], bu[kFxMaxCluster];
+#pragma unroll
+            for (int r = 0; r < kFxMaxCluster; ++r) {
+                if (r < p.splits) {
+                    const double *rp = cl.map_shared_rank(cpart, r);
+                    const float2 *rb = cl.map_shared_rank(cbnd, r);
+                    pg[r] = rp[(warp * 2 + 0) * kFxTileRows + lr];
+                    bg[r] = rb[(warp * 2 + 0) * kFxTileRows + lr];
+                    if (NS == 2) {
+                        pu[r] = rp[(warp * 2 + 1) * kFxTileRows + lr];
+                        bu[r] = rb[(warp * 2 + 1) * kFxTileRows + lr];
+                    }
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < kFxMaxCluster; ++r) {
+                if (r < p.splits) {
+                    g += pg[r];
+                    ge = __fadd_ru(ge, bg[r].x);
+                    gs = __fadd_rd(gs, bg[r].y);
+                    if (NS == 2) {
+                        u += pu[r];
+                        ue = __fadd_ru(ue, bu[r].x);
+                        us = __fadd_rd(us, bu[r].y);
+                    }
+                }
             }
             const long long n = t0 * kFxTileRows + lane;
             const FxRows fr = fx_rows(p, 0, t0 * kFxTileRows);
