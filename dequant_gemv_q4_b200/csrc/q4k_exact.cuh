@@ -64,8 +64,9 @@ static __device__ __noinline__ double q4k_exact_row(const uint8_t *wrow, int nb,
         const float *xl = x + static_cast<long long>(kb) * kQ4KBlockElems + 64 * c + 16 * (s & 1);
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
-            const float4 xa = __ldg(reinterpret_cast<const float4 *>(xl + 4 * v));
-            const float4 xb = __ldg(reinterpret_cast<const float4 *>(xl + 32 + 4 * v));
+            // x through L2 (it may have been written earlier in the same kernel)
+            const float4 xa = __ldcg(reinterpret_cast<const float4 *>(xl + 4 * v));
+            const float4 xb = __ldcg(reinterpret_cast<const float4 *>(xl + 32 + 4 * v));
             const float xlo[4] = {xa.x, xa.y, xa.z, xa.w};
             const float xhi[4] = {xb.x, xb.y, xb.z, xb.w};
 #pragma unroll

@@ -137,10 +137,10 @@ dq_status q4k_gemv_residual(const void *w, int layout, const float *x, const flo
 /*
  * A decoder layer's FFN block in one call (qualiaDB cuda_lane:
  * try_q4k_soa_ffn_block, try_q4k_soa_ffn_block_residual):
- *   h = silu(W_gate x) * (W_up x)        (B x F; q4k_swiglu_gemv)
- *   y = W_down h [+ residual]            (B x H; q4k_gemv / q4k_gemv_residual)
+ *   h = silu(W_gate x) * (W_up x)        (B x F)
+ *   y = W_down h [+ residual]            (B x H)
  * as two launches on `stream`, the second chained to the first by programmatic
- * dependent launch; h lives in the workspace.
+ * dependent launch; h (B x F fp32) is left at the start of the workspace.
  *   w_gate, w_up  F x H Q4_K matrices;  w_down  H x F;  all in `layout`,
  *                 16-byte aligned.
  *   x             B x H fp32, 16-byte aligned.   y  B x H fp32, 4-byte aligned.

@@ -641,6 +641,7 @@ def test_q4k_gemv_residual_is_the_gemv_plus_the_residual(N, K, B, inplace):
     (4096, 12288, 1, "inplace"),      # x = x + FFN(x) in place
     (1024, 4096, 3, "none"),          # batch 3, no residual
     (512, 1536, 2, "residual_x"),
+    (2560, 9728, 1, "residual_x"),    # K not a multiple of the 1024-wide chunk
 ])
 def test_q4k_ffn_block_matches_the_separate_calls_and_the_oracle(H, F, B, mode):
     rng = np.random.default_rng(H + F + B)
@@ -651,13 +652,16 @@ def test_q4k_ffn_block_matches_the_separate_calls_and_the_oracle(H, F, B, mode):
     # the separate calls
     h = dq.q4k_swiglu_gemv(dwg, dwu, dx, F, H)
     sep = host(dq.q4k_gemv_residual(dwd, h, dx, H, F) if mode != "none" else dq.q4k_gemv(dwd, h, H, F))
-    hv = host(h).reshape(B, F)
+    ws = torch.empty(dq.dq_workspace_bytes(dq.DQ_OP_Q4K_FFN, H, F, B), dtype=torch.uint8, device="cuda")
     if mode == "inplace":
         xin = dev(x)
-        y = dq.q4k_ffn_block(dwg, dwu, dwd, xin, H, F, residual=xin, y=xin)
+        y = dq.q4k_ffn_block(dwg, dwu, dwd, xin, H, F, residual=xin, y=xin, workspace=ws)
     else:
-        y = dq.q4k_ffn_block(dwg, dwu, dwd, dx, H, F, residual=dx if mode == "residual_x" else None)
+        y = dq.q4k_ffn_block(dwg, dwu, dwd, dx, H, F, residual=dx if mode == "residual_x" else None, workspace=ws)
     got = host(y).reshape(B, H)
+    # h, the GPU's own SwiGLU output, is left at the start of the workspace
+    hv = host(ws[:4 * B * F].view(torch.float32)).reshape(B, F)
+    # two launches: exactly the separate calls
     assert np.array_equal(got.view(np.uint32), sep.reshape(B, H).view(np.uint32))
     # the oracle: SwiGLU within its bound, then the down projection of the GPU's own h
     g_ref, a_g = oracle_rows(lambda rows: oracle.q4k_gemv(wg, F, H, x, rows=rows), F, np.arange(F))
