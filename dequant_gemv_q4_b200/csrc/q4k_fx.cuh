@@ -362,10 +362,11 @@ __device__ __forceinline__ void fx_slot(const uint8_t *slot, const uint8_t *limb
     const float rres = __uint_as_float(sn.z);
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-        double is = static_cast<double>(isum[r][3]);
-        is = fma(is, 256.0, static_cast<double>(isum[r][2]));
-        is = fma(is, 256.0, static_cast<double>(isum[r][1]));
-        is = fma(is, 256.0, static_cast<double>(isum[r][0]));
+        // I_s = sum_l 2^(8l) I_l: exact in int64 (below 2^53), then one conversion
+        const long long is64 =
+            ((static_cast<long long>(isum[r][3]) << 24) + (static_cast<long long>(isum[r][2]) << 16)) +
+            ((static_cast<long long>(isum[r][1]) << 8) + static_cast<long long>(isum[r][0]));
+        const double is = static_cast<double>(is64);
         const uint32_t mn03 = hd[r].z & 0x3F3F3F3Fu;
         const uint32_t mn47 = ((hd[r].w >> 4) & 0x0F0F0F0Fu) | ((hd[r].z >> 2) & 0x30303030u);
         // I_m as a tree of exact products and sums (integers below 2^53)
@@ -373,7 +374,9 @@ __device__ __forceinline__ void fx_slot(const uint8_t *slot, const uint8_t *limb
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const uint32_t mw = (j < 4) ? mn03 : mn47;
-            pmn[j] = static_cast<double>((mw >> (8 * (j & 3))) & 0xFFu) * X[j];
+            // min_j as a double without a conversion: the bits of 2^52 + m, minus 2^52 (exact)
+            const double mj = __hiloint2double(0x43300000, static_cast<int>((mw >> (8 * (j & 3))) & 0xFFu)) - 0x1p52;
+            pmn[j] = mj * X[j];
         }
         const double im = ((pmn[0] + pmn[1]) + (pmn[2] + pmn[3])) + ((pmn[4] + pmn[5]) + (pmn[6] + pmn[7]));
         const float df = __half2float(__ushort_as_half(static_cast<unsigned short>(hd[r].x & 0xFFFFu)));
