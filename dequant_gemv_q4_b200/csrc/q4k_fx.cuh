@@ -33,6 +33,12 @@
 // pitch, which places the eight rows a quarter-warp reads at one time in eight
 // distinct bank groups); the four quarter sums of a row are added with two
 // shuffles.
+//   Warp pairs (R = 1).  When each warp would own only a few slots, the time a
+// warp takes to work through them one after another, not the memory, bounds a
+// small matrix.  Then two warps own each ring and its row tiles: warp h of the
+// pair takes rows 8h .. 8h + 7 of every slot (lane (g, i): super-block g, row
+// 8h + i), so a slot's arithmetic is done by twice the warps in half the time.
+// The second warp of the pair to finish a slot refills it.
 #pragma once
 
 #include <cuda.h>
@@ -83,10 +89,12 @@ constexpr int kFxRowPitch = kFxChunkBytes + 16;           // 592
 constexpr int kFxSlotBytes = kFxTileRows * kFxRowPitch;
 static_assert(kFxSlotBytes % 128 == 0, "slots must keep the ring 128-byte aligned");
 constexpr int kFxMaxWarps = 12;
+constexpr int kFxMaxPairWarps = 16;            // R = 1: eight pairs of warps
+constexpr int kFxPairMaxSlots = 8;             // R = 1 for rings of at most this many slots
 // Ring slots a warp fills before it stages its activations (the rest after).
 constexpr int kFxPreIssue = 1;
-// In-cluster split reduction: per warp and stream, the 16 row partials (fp64)
-// and their bounds (two floats).
+// In-cluster split reduction: per ring a CTA finishes, stream and source rank,
+// the 16 row partials (fp64) and their bounds (two floats).
 constexpr int kFxClusterPartBytes = 2 * kFxTileRows * (8 + 8);
 constexpr int kFxMaxCluster = 8;
 
@@ -130,100 +138,165 @@ __device__ __forceinline__ void fx_stage_load(const float *x, int kb_begin, int 
     }
 }
 
-// Converts the activations of super-block sb (this lane's eight: a, b) into
-// limb planes and its FxAux record; one warp per super-block.
-__device__ __forceinline__ void fx_stage_one(int sb, float4 a, float4 b, uint8_t *limbs, uint8_t *aux, int lane,
-                                             bool allow3)
+// Converts the activations of NB super-blocks sb[k] (this lane's eight of each:
+// a[k], b[k]) into limb planes and FxAux records; one warp per super-block, NB
+// of them at once so that their dependency chains interleave.  Block k is
+// stored only when valid[k].
+template <int NB>
+__device__ __forceinline__ void fx_stage_blocks(const int (&sb)[NB], const float4 (&a)[NB], const float4 (&b)[NB],
+                                                const bool (&valid)[NB], uint8_t *limbs, uint8_t *aux, int lane,
+                                                bool allow3)
 {
-    {
-        const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-        uint32_t m = 0;
+    float v[NB][8];
+    uint32_t m[NB];
+#pragma unroll
+    for (int k = 0; k < NB; ++k) {
+        v[k][0] = a[k].x; v[k][1] = a[k].y; v[k][2] = a[k].z; v[k][3] = a[k].w;
+        v[k][4] = b[k].x; v[k][5] = b[k].y; v[k][6] = b[k].z; v[k][7] = b[k].w;
+        m[k] = 0;
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-            m = max(m, __float_as_uint(v[i]) & 0x7FFFFFFFu);
-        m = __reduce_max_sync(0xffffffffu, m);   // |x| bit patterns order like the values
-        const bool finite = m < 0x7F800000u;
-        int e = 0;
-        if (m >= 0x00800000u)
-            e = static_cast<int>(m >> 23) - 127;
-        else if (m != 0)
-            e = (31 - __clz(static_cast<int>(m))) - 149;
-        // three limbs when max |x| <= 6 rms (sum of squares in fp64: no overflow)
-        double sq = 0.0;
+            m[k] = max(m[k], __float_as_uint(v[k][i]) & 0x7FFFFFFFu);
+    }
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-            sq = fma(static_cast<double>(v[i]), static_cast<double>(v[i]), sq);
+    for (int k = 0; k < NB; ++k)
+        m[k] = __reduce_max_sync(0xffffffffu, m[k]);   // |x| bit patterns order like the values
+    int e[NB];
+    bool finite[NB];
+    float sq[NB];
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1)
-            sq += __shfl_xor_sync(0xffffffffu, sq, o);
-        const double mx = static_cast<double>(__uint_as_float(m));
-        const bool three = allow3 && finite && mx * mx * 256.0 <= 36.0 * sq;
+    for (int k = 0; k < NB; ++k) {
+        finite[k] = m[k] < 0x7F800000u;
+        e[k] = 0;
+        if (m[k] >= 0x00800000u)
+            e[k] = static_cast<int>(m[k] >> 23) - 127;
+        else if (m[k] != 0)
+            e[k] = (31 - __clz(static_cast<int>(m[k]))) - 149;
+        // the limb-count test on x 2^-e (largest |value| in [1, 2), squares
+        // below 4, no overflow); blocks of extreme exponent take four limbs
+        const float sc = (e[k] >= -100 && e[k] <= 100) ? __int_as_float((127 - e[k]) << 23) : 0.f;
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) {
+            s0 = fmaf(v[k][i] * sc, v[k][i] * sc, s0);
+            s1 = fmaf(v[k][i + 1] * sc, v[k][i + 1] * sc, s1);
+        }
+        sq[k] = s0 + s1;
+    }
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1)
+#pragma unroll
+        for (int k = 0; k < NB; ++k)
+            sq[k] += __shfl_xor_sync(0xffffffffu, sq[k], o);
+
+    uint32_t w[NB][4][2];
+    double part[NB];
+    float res[NB];   // sum of |x_k 2^F - xi_k| over this lane's elements
+    bool three[NB];
+    int F[NB];
+#pragma unroll
+    for (int k = 0; k < NB; ++k) {
+        // three limbs when max |x| <= 6 rms, i.e. 256 max^2 <= 36 sum x^2 (taken
+        // with a 2^-10 margin: the fp32 sum is not exact)
+        const float mxs = (e[k] >= -100 && e[k] <= 100) ? __uint_as_float(m[k]) * __int_as_float((127 - e[k]) << 23)
+                                                         : 0.f;
+        three[k] = allow3 && finite[k] && e[k] >= -100 && e[k] <= 100 &&
+                   256.f * mxs * mxs <= 36.f * sq[k] * (1.f - 0x1p-10f);
         // |x 2^F| < 2^(30 - 8 (4 - limbs)): the top signed digit stays within +-64
-        const int F = (three ? 21 : 29) - e;   // in [-106, 178]
-        const int F1 = F / 2, F2 = F - F1;     // each in [-53, 89]: normal powers of two
+        F[k] = (three[k] ? 21 : 29) - e[k];   // in [-106, 178]
+        const int F1 = F[k] / 2, F2 = F[k] - F1;   // each in [-53, 89]: normal powers of two
         const float p1 = __int_as_float((127 + F1) << 23);
         const float p2 = __int_as_float((127 + F2) << 23);
-
-        uint32_t w[4][2] = {};
-        double part = 0.0;
-        double res = 0.0;   // sum of |x_k 2^F - xi_k| over this lane's elements
+        float d[8];
+        double pi[8];
+#pragma unroll
+        for (int l = 0; l < 4; ++l)
+            w[k][l][0] = w[k][l][1] = 0u;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             // x * 2^F is exact wherever it is >= 1/2 in magnitude (two power-of-two
             // products with normal results), and then so is t - rint(t); below 1/2 it
             // rounds to 0, and the first product may have lost bits below 2^-150,
             // i.e. below 2^-61 after the second: 2^-60 covers that
-            const float t = finite ? (v[i] * p1) * p2 : 0.f;
+            const float t = finite[k] ? (v[k][i] * p1) * p2 : 0.f;
             const float r = rintf(t);
-            res += static_cast<double>(fabsf(t - r)) + ((r == 0.f && v[i] != 0.f) ? 0x1p-60 : 0.0);
+            d[i] = fabsf(t - r) + ((r == 0.f && v[k][i] != 0.f) ? 0x1p-60f : 0.f);
             int ti = static_cast<int>(r);
-            part += static_cast<double>(ti);
+            pi[i] = static_cast<double>(ti);
             // signed digits: the stored byte is ti's low byte, the carry rounds ti / 256
 #pragma unroll
             for (int l = 0; l < 4; ++l) {
-                w[l][i >> 2] |= (static_cast<uint32_t>(ti) & 0xFFu) << (8 * (i & 3));
+                w[k][l][i >> 2] |= (static_cast<uint32_t>(ti) & 0xFFu) << (8 * (i & 3));
                 ti = (ti + 128) >> 8;
             }
         }
-        uint8_t *lp = limbs + sb * kFxLimbPitch + lane * 8;
+        // sums as trees: part exact (integers below 2^33), res rounded (the bound
+        // below allows for it)
+        part[k] = ((pi[0] + pi[1]) + (pi[2] + pi[3])) + ((pi[4] + pi[5]) + (pi[6] + pi[7]));
+        res[k] = ((d[0] + d[1]) + (d[2] + d[3])) + ((d[4] + d[5]) + (d[6] + d[7]));
+        if (valid[k]) {
+            uint8_t *lp = limbs + sb[k] * kFxLimbPitch + lane * 8;
 #pragma unroll
-        for (int l = 0; l < 4; ++l)
-            *reinterpret_cast<uint2 *>(lp + 256 * l) = make_uint2(w[l][0], w[l][1]);
-        // sub-block j = lanes 4j .. 4j+3; sums of at most 32 values below 2^30 are exact
-        // (with three limbs the fourth plane is zero)
-        part += __shfl_xor_sync(0xffffffffu, part, 1);
-        part += __shfl_xor_sync(0xffffffffu, part, 2);
+            for (int l = 0; l < 4; ++l)
+                *reinterpret_cast<uint2 *>(lp + 256 * l) = make_uint2(w[k][l][0], w[k][l][1]);
+        }
+    }
+    // sub-block j = lanes 4j .. 4j+3; sums of at most 32 values below 2^30 are exact
+    // (with three limbs the fourth plane is zero)
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1)
-            res += __shfl_xor_sync(0xffffffffu, res, o);
-        FxAux *ap = reinterpret_cast<FxAux *>(aux + sb * kFxAuxPitch);
+    for (int o = 1; o < 4; o <<= 1)
+#pragma unroll
+        for (int k = 0; k < NB; ++k)
+            part[k] += __shfl_xor_sync(0xffffffffu, part[k], o);
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1)
+#pragma unroll
+        for (int k = 0; k < NB; ++k)
+            res[k] += __shfl_xor_sync(0xffffffffu, res[k], o);
+#pragma unroll
+    for (int k = 0; k < NB; ++k) {
+        if (!valid[k])
+            continue;
+        FxAux *ap = reinterpret_cast<FxAux *>(aux + sb[k] * kFxAuxPitch);
         if ((lane & 3) == 0)
-            ap->X[lane >> 2] = part;
+            ap->X[lane >> 2] = part[k];
         if (lane == 0) {
-            const double s2f = __longlong_as_double(static_cast<long long>(1023 - F) << 52);
-            ap->s2f = finite ? s2f : __longlong_as_double(0x7FF8000000000000LL);
-            // the fp64 sum of 256 terms is within 2^-44 of the exact one
-            ap->R = finite ? __double2float_ru(res * (1.0 + 0x1p-40) * s2f) : 0.f;
-            ap->nl = three ? 3 : 4;
+            const double s2f = __longlong_as_double(static_cast<long long>(1023 - F[k]) << 52);
+            ap->s2f = finite[k] ? s2f : __longlong_as_double(0x7FF8000000000000LL);
+            // the fp32 sum of 256 terms (a tree eight deep) is within 2^-20 of
+            // the exact one: 2^-16 more keeps R an upper bound
+            ap->R = finite[k] ? __double2float_ru(static_cast<double>(res[k]) * (1.0 + 0x1p-16) * s2f) : 0.f;
+            ap->nl = three[k] ? 3 : 4;
         }
     }
 }
 
 // Stages super-blocks kb_begin .. kb_begin + nbs - 1: this warp's first
-// kFxStagePre from the registers fx_stage_load filled, the rest loaded here.
+// kFxStagePre (= 2, together) from the registers fx_stage_load filled, the
+// rest loaded here.
 template <bool COHERENT = false>
 __device__ __forceinline__ void fx_stage(const float *x, int kb_begin, int nbs, uint8_t *limbs, uint8_t *aux,
                                          int warp, int nwarps, int lane, const FxXPre &pre, bool allow3)
 {
-#pragma unroll
-    for (int k = 0; k < kFxStagePre; ++k) {
-        const int sb = warp + k * nwarps;
-        if (sb < nbs)
-            fx_stage_one(sb, pre.a[k], pre.b[k], limbs, aux, lane, allow3);
+    static_assert(kFxStagePre == 2, "the preloaded blocks are staged as a pair");
+    if (warp < nbs) {
+        const int sb[2] = {warp, warp + nwarps};
+        const bool valid[2] = {true, warp + nwarps < nbs};
+        if (valid[1]) {
+            fx_stage_blocks<2>(sb, pre.a, pre.b, valid, limbs, aux, lane, allow3);
+        } else {
+            const int sb1[1] = {warp};
+            const float4 a1[1] = {pre.a[0]}, b1[1] = {pre.b[0]};
+            const bool v1[1] = {true};
+            fx_stage_blocks<1>(sb1, a1, b1, v1, limbs, aux, lane, allow3);
+        }
     }
-    for (int sb = warp + kFxStagePre * nwarps; sb < nbs; sb += nwarps) {
-        const float *xg = x + static_cast<long long>(kb_begin + sb) * 256 + lane * 8;
-        fx_stage_one(sb, fx_ld4<COHERENT>(xg), fx_ld4<COHERENT>(xg + 4), limbs, aux, lane, allow3);
+    for (int s = warp + kFxStagePre * nwarps; s < nbs; s += nwarps) {
+        const float *xg = x + static_cast<long long>(kb_begin + s) * 256 + lane * 8;
+        const int sb1[1] = {s};
+        const float4 a1[1] = {fx_ld4<COHERENT>(xg)}, b1[1] = {fx_ld4<COHERENT>(xg + 4)};
+        const bool v1[1] = {true};
+        fx_stage_blocks<1>(sb1, a1, b1, v1, limbs, aux, lane, allow3);
     }
 }
 
@@ -308,7 +381,7 @@ __device__ __forceinline__ void fx_block_sums(const uint8_t *slot_row, BlockOffs
 }
 
 // One slot (a K-chunk of kFxBPC super-blocks of one row tile) for this lane:
-// super-block g of the chunk, rows i and i + 8 (R = 2).  slot is the slot's
+// super-block g of the chunk, slot rows i + 8r (r < R).  slot is the slot's
 // shared memory, limbs/aux point at the staged activations of the chunk's first
 // super-block, nblk is the chunk's super-block count.  Adds each row's partial
 // y_sb = 2^-F (d I_s - dmin I_m) (fp64), its error bound and |y_sb|.
@@ -394,18 +467,25 @@ __device__ __forceinline__ void fx_slot(const uint8_t *slot, const uint8_t *limb
     }
 }
 
-// Adds the four quarter-warps' row sums (and their bounds, rounded outwards):
-// afterwards lanes of quarters 0, 1 hold row i and quarters 2, 3 row i + 8.
+// Adds the four quarter-warps' row sums (and their bounds, rounded outwards).
+// R = 2: afterwards lanes of quarters 0, 1 hold row i and quarters 2, 3 row
+// i + 8.  R = 1: every quarter holds the sums of its lanes' row.
 template <int R>
 __device__ __forceinline__ void fx_quarter_rows(double (&acc)[R], float (&ebound)[R], float (&sabs)[R], int lane,
                                                 double &t, float &te, float &ts)
 {
-    const bool up = (lane & 16) != 0;
-    t = (up ? acc[1] : acc[0]) + __shfl_xor_sync(0xffffffffu, up ? acc[0] : acc[1], 16);
+    if constexpr (R == 2) {
+        const bool up = (lane & 16) != 0;
+        t = (up ? acc[1] : acc[0]) + __shfl_xor_sync(0xffffffffu, up ? acc[0] : acc[1], 16);
+        te = __fadd_ru(up ? ebound[1] : ebound[0], __shfl_xor_sync(0xffffffffu, up ? ebound[0] : ebound[1], 16));
+        ts = __fadd_rd(up ? sabs[1] : sabs[0], __shfl_xor_sync(0xffffffffu, up ? sabs[0] : sabs[1], 16));
+    } else {
+        t = acc[0] + __shfl_xor_sync(0xffffffffu, acc[0], 16);
+        te = __fadd_ru(ebound[0], __shfl_xor_sync(0xffffffffu, ebound[0], 16));
+        ts = __fadd_rd(sabs[0], __shfl_xor_sync(0xffffffffu, sabs[0], 16));
+    }
     t += __shfl_xor_sync(0xffffffffu, t, 8);
-    te = __fadd_ru(up ? ebound[1] : ebound[0], __shfl_xor_sync(0xffffffffu, up ? ebound[0] : ebound[1], 16));
     te = __fadd_ru(te, __shfl_xor_sync(0xffffffffu, te, 8));
-    ts = __fadd_rd(up ? sabs[1] : sabs[0], __shfl_xor_sync(0xffffffffu, up ? sabs[0] : sabs[1], 16));
     ts = __fadd_rd(ts, __shfl_xor_sync(0xffffffffu, ts, 8));
 #pragma unroll
     for (int r = 0; r < R; ++r) {

@@ -97,11 +97,13 @@ __device__ __forceinline__ void fx_issue_copy(const Q4KParams &p, const FxMaps &
                 return;
             const CUtensorMap *m = fr.sel == 0 ? &maps.m[0] : fr.sel == 1 ? &maps.m[1] : fr.sel == 2 ? &maps.m[2]
                                                                                                       : &maps.m[3];
-            // x = kb0 * 36 words: a multiple of 4 words, i.e. of 16 bytes
+            // x = kb0 * 36 words: a multiple of 4 words, i.e. of 16 bytes.  The
+            // weights are read once: first out of L2
             asm volatile(
-                "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-                "[%4];" ::"r"(dst),
-                "l"(m), "r"(kb0 * (kQ4KBlockBytes / 4)), "r"(static_cast<int>(fr.row0)), "r"(bar)
+                "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], "
+                "[%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+                "l"(m), "r"(kb0 * (kQ4KBlockBytes / 4)), "r"(static_cast<int>(fr.row0)), "r"(bar),
+                "l"(l2_evict_first_policy())
                 : "memory");
         }
     } else {
@@ -115,7 +117,7 @@ __device__ __forceinline__ void fx_issue_copy(const Q4KParams &p, const FxMaps &
         if (lane < rows && !lost) {
             const uint8_t *src = fx_weights(p, fr.sel) + (fr.row0 + lane) * row_bytes_g +
                                  static_cast<long long>(kb0) * kQ4KBlockBytes;
-            bulk_g2s(dst + lane * kFxRowPitch, src, bytes, bar);
+            bulk_g2s_hint(dst + lane * kFxRowPitch, src, bytes, bar, l2_evict_first_policy());
         }
     }
 }
@@ -131,19 +133,27 @@ __device__ __forceinline__ void fx_issue_slot(const Q4KParams &p, const FxMaps &
                        bars_s + slot * 8, lane, lost);
 }
 
-template <int NS, bool SOA, bool TMA>
-__global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
+// R = 2: every warp owns a ring and its tiles.  R = 1: warps 2t and 2t + 1 own
+// ring t and its tiles together, warp 2t + h reading rows 8h .. 8h + 7 of each
+// slot; a counter per slot tells the second of the two to finish it, which
+// refills it.
+template <int NS, bool SOA, bool TMA, int R>
+__global__ void __launch_bounds__((R == 2 ? kFxMaxWarps : kFxMaxPairWarps) * 32, 1)
     q4k_gemv_fx_kernel(const __grid_constant__ Q4KParams p, const __grid_constant__ FxMaps maps)
 {
-    constexpr int R = kFxRows;
-    static_assert(R == 2, "the quarter reduction below is written for two rows per lane");
+    static_assert(R == 1 || R == 2, "one or two rows per lane");
+    constexpr int kTeam = 3 - R;   // warps per ring
 
     extern __shared__ __align__(128) uint8_t smem[];
     const int nwarps = blockDim.x >> 5;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int g = lane >> 3;   // super-block of each chunk
-    const int i = lane & 7;    // rows i and i + 8 of each tile
+    const int nteams = nwarps / kTeam;
+    const int team = warp / kTeam;
+    const int half = warp % kTeam;       // R = 1: rows 8 half .. 8 half + 7 of each slot
+    const int g = lane >> 3;             // super-block of each chunk
+    const int i = lane & 7;
+    const int srow = i + 8 * half;       // this lane's (first) row of each slot: rows srow + 8r, r < R
 
     // the splits of one CTA column are consecutive blocks (one cluster when the
     // splits are reduced in-kernel)
@@ -157,7 +167,10 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
     const int nbs = min(nch * kFxBPC, p.nb - kb_begin);  // super-blocks of this split
 
     // shared memory: [limb planes][sums and scales][barriers][ring][argmax scratch]
-    const int x_bytes = (nbs * (kFxLimbPitch + kFxAuxPitch) + 127) & ~127;
+    // [cluster scratch], laid out for a full split in every CTA, so that each
+    // part sits at the same offset in all CTAs of a cluster (a shorter last
+    // split stages fewer super-blocks)
+    const int x_bytes = (p.chunks_per_split * kFxBPC * (kFxLimbPitch + kFxAuxPitch) + 127) & ~127;
     uint8_t *limbs = smem;
     uint8_t *aux = smem + nbs * kFxLimbPitch;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + x_bytes);
@@ -165,32 +178,43 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
     // TMA writes shared memory at 128-byte aligned addresses: align the ring
     const uint32_t ring_pad = (128u - ((smem_u32(smem) + x_bytes + bar_bytes) & 127u)) & 127u;
     uint8_t *ring = smem + x_bytes + bar_bytes + ring_pad;
-    uint8_t *my_ring = ring + static_cast<size_t>(warp) * p.depth * kFxSlotBytes;
+    uint8_t *my_ring = ring + static_cast<size_t>(team) * p.depth * kFxSlotBytes;
     const uint32_t my_ring_s = smem_u32(my_ring);
-    const uint32_t my_bars_s = smem_u32(bars + warp * p.depth);
-    ArgmaxCand *red = reinterpret_cast<ArgmaxCand *>(ring + static_cast<size_t>(nwarps) * p.depth * kFxSlotBytes);
-    // cluster reduction scratch: per warp, stream and tile row the fp64 partial
-    // sum, then its (error bound, sum of |y_sb|)
+    const uint32_t my_bars_s = smem_u32(bars + team * p.depth);
+    // R = 1: per slot, how many times a warp of the pair has finished it (after the barriers)
+    const uint32_t my_cnt_s = smem_u32(bars + nteams * p.depth) + team * p.depth * 4;
+    ArgmaxCand *red = reinterpret_cast<ArgmaxCand *>(ring + static_cast<size_t>(nteams) * p.depth * kFxSlotBytes);
+    // cluster reduction scratch of the rings this CTA finishes (ring t is
+    // finished by rank t % splits, as its local ring t / splits): per local ring,
+    // stream, source rank and tile row the fp64 partial sum, then its (error
+    // bound, sum of |y_sb|)
+    const int cl_rings = (nteams + p.splits - 1) / p.splits;
     double *cpart = reinterpret_cast<double *>(reinterpret_cast<uint8_t *>(red) + 256);
-    float2 *cbnd = reinterpret_cast<float2 *>(cpart + nwarps * 2 * kFxTileRows);
+    float2 *cbnd = reinterpret_cast<float2 *>(cpart + cl_rings * 2 * p.splits * kFxTileRows);
+    if (p.cluster)   // first phase of the cluster barrier: this CTA has started
+        asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 
-    // this warp's tiles: t0, t0 + tstride, ... (warp-major order)
-    const long long tstride = static_cast<long long>(p.ctas_per_split) * nwarps;
-    const long long t0 = static_cast<long long>(warp) * p.ctas_per_split + cj;
+    // this ring's tiles: t0, t0 + tstride, ... (ring-major order)
+    const long long tstride = static_cast<long long>(p.ctas_per_split) * nteams;
+    const long long t0 = static_cast<long long>(team) * p.ctas_per_split + cj;
     const long long ntiles_w = (t0 < p.tiles) ? (p.tiles - t0 + tstride - 1) / tstride : 0;
     const long long total = ntiles_w * NS * nch;
     const long long row_step = tstride * kFxTileRows;
 
-    // after the quarter reduction lanes of quarters 0, 1 hold row i and
-    // quarters 2, 3 row i + 8; quarters 0 and 2 store
-    const bool writer = (lane & 8) == 0;
-    const int wrow = i + ((lane & 16) ? 8 : 0);
+    // after the quarter reduction (R = 2) lanes of quarters 0, 1 hold row i and
+    // quarters 2, 3 row i + 8, and quarters 0 and 2 store; (R = 1) every
+    // quarter holds row srow, and quarter 0 stores
+    const bool writer = (R == 2) ? (lane & 8) == 0 : lane < 8;
+    const int wrow = (R == 2) ? i + ((lane & 16) ? 8 : 0) : srow;
 
     Cursor pc{t0 * kFxTileRows, 0, 0};
     long long issued = 0;
-    if (lane == 0) {
-        for (int s = 0; s < p.depth; ++s)
+    if (lane == 0 && half == 0) {
+        for (int s = 0; s < p.depth; ++s) {
             mbar_init(my_bars_s + s * 8, 1);
+            if (R == 1)
+                st_shared_u32(my_cnt_s + s * 4, 0u);
+        }
         mbar_fence_init();
         if (TMA && warp < (p.grp.n > 0 ? p.grp.n : NS))
             asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.m[warp]) : "memory");
@@ -203,16 +227,19 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
     fx_stage_load(p.x, kb_begin, nbs, warp, nwarps, lane, pre);
     // only the first slots before staging: the activation loads are not to
     // wait behind every SM's full ring of weight requests
+    // (R = 1: the first warp of the pair issues, both follow the cursor)
     for (int s = 0; s < min(p.depth, kFxPreIssue) && issued < total; ++s, ++issued) {
         const bool lost = p.lost_copy && s == 0 && warp == 0 && blockIdx.x == 0;
-        fx_issue_slot<TMA>(p, maps, pc, s, c_begin, my_ring_s, my_bars_s, lane, lost);
+        if (half == 0)
+            fx_issue_slot<TMA>(p, maps, pc, s, c_begin, my_ring_s, my_bars_s, lane, lost);
         pc.advance(nch, NS, row_step);
     }
 
     fx_stage(p.x, kb_begin, nbs, limbs, aux, warp, nwarps, lane, pre, p.nb >= kFxMin3LimbBlocks);
     for (int s = static_cast<int>(issued); s < p.depth && issued < total; ++s, ++issued) {
         const bool lost = p.lost_copy && s == 0 && warp == 0 && blockIdx.x == 0;
-        fx_issue_slot<TMA>(p, maps, pc, s, c_begin, my_ring_s, my_bars_s, lane, lost);
+        if (half == 0)
+            fx_issue_slot<TMA>(p, maps, pc, s, c_begin, my_ring_s, my_bars_s, lane, lost);
         pc.advance(nch, NS, row_step);
     }
     __syncthreads();
@@ -231,6 +258,8 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
     }
     double gsum = 0.0;  // stream-0 sum kept for the SwiGLU epilogue
     float gE = 0.f, gS = 0.f;
+    double csum = 0.0;  // cluster mode: the last stream's sum of the ring's one tile
+    float cE = 0.f, cS = 0.f;
 
     Cursor cc{t0 * kFxTileRows, 0, 0};
     int slot = 0;
@@ -244,13 +273,21 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
         const int kb0 = (c_begin + cc.kcl) * kFxBPC;
         const int nblk = min(kFxBPC, p.nb - kb0);
         fx_slot<R, SOA>(my_ring + slot * kFxSlotBytes, limbs + (kb0 - kb_begin) * kFxLimbPitch,
-                        aux + (kb0 - kb_begin) * kFxAuxPitch, nblk, g, i, acc, ebound, sabs);
+                        aux + (kb0 - kb_begin) * kFxAuxPitch, nblk, g, srow, acc, ebound, sabs);
 
         // every lane's reads of this slot are done (their values are used):
-        // the slot may be refilled
+        // the slot may be refilled (R = 1: once both warps of the pair are done)
         __syncwarp();
         if (issued < total) {
-            fx_issue_slot<TMA>(p, maps, pc, slot, c_begin, my_ring_s, my_bars_s, lane);
+            bool refill = true;
+            if constexpr (R == 1) {
+                uint32_t done = 0;
+                if (lane == 0)
+                    done = atom_add_acq_rel_shared_u32(my_cnt_s + slot * 4, 1u);
+                refill = (__shfl_sync(0xffffffffu, done, 0) & 1u) != 0;
+            }
+            if (refill)
+                fx_issue_slot<TMA>(p, maps, pc, slot, c_begin, my_ring_s, my_bars_s, lane);
             pc.advance(nch, NS, row_step);
             ++issued;
         }
@@ -280,13 +317,10 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
         }
         const long long n = row0 + wrow;
         if (p.cluster) {
-            // this warp's only tile: keep its partials for the cluster reduction
-            if (writer) {
-                cpart[(warp * 2 + 0) * kFxTileRows + wrow] = (NS == 2) ? gsum : t;
-                cpart[(warp * 2 + 1) * kFxTileRows + wrow] = t;
-                cbnd[(warp * 2 + 0) * kFxTileRows + wrow] = (NS == 2) ? make_float2(gE, gS) : make_float2(te, ts);
-                cbnd[(warp * 2 + 1) * kFxTileRows + wrow] = make_float2(te, ts);
-            }
+            // the ring's only tile: its partials go to the cluster reduction
+            csum = t;
+            cE = te;
+            cS = ts;
             continue;
         }
         if (p.splits > 1) {
@@ -350,46 +384,49 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
     }
 
     if (p.cluster) {
-        // Splits of a CTA column are one cluster and their warps hold the same
-        // tiles: each tile is finished by the CTA whose rank is the warp index
-        // modulo the split count, adding the partials of ranks 0, 1, ... in order.
+        // Splits of a CTA column are one cluster and their rings hold the same
+        // tiles: ring t's tile is finished (by the ring's first warp) in the CTA
+        // of rank t % splits.  Every CTA stores its partials into that CTA's
+        // shared memory, one cluster barrier makes them visible there, and the
+        // finishing warp adds them in rank order 0, 1, ...
         namespace cg = cooperative_groups;
         cg::cluster_group cl = cg::this_cluster();
+        // every CTA of the cluster has started (the first phase), so its shared
+        // memory may be written
+        asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+        const int fin = team % p.splits;
+        const int lt = team / p.splits;
+        if (writer && t0 < p.tiles && !failed) {
+            double *rp = cl.map_shared_rank(cpart, fin);
+            float2 *rb = cl.map_shared_rank(cbnd, fin);
+            const int e0 = ((lt * 2 + 0) * p.splits + split) * kFxTileRows + wrow;
+            rp[e0] = (NS == 2) ? gsum : csum;
+            rb[e0] = (NS == 2) ? make_float2(gE, gS) : make_float2(cE, cS);
+            if (NS == 2) {
+                const int e1 = ((lt * 2 + 1) * p.splits + split) * kFxTileRows + wrow;
+                rp[e1] = csum;
+                rb[e1] = make_float2(cE, cS);
+            }
+        }
         cl.sync();
-        if (warp % p.splits == split && t0 < p.tiles) {
+        if (fin == split && half == 0 && t0 < p.tiles) {
             // lane r < 16 finishes row r of the tile: partial sums in fp64, bounds
             // rounded outwards, in rank order
             double g = 0.0, u = 0.0;
             float ge = 0.f, gs = 0.f, ue = 0.f, us = 0.f;
             const int lr = lane & (kFxTileRows - 1);
-            // all remote loads first (each is a round trip to another SM), then
-            // the sums in rank order
-            double pg[kFxMaxCluster], pu[kFxMaxCluster];
-            float2 bg[kFxMaxCluster], bu[kFxMaxCluster];
-#pragma unroll
-            for (int r = 0; r < kFxMaxCluster; ++r) {
-                if (r < p.splits) {
-                    const double *rp = cl.map_shared_rank(cpart, r);
-                    const float2 *rb = cl.map_shared_rank(cbnd, r);
-                    pg[r] = rp[(warp * 2 + 0) * kFxTileRows + lr];
-                    bg[r] = rb[(warp * 2 + 0) * kFxTileRows + lr];
-                    if (NS == 2) {
-                        pu[r] = rp[(warp * 2 + 1) * kFxTileRows + lr];
-                        bu[r] = rb[(warp * 2 + 1) * kFxTileRows + lr];
-                    }
-                }
-            }
-#pragma unroll
-            for (int r = 0; r < kFxMaxCluster; ++r) {
-                if (r < p.splits) {
-                    g += pg[r];
-                    ge = __fadd_ru(ge, bg[r].x);
-                    gs = __fadd_rd(gs, bg[r].y);
-                    if (NS == 2) {
-                        u += pu[r];
-                        ue = __fadd_ru(ue, bu[r].x);
-                        us = __fadd_rd(us, bu[r].y);
-                    }
+            for (int r = 0; r < p.splits; ++r) {
+                const int e0 = ((lt * 2 + 0) * p.splits + r) * kFxTileRows + lr;
+                const float2 b0 = cbnd[e0];
+                g += cpart[e0];
+                ge = __fadd_ru(ge, b0.x);
+                gs = __fadd_rd(gs, b0.y);
+                if (NS == 2) {
+                    const int e1 = ((lt * 2 + 1) * p.splits + r) * kFxTileRows + lr;
+                    const float2 b1 = cbnd[e1];
+                    u += cpart[e1];
+                    ue = __fadd_ru(ue, b1.x);
+                    us = __fadd_rd(us, b1.y);
                 }
             }
             const long long n = t0 * kFxTileRows + lane;
@@ -419,7 +456,6 @@ __global__ void __launch_bounds__(kFxMaxWarps * 32, 1)
                 }
             }
         }
-        cl.sync();  // no CTA leaves while another reads its shared memory
     }
 
     if (p.argmax && (p.splits == 1 || p.cluster)) {
@@ -734,18 +770,18 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 }
 
 // How many clusters of `size` CTAs of the batch-1 kernel (warps x 32 threads,
-// smem bytes of shared memory each) the device runs at once; 0 when the runtime
-// cannot tell.  Cached per shape.
-static int cluster_capacity(int size, int warps, int smem)
+// smem bytes of shared memory each, R rows per lane) the device runs at once; 0
+// when the runtime cannot tell.  Cached per shape.
+static int cluster_capacity(int size, int warps, int smem, int R)
 {
     static std::mutex mu;
-    static std::map<std::tuple<int, int, int>, int> cache;
-    const auto key = std::make_tuple(size, warps, smem);
+    static std::map<std::tuple<int, int, int, int>, int> cache;
+    const auto key = std::make_tuple(size, warps, smem, R);
     std::lock_guard<std::mutex> lock(mu);
     const auto it = cache.find(key);
     if (it != cache.end())
         return it->second;
-    auto k = q4k_gemv_fx_kernel<1, false, true>;
+    auto k = R == 1 ? q4k_gemv_fx_kernel<1, false, true, 1> : q4k_gemv_fx_kernel<1, false, true, 2>;
     int n = 0;
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess) {
         cudaLaunchConfig_t cfg = {};
@@ -775,7 +811,9 @@ static int cluster_capacity(int size, int warps, int smem)
 // is as deep as shared memory allows, up to 4 slots.  When the batch-1 splits
 // are added inside clusters, all clusters must be resident at once: the plan
 // then takes the fewest warps per CTA (the most CTAs, hence SMs) whose clusters
-// fit in one wave, and gives up the clusters if none does.
+// fit in one wave, and gives up the clusters if none does.  At batch 1, rings
+// that would hold at most kFxPairMaxSlots slots are owned by pairs of warps
+// (R = 1), when the CTA has room for twice the warps.
 static Q4KPlan plan_quarter_warp(long long N, int nb, int B, int NS, int sm_count, int smem_optin)
 {
     // DQGEMV_NO_TMA=1 selects the per-row bulk copies (same shared-memory
@@ -815,22 +853,28 @@ static Q4KPlan plan_quarter_warp(long long N, int nb, int B, int NS, int sm_coun
         const long long max_ctas = sm_count / splits > 0 ? sm_count / splits : 1;
         if (ctas > max_ctas)
             ctas = max_ctas;
+        // `warps` rings; each owned by two warps when it holds few slots
+        const long long ring_slots = (tiles + ctas * warps - 1) / (ctas * warps) * NS * cps;
+        const int team = (B == 1 && 2 * warps <= kFxMaxPairWarps && ring_slots <= kFxPairMaxSlots) ? 2 : 1;
         pl.tma = tma;
-        pl.R = kFxRows;
-        pl.warps = warps;
+        pl.R = team == 2 ? 1 : kFxRows;
+        pl.warps = warps * team;
         pl.tiles = tiles;
         pl.splits = splits;
         pl.chunks_per_split = cps;
         pl.depth = depth;
         pl.ctas_per_split = static_cast<int>(ctas);
         pl.grid = pl.ctas_per_split * splits;
-        pl.smem = x_bytes + ((warps * depth * 8 + 127) & ~127) + 128 + warps * depth * kFxSlotBytes + 256;
+        // barriers (and R = 1 refill counters) are sized for 8 bytes per warp and slot
+        pl.smem = x_bytes + ((pl.warps * depth * 8 + 127) & ~127) + 128 + warps * depth * kFxSlotBytes + 256;
         // batch-1 splits of at most one tile per warp are added inside a cluster
+        // (each CTA finishes the tiles of every splits-th ring and holds the
+        // partials of all splits for them)
+        const int cl_bytes = (warps + splits - 1) / splits * splits * kFxClusterPartBytes;
         pl.cluster = allow_cluster && B == 1 && splits > 1 && splits <= kFxMaxCluster &&
-                     tiles <= static_cast<long long>(pl.ctas_per_split) * warps &&
-                     pl.smem + warps * kFxClusterPartBytes <= smem_optin;
+                     tiles <= static_cast<long long>(pl.ctas_per_split) * warps && pl.smem + cl_bytes <= smem_optin;
         if (pl.cluster)
-            pl.smem += warps * kFxClusterPartBytes;
+            pl.smem += cl_bytes;
         pl.ok = pl.smem <= smem_optin;
         return pl;
     };
@@ -858,11 +902,11 @@ static Q4KPlan plan_quarter_warp(long long N, int nb, int B, int NS, int sm_coun
     };
     Q4KPlan pl = first_fit(true);
     if (pl.ok && pl.cluster) {
-        const int cap = cluster_capacity(pl.splits, pl.warps, pl.smem);
+        const int cap = cluster_capacity(pl.splits, pl.warps, pl.smem, pl.R);
         if (cap > 0) {
             for (int warps = 4; warps <= max_warps; ++warps) {
                 const Q4KPlan c = plan_for(warps, true);
-                if (c.ok && c.cluster && c.ctas_per_split <= cluster_capacity(c.splits, c.warps, c.smem))
+                if (c.ok && c.cluster && c.ctas_per_split <= cluster_capacity(c.splits, c.warps, c.smem, c.R))
                     return c;
             }
             if (pl.ctas_per_split > cap)
@@ -890,7 +934,8 @@ static cudaError_t encode_weight_map(CUtensorMap *m, const uint8_t *w, long long
 template <int NS, bool TMA>
 static cudaError_t launch_fx(const Q4KParams &p, const FxMaps &maps, const Q4KPlan &pl, cudaStream_t s)
 {
-    auto k = p.soa ? q4k_gemv_fx_kernel<NS, true, TMA> : q4k_gemv_fx_kernel<NS, false, TMA>;
+    auto k = pl.R == 1 ? (p.soa ? q4k_gemv_fx_kernel<NS, true, TMA, 1> : q4k_gemv_fx_kernel<NS, false, TMA, 1>)
+                       : (p.soa ? q4k_gemv_fx_kernel<NS, true, TMA, 2> : q4k_gemv_fx_kernel<NS, false, TMA, 2>);
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
     if (e != cudaSuccess)
         return e;

@@ -190,7 +190,9 @@ def test_q4k_lm_head_248320x4096_with_argmax():
 # --- edge cases -----------------------------------------------------------------------------
 
 @pytest.mark.parametrize("N,K,B", [(1, 256, 1), (5, 256, 3), (17, 1024, 1), (4097, 1024, 2), (33, 5120, 1),
-                                   (9, 12288, 5), (130, 4096, 7), (3, 768, 8), (64, 65536, 1), (16, 262144, 2)])
+                                   (9, 12288, 5), (130, 4096, 7), (3, 768, 8), (64, 65536, 1), (16, 262144, 2),
+                                   # K split unevenly (2 + 1 chunks) inside clusters of two CTAs
+                                   (9728, 2560, 1)])
 @pytest.mark.parametrize("layout", ["aos", "soa"])
 def test_q4k_gemv_ragged_and_split_shapes(N, K, B, layout):
     rng = np.random.default_rng(N * 7 + K + B)
