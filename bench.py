@@ -61,13 +61,15 @@ NOMINAL_HBM_GBS = 8000.0   # B200 HBM3e, nominal
 
 # DRAM bytes (read + write) per launch of q4k_gemv_fx_kernel, from one ncu
 # capture per workload, valid only for the kernel sources whose hash is recorded.
-NCU_TRAFFIC = {"sources_sha1": "97e73226d35cc0a24934390a6c594a86437ad853",
-               "bytes_per_launch": {"q4k_lmhead_248320x4096": 572207616 + 4335872}}
+NCU_TRAFFIC = {"sources_sha1": "4aeb0b3924fb4e8ffb6faa31e154a8d4f969214f",
+               "bytes_per_launch": {"q4k_lmhead_248320x4096": 572227584 + 3427072,
+                                    "q4k_down_4096x12288": 28427776 + 0,
+                                    "q4k_swiglu_12288x4096": 56720640 + 9472}}
 
 
 def kernel_sources_sha1() -> str:
     h = hashlib.sha1()
-    for f in ("q4k_gemv.cu", "q4k_stream.cuh", "dq_common.cuh"):
+    for f in ("q4k_gemv.cu", "q4k_fx.cuh", "q4k_exact.cuh", "q4k_stream.cuh", "dq_common.cuh"):
         with open(os.path.join(ROOT, "dequant_gemv_q4_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
