@@ -67,6 +67,7 @@ constexpr int kPfDqWarp0 = 4;                             // first dequantizing 
 constexpr int kPfDqWarps = kPfWarps - kPfDqWarp0;
 constexpr int kPfMaxRaw = 4;                              // raw weight ring, super-blocks
 constexpr int kPfMaxStages = 4;                           // operand ring, stages
+constexpr int kPfEpiPitch = kPfRows + 4;                  // epilogue tile: floats per token row
 
 struct PrefillMaps {
     CUtensorMap w;        // raw weight rows (AoS: 2-D bytes; SoA: 5-D gather of one block)
@@ -308,6 +309,7 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1)
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
+    __shared__ int s_epi_bad;   // a dequantizing warp saw an abort before the epilogue
     __shared__ int s_go[4];
     __shared__ __align__(8) uint64_t s_bars[2 * (kPfMaxRaw + kPfMaxStages) + 1];
 
@@ -351,6 +353,7 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1)
         }
         mbar_init(acc_full, 1);
         s_abort = 0;
+        s_epi_bad = 0;
         mbar_fence_init();
     }
     if (warp == 1) {
@@ -524,34 +527,57 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1)
             rr.next();
         }
 
-        // ---- epilogue: warp (q = warp % 4, e = d / 4) reads accumulator lanes 32q .. 32q+31 (tokens)
-        // and columns 64e .. 64e+63 (weight rows) of each accumulator
+        // ---- epilogue, per accumulator: warp (q = warp % 4, e = d / 4) reads accumulator lanes
+        // 32q .. 32q+31 (tokens) and columns 64e .. 64e+63 (weight rows) into a token-major tile in
+        // the now idle rings (rows of 256 floats at a 260-float pitch); then warp d stores tokens
+        // d, d + 16, ...: each token's 256 outputs are one contiguous run of Y (or of the split's
+        // partial sums), written 512 bytes per instruction.  Every dequantizing warp passes both
+        // named barriers; if any of them saw an abort, nothing is stored.
         const bool done = pf_wait_warp(acc_full, 0, p.err, nullptr);
         pf_fence_after();
         // tcgen05.ld is warp-collective: the whole warp reads, or none of it
-        if (__all_sync(0xFFFFFFFFu, done && !*abort)) {
-            const int q = warp & 3;
-            const int e = d >> 2;
-            float *out = p.out + static_cast<long long>(split) * p.M * p.N;
-            const bool vec = (p.N & 3) == 0;
-            for (int t = 0; t < TH; ++t) {
-                const long long m = m0 + t * kPfTok + 32 * q + lane;
+        const bool ok_w = __all_sync(0xFFFFFFFFu, done && !*abort);
+        if (!ok_w && lane == 0)
+            s_epi_bad = 1;
+        const int q = warp & 3;
+        const int e = d >> 2;
+        float *out = p.out + static_cast<long long>(split) * p.M * p.N;
+        const bool vec = (p.N & 3) == 0;
+        float *tile = reinterpret_cast<float *>(smem + (st_s - smem_u32(smem)));
+        for (int t = 0; t < TH; ++t) {
+            if (ok_w) {
+                float *trow = tile + (32 * q + lane) * kPfEpiPitch;
                 for (int c0 = 64 * e; c0 < 64 * e + 64; c0 += 8) {
                     float v[8];
                     pf_tmem_ld8(tmem + (static_cast<uint32_t>(32 * q) << 16) + t * kPfRows + c0, v);
-                    const long long n = row0 + c0;
-                    if (m >= p.M || n >= p.N)
-                        continue;
-                    float *o = out + m * p.N + n;
-                    if (vec && n + 8 <= p.N) {
-                        reinterpret_cast<float4 *>(o)[0] = make_float4(v[0], v[1], v[2], v[3]);
-                        reinterpret_cast<float4 *>(o)[1] = make_float4(v[4], v[5], v[6], v[7]);
-                    } else {
-                        for (int u = 0; u < 8 && n + u < p.N; ++u)
-                            o[u] = v[u];
+                    reinterpret_cast<float4 *>(trow + c0)[0] = make_float4(v[0], v[1], v[2], v[3]);
+                    reinterpret_cast<float4 *>(trow + c0)[1] = make_float4(v[4], v[5], v[6], v[7]);
+                }
+            }
+            asm volatile("bar.sync 3, %0;" ::"n"(kPfDqWarps * 32) : "memory");
+            if (!s_epi_bad) {
+                for (int mm = d; mm < kPfTok; mm += kPfDqWarps) {
+                    const long long m = m0 + t * kPfTok + mm;
+                    if (m >= p.M)
+                        break;
+                    const float *trow = tile + mm * kPfEpiPitch;
+                    float *o = out + m * p.N + row0;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int c = 128 * h + 4 * lane;
+                        const float4 v = reinterpret_cast<const float4 *>(trow + c)[0];
+                        if (vec && row0 + c + 4 <= p.N) {
+                            reinterpret_cast<float4 *>(o + c)[0] = v;
+                        } else {
+                            const float vv[4] = {v.x, v.y, v.z, v.w};
+                            for (int u = 0; u < 4 && row0 + c + u < p.N; ++u)
+                                o[c + u] = vv[u];
+                        }
                     }
                 }
             }
+            // the tile is rewritten by the next accumulator only after every warp has stored it
+            asm volatile("bar.sync 3, %0;" ::"n"(kPfDqWarps * 32) : "memory");
         }
     }
 
@@ -645,6 +671,9 @@ PrefillPlan q4k_prefill_plan(long long N, int K, long long M, int sm_count, int 
     int rd = (budget - depth * stage) / kPfRawBytes;
     if (rd > kPfMaxRaw)
         rd = kPfMaxRaw;
+    // the epilogue stages one accumulator as a token-major tile in the rings
+    if (depth * stage + rd * kPfRawBytes < kPfTok * kPfEpiPitch * 4)
+        return pl;
     pl.th = th;
     pl.mtiles = static_cast<int>(mtiles);
     pl.ntiles = static_cast<int>(ntiles);
